@@ -1,0 +1,185 @@
+"""CPU oracle for KVpop future-attention targets.  TEST INFRASTRUCTURE ONLY.
+
+Only the tests, the package's ``smoke()`` check and ``bench.py``'s CPU
+baseline may import this module.  The CUDA library never calls it, and it
+shares no code, constants or helpers with the CUDA path.
+
+It is the plain definition written out in float64, with an explicitly
+materialised causal softmax (one block of query rows at a time):
+
+* Row logsumexp.  For query head g and query position i of a sequence,
+  ``lse[g, i] = log sum_{j <= i} exp(s * q_{g,i} . k_{h(g),j})`` with the
+  causal mask (attention from a query only to itself and earlier keys) and
+  the GQA mapping ``h(g) = g // G``, ``G = H_q / H_kv``.
+* Future-attention target (KVpop paper summary; the aiweekly article
+  "KVpop shrinks Qwen3 KV cache 88%", second paragraph; its French
+  edition, second paragraph).  The target of key j is the attention mass it
+  receives from queries that come after it has left the protected recent
+  window of W positions.  At query i the window holds positions
+  i-W+1 .. i, so key j has left it exactly when i >= j + W.  The mass is
+  the softmax probability ``A[i, j] = exp(S[i, j] - lse[i])`` and the
+  target of a KV head is summed over the G query heads that share it:
+  ``target[h, j] = sum_{g in group(h)} sum_{i = j+W}^{L-1} A_g[i, j]``.
+* Keep mask (KVpop model card, intro: "a bounded sink + scored top-k +
+  recent-window cache", 4,032 = 4 sink + 3,772 scored + 256 recent; the
+  French article, second paragraph: sinks + protected recent window +
+  learned top-k over the older tokens).  Per sequence and KV head: keep
+  p < S (sinks), keep p >= L - W (recent window), and among p in [S, L-W)
+  keep the k = budget - S - W largest scores; equal scores go to the
+  smaller position first.  Everything is kept when L <= budget.
+
+Readings taken where the pages are silent: the window condition is
+``i >= j + W``; the GQA group is summed (not averaged) with consecutive
+grouping ``g // G``; the softmax normaliser is the full causal row (sinks
+included); the target is the raw mass (no normalisation by the number of
+future queries); V is not used; ties in the keep set go to the smaller
+position; NaN scores rank below every number.
+
+Inputs may be bf16 bit patterns (uint16 arrays, converted exactly) or float
+arrays; the arithmetic is float64 throughout.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = ["as_f64", "row_lse", "future_target", "keep_mask", "ROW_BLOCK"]
+
+ROW_BLOCK = 256  # query rows materialised at once
+
+
+def as_f64(x: np.ndarray) -> np.ndarray:
+    """bf16 bits (uint16) -> exact float64; float arrays are widened as they are."""
+    x = np.asarray(x)
+    if x.dtype == np.uint16:
+        return (x.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    return x.astype(np.float64)
+
+
+def _sequences(cu_seqlens):
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    return [(int(cu[b]), int(cu[b + 1] - cu[b])) for b in range(len(cu) - 1)]
+
+
+def _softmax_rows(qg: np.ndarray, kh: np.ndarray, r0: int, r1: int, scale: float):
+    """Materialised causal softmax rows r0..r1-1 of one head of one sequence.
+
+    Returns (A, lse) with A[i - r0, j] for j < r1 (entries j > i are 0).
+    """
+    S = scale * (qg[r0:r1] @ kh[:r1].T)                       # [r1-r0, r1]
+    rows = np.arange(r0, r1)[:, None]
+    cols = np.arange(r1)[None, :]
+    S = np.where(cols <= rows, S, -np.inf)                      # causal mask
+    m = S.max(axis=1, keepdims=True)
+    P = np.exp(S - m)
+    Z = P.sum(axis=1, keepdims=True)
+    A = P / Z
+    lse = (m + np.log(Z))[:, 0]
+    return A, lse
+
+
+def row_lse(q, k, cu_seqlens, scale: float, rows=None) -> np.ndarray:
+    """Natural-log row logsumexp, float64 [H_q, T].
+
+    ``rows`` (optional, sorted int array of global positions) restricts the
+    computation to those query rows; other entries are NaN.
+    """
+    q, k = as_f64(q), as_f64(k)
+    T, Hq, _ = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    out = np.full((Hq, T), np.nan)
+    want = None if rows is None else np.zeros(T, dtype=bool)
+    if want is not None:
+        want[np.asarray(rows, dtype=np.int64)] = True
+    for s, L in _sequences(cu_seqlens):
+        for g in range(Hq):
+            qg, kh = q[s:s + L, g, :], k[s:s + L, g // G, :]
+            for r0 in range(0, L, ROW_BLOCK):
+                r1 = min(r0 + ROW_BLOCK, L)
+                if want is not None:
+                    sel = np.nonzero(want[s + r0:s + r1])[0]
+                    for i in sel + r0:                         # one row at a time
+                        _, l1 = _softmax_rows(qg, kh, int(i), int(i) + 1, scale)
+                        out[g, s + i] = l1[0]
+                    continue
+                _, lse = _softmax_rows(qg, kh, r0, r1, scale)
+                out[g, s + r0:s + r1] = lse
+    return out
+
+
+def future_target(q, k, cu_seqlens, window: int, scale: float, key_lo: int | None = None,
+                  return_lse: bool = False, return_far: bool = False):
+    """Future-attention target, float64 [H_kv, T].
+
+    ``key_lo`` (optional, a position relative to each sequence's start)
+    restricts the work to keys j >= key_lo: only query rows i >= key_lo + W
+    are materialised (each in full, so its normaliser is exact); entries of
+    keys below key_lo are NaN.
+
+    ``return_lse`` adds the row logsumexp [H_q, T] of the rows materialised;
+    ``return_far`` adds ``far[g, i] = sum_{j <= i - W} A_g[i, j]``, the mass
+    each query puts on keys at least W back (used by the mass-conservation
+    check).
+    """
+    q, k = as_f64(q), as_f64(k)
+    T, Hq, _ = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    W = int(window)
+    target = np.zeros((Hkv, T))
+    lse_all = np.full((Hq, T), np.nan)
+    far = np.full((Hq, T), np.nan)
+    for s, L in _sequences(cu_seqlens):
+        j_lo = 0 if key_lo is None else max(0, min(int(key_lo), L))
+        if key_lo is not None:
+            target[:, s:s + j_lo] = np.nan
+        i_start = min(L, j_lo + W) if key_lo is not None else 0
+        for g in range(Hq):
+            h = g // G
+            qg, kh = q[s:s + L, g, :], k[s:s + L, h, :]
+            for r0 in range(i_start, L, ROW_BLOCK):
+                r1 = min(r0 + ROW_BLOCK, L)
+                A, lse = _softmax_rows(qg, kh, r0, r1, scale)
+                lse_all[g, s + r0:s + r1] = lse
+                rows = np.arange(r0, r1)[:, None]
+                cols = np.arange(r1)[None, :]
+                F = np.where(rows - cols >= W, A, 0.0)         # key has left the window
+                far[g, s + r0:s + r1] = F.sum(axis=1)
+                col_sum = F.sum(axis=0)                         # mass each key receives
+                target[h, s + j_lo:s + r1] += col_sum[j_lo:]
+    out = [target]
+    if return_lse:
+        out.append(lse_all)
+    if return_far:
+        out.append(far)
+    return out[0] if len(out) == 1 else tuple(out)
+
+
+def keep_mask(score, cu_seqlens, window: int, sinks: int, budgets) -> np.ndarray:
+    """Sink + top-k + recent-window keep set, uint8 [H_kv, T] (1 = kept).
+
+    The top-k ranking orders the candidates by (-score, position) with
+    NumPy's stable lexsort, which puts NaN scores last.
+    """
+    score = np.asarray(score)
+    Hkv, T = score.shape
+    keep = np.zeros((Hkv, T), dtype=np.uint8)
+    budgets = np.asarray(budgets, dtype=np.int64)
+    W, S = int(window), int(sinks)
+    for b, (s, L) in enumerate(_sequences(cu_seqlens)):
+        B = int(budgets[b])
+        if B < S + W:
+            raise ValueError("budget below sinks + window")
+        if L <= B:
+            keep[:, s:s + L] = 1
+            continue
+        k_top = B - S - W
+        lo, hi = S, L - W                                       # candidate range
+        pos = np.arange(lo, hi)
+        for h in range(Hkv):
+            keep[h, s:s + S] = 1
+            keep[h, s + L - W:s + L] = 1
+            sc = score[h, s + lo:s + hi].astype(np.float64)
+            order = np.lexsort((pos, -sc))                      # -score ascending, then position
+            keep[h, s + pos[order[:k_top]]] = 1
+    return keep

@@ -1,0 +1,272 @@
+"""Pins for the CPU oracle: checks against facts other than the oracle itself.
+
+Each ``pin_*`` function takes an oracle module (the real one, or a copy with
+a planted mistake) and raises AssertionError when the oracle disagrees with
+what the definition, the mathematics or the pages fix.  ``test_oracle_pins``
+runs them on the real oracle; ``test_oracle_mutants`` checks that every
+planted mistake is caught by at least one of them.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+
+from future_attention_targets_b200.workloads import bf16_bits_to_f32, random_qk
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+# ------------------------------------------------------------ brute force
+
+def brute_force(q, k, cu, W, scale):
+    """Scalar triple loop with math.exp / math.fsum: lse [Hq,T], target [Hkv,T], far [Hq,T]."""
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    lse = [[0.0] * T for _ in range(Hq)]
+    far = [[0.0] * T for _ in range(Hq)]
+    terms = [[[] for _ in range(T)] for _ in range(Hkv)]
+    for b in range(len(cu) - 1):
+        s, e = int(cu[b]), int(cu[b + 1])
+        for g in range(Hq):
+            h = g // G
+            for i in range(s, e):
+                logits = []
+                for j in range(s, i + 1):
+                    logits.append(scale * math.fsum(float(q[i, g, t]) * float(k[j, h, t]) for t in range(d)))
+                m = max(logits)
+                Z = math.fsum(math.exp(x - m) for x in logits)
+                lse[g][i] = m + math.log(Z)
+                far_terms = []
+                for jj, x in enumerate(logits):
+                    j = s + jj
+                    if i - j >= W:
+                        a = math.exp(x - m) / Z
+                        terms[h][j].append(a)
+                        far_terms.append(a)
+                far[g][i] = math.fsum(far_terms)
+    target = np.array([[math.fsum(terms[h][j]) for j in range(T)] for h in range(Hkv)])
+    return np.array(lse), target, np.array(far)
+
+
+def _tiny_case(seed, seqlens=(7, 13), Hkv=2, G=2, d=6):
+    q_bits, k_bits = random_qk(sum(seqlens), Hkv * G, Hkv, d, seed, gain=2.0)
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    return q_bits, k_bits, cu
+
+
+def pin_brute_force(orc):
+    for seed, W in [(1, 0), (2, 1), (3, 5), (4, 12), (5, 13), (6, 40)]:
+        q_bits, k_bits, cu = _tiny_case(seed)
+        q = bf16_bits_to_f32(q_bits).astype(np.float64)
+        k = bf16_bits_to_f32(k_bits).astype(np.float64)
+        scale = 1.0 / math.sqrt(q.shape[2])
+        lse_b, tgt_b, far_b = brute_force(q, k, cu, W, scale)
+        tgt, lse, far = orc.future_target(q_bits, k_bits, cu, W, scale, return_lse=True, return_far=True)
+        np.testing.assert_allclose(tgt, tgt_b, rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(lse, lse_b, rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(far, far_b, rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(orc.row_lse(q_bits, k_bits, cu, scale), lse_b, rtol=1e-12, atol=1e-14)
+
+
+# ------------------------------------------------------------ closed forms
+
+def harmonic_target(L, W, G):
+    """All logits equal => A[i, j] = 1/(i+1); target_j = G * sum_{i=j+W}^{L-1} 1/(i+1)."""
+    inv = 1.0 / np.arange(1, L + 1, dtype=np.float64)
+    tail = np.concatenate([np.cumsum(inv[::-1])[::-1], [0.0]])     # tail[m] = sum_{i>=m} 1/(i+1)
+    return G * np.array([tail[min(j + W, L)] for j in range(L)])
+
+
+def pin_closed_form_zero_keys(orc):
+    seqlens = (300, 517)
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    for W, which in [(0, "k"), (64, "k"), (5, "q"), (299, "k")]:
+        q_bits, k_bits = random_qk(sum(seqlens), 4, 2, 16, seed=7,
+                                   q_zero=(which == "q"), k_zero=(which == "k"))
+        tgt, lse = orc.future_target(q_bits, k_bits, cu, W, 0.25, return_lse=True)
+        for b, L in enumerate(seqlens):
+            s = int(cu[b])
+            for h in range(2):
+                np.testing.assert_allclose(tgt[h, s:s + L], harmonic_target(L, W, 2), rtol=1e-12, atol=1e-15)
+            np.testing.assert_allclose(lse[:, s:s + L], np.log(np.arange(1, L + 1))[None, :].repeat(4, 0),
+                                       rtol=1e-13, atol=1e-13)
+
+
+def pin_gqa_grouping(orc):
+    """Query heads g // G map to KV head h: zero queries in group 1 force its closed form."""
+    T, Hkv, G, d, W = 200, 2, 2, 8, 10
+    q_bits, k_bits = random_qk(T, Hkv * G, Hkv, d, seed=11, gain=3.0)
+    q_bits = q_bits.copy()
+    q_bits[:, 2:4, :] = 0                                  # heads 2, 3 = group of KV head 1
+    cu = np.array([0, T], dtype=np.int32)
+    tgt = orc.future_target(q_bits, k_bits, cu, W, 1.0 / math.sqrt(d))
+    np.testing.assert_allclose(tgt[1], harmonic_target(T, W, G), rtol=1e-12, atol=1e-15)
+    assert not np.allclose(tgt[0], harmonic_target(T, W, G), rtol=1e-3)
+
+
+def pin_row_stochastic(orc):
+    """W = 0: every query row sums to 1, so the targets of a KV head sum to G * L."""
+    seqlens = (33, 90)
+    q_bits, k_bits = random_qk(sum(seqlens), 6, 3, 16, seed=5, gain=4.0)
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    tgt = orc.future_target(q_bits, k_bits, cu, 0, 0.25)
+    for b, L in enumerate(seqlens):
+        s = int(cu[b])
+        np.testing.assert_allclose(tgt[:, s:s + L].sum(axis=1), 2 * L, rtol=1e-12)
+    # W >= L: nothing has left the window.
+    tgt = orc.future_target(q_bits, k_bits, cu, 90, 0.25)
+    assert np.all(tgt[:, cu[1]:] == 0) and np.all(tgt[:, :cu[1]] == 0)
+
+
+def pin_mass_conservation(orc):
+    """sum_j target[h, j] = sum_{g in group(h)} sum_i far[g, i], and target = 0 for j >= L - W."""
+    seqlens = (150, 61)
+    q_bits, k_bits = random_qk(sum(seqlens), 8, 2, 16, seed=9, gain=3.0)
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    W = 20
+    tgt, far = orc.future_target(q_bits, k_bits, cu, W, 0.3, return_far=True)
+    for b, L in enumerate(seqlens):
+        s = int(cu[b])
+        for h in range(2):
+            np.testing.assert_allclose(tgt[h, s:s + L].sum(), far[4 * h:4 * h + 4, s:s + L].sum(), rtol=1e-12)
+            assert np.all(tgt[h, s + L - W:s + L] == 0)
+            assert np.all(tgt[h, s:s + L - W] > 0)
+
+
+def pin_single_token(orc):
+    """L = 1: the row holds one term, lse = s q.k exactly."""
+    q_bits, k_bits = random_qk(1, 2, 1, 8, seed=3, gain=2.0)
+    cu = np.array([0, 1], dtype=np.int32)
+    q = bf16_bits_to_f32(q_bits).astype(np.float64)
+    k = bf16_bits_to_f32(k_bits).astype(np.float64)
+    lse = orc.row_lse(q_bits, k_bits, cu, 0.7)
+    for g in range(2):
+        assert abs(lse[g, 0] - 0.7 * float(q[0, g] @ k[0, 0])) < 1e-14
+    tgt = orc.future_target(q_bits, k_bits, cu, 0, 0.7)
+    assert abs(tgt[0, 0] - 2.0) < 1e-14                   # each head's row is that one key
+
+
+def pin_dominant_key(orc):
+    """A key with a huge logit for every later query takes ~all of their mass."""
+    T, d, W, jstar = 120, 16, 7, 30
+    rng = np.random.default_rng(4)
+    v = np.ones(d)
+    q = np.tile(v, (T, 2, 1)) + 0.01 * rng.standard_normal((T, 2, d))
+    k = 0.01 * rng.standard_normal((T, 1, d))
+    k[jstar, 0] = 8.0 * v
+    cu = np.array([0, T], dtype=np.int32)
+    tgt = orc.future_target(q, k, cu, W, 1.0)
+    expect = 2.0 * (T - jstar - W)
+    assert abs(tgt[0, jstar] - expect) < 1e-6 * expect
+    # Queries at or after j* give (almost) nothing to earlier keys: their targets
+    # equal those of the sequence cut just before j*.
+    cut = orc.future_target(q[:jstar], k[:jstar], np.array([0, jstar], dtype=np.int32), W, 1.0)
+    np.testing.assert_allclose(tgt[0, :jstar], cut[0], rtol=0, atol=1e-6)
+
+
+# ------------------------------------------------------------ keep mask
+
+def keep_mask_by_sorting(score, cu, W, S, budgets):
+    """Independent ranking: Python's sorted() on (nan-flag, -score, position)."""
+    Hkv, T = score.shape
+    keep = np.zeros((Hkv, T), dtype=np.uint8)
+    for b in range(len(cu) - 1):
+        s, L = int(cu[b]), int(cu[b + 1] - cu[b])
+        B = int(budgets[b])
+        for h in range(Hkv):
+            if L <= B:
+                keep[h, s:s + L] = 1
+                continue
+            cand = []
+            for p in range(S, L - W):
+                x = float(score[h, s + p])
+                cand.append((1 if math.isnan(x) else 0, 0.0 if math.isnan(x) else -x, p))
+            for _, _, p in sorted(cand)[:B - S - W]:
+                keep[h, s + p] = 1
+            keep[h, s:s + S] = 1
+            keep[h, s + L - W:s + L] = 1
+    return keep
+
+
+def pin_keep_mask(orc):
+    rng = np.random.default_rng(21)
+    seqlens = (12, 400, 37, 250, 300)                    # the first is shorter than sinks + window
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    T = int(cu[-1])
+    W, S = 16, 4
+    budgets = np.array([30, 100, 60, 250, 20], dtype=np.int32)
+    score = rng.random((3, T)).astype(np.float32)
+    score[0, ::7] = 0.5                                   # many exact ties
+    score[1, 62:162] = 2.0                                # 100 tied top scores, k = 80: the tie rule decides
+    score[2, 22] = np.nan
+    score[2, 23] = -0.0
+    score[2, 24] = 0.0
+    score[2, 25] = np.inf
+    got = orc.keep_mask(score, cu, W, S, budgets)
+    ref = keep_mask_by_sorting(score, cu, W, S, budgets)
+    np.testing.assert_array_equal(got, ref)
+    for b, L in enumerate(seqlens):
+        s = int(cu[b])
+        assert np.all(got[:, s:s + L].sum(axis=1) == min(int(budgets[b]), L))
+        if L > budgets[b]:
+            mid = slice(s + S, s + L - W)
+            for h in range(3):
+                kept = score[h, mid][got[h, mid] == 1]
+                drop = score[h, mid][got[h, mid] == 0]
+                kept, drop = kept[~np.isnan(kept)], drop[~np.isnan(drop)]
+                if len(kept) and len(drop):
+                    assert kept.min() >= drop.max()
+
+
+def pin_budget_from_pages(orc):
+    """The model card's 16k budget: 4 + 3,772 + 256 = 4,032 kept per head."""
+    with open(os.path.join(GOLDEN, "kvpop_budget_16k.json")) as f:
+        g = json.load(f)
+    assert g["sinks"] + g["scored_top_k"] + g["recent_window"] == g["entries_per_head"]
+    assert g["context"] // 4 == g["quarter_of_context"] == g["entries_per_head"] + g["reserved_for_scorer_memory"]
+    L = g["context"]
+    rng = np.random.default_rng(0)
+    score = rng.random((2, L))
+    cu = np.array([0, L], dtype=np.int32)
+    keep = orc.keep_mask(score, cu, g["recent_window"], g["sinks"], [g["entries_per_head"]])
+    assert np.all(keep.sum(axis=1) == g["entries_per_head"])
+    assert np.all(keep[:, :g["sinks"]] == 1) and np.all(keep[:, L - g["recent_window"]:] == 1)
+    mid = keep[:, g["sinks"]:L - g["recent_window"]]
+    assert np.all(mid.sum(axis=1) == g["scored_top_k"])
+
+
+# ------------------------------------------------------------ restrictions
+
+def pin_restrictions(orc):
+    """key_lo / rows restrictions agree with the full computation where defined."""
+    seqlens = (140, 333)
+    q_bits, k_bits = random_qk(sum(seqlens), 4, 2, 16, seed=13, gain=2.0)
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    W = 9
+    full, lse = orc.future_target(q_bits, k_bits, cu, W, 0.3, return_lse=True)
+    part = orc.future_target(q_bits, k_bits, cu, W, 0.3, key_lo=100)
+    for b, L in enumerate(seqlens):
+        s = int(cu[b])
+        assert np.all(np.isnan(part[:, s:s + 100]))
+        np.testing.assert_allclose(part[:, s + 100:s + L], full[:, s + 100:s + L], rtol=1e-13, atol=1e-16)
+    rows = np.array([0, 5, 139, 140, 141, 300, 472])
+    lr = orc.row_lse(q_bits, k_bits, cu, 0.3, rows=rows)
+    np.testing.assert_allclose(lr[:, rows], lse[:, rows], rtol=1e-13)
+
+
+ALL_PINS = [
+    pin_brute_force,
+    pin_closed_form_zero_keys,
+    pin_gqa_grouping,
+    pin_row_stochastic,
+    pin_mass_conservation,
+    pin_single_token,
+    pin_dominant_key,
+    pin_keep_mask,
+    pin_budget_from_pages,
+    pin_restrictions,
+]

@@ -1,0 +1,69 @@
+"""The CPU oracle against brute force, closed forms, invariants and the pages' budget.
+
+Also plants mistakes in copies of the oracle (on the CPU) and checks that
+each one is caught by at least one pin.
+"""
+import importlib.util
+import os
+import sys
+
+import pytest
+
+from oracle_pins import ALL_PINS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+ORACLE_SRC = os.path.join(ROOT, "oracle", "kvpop_oracle.py")
+
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+
+import oracle  # noqa: E402
+
+
+@pytest.mark.parametrize("pin", ALL_PINS, ids=lambda f: f.__name__)
+def test_oracle_pins(pin):
+    pin(oracle)
+
+
+# Each mutant: (name, original text, replacement).  Every original must occur in the source.
+MUTANTS = [
+    ("window_strict", "rows - cols >= W", "rows - cols > W"),
+    ("causal_excludes_self", "cols <= rows, S, -np.inf", "cols < rows, S, -np.inf"),
+    ("causal_mask_dropped", "S = np.where(cols <= rows, S, -np.inf)", "S = S"),
+    ("gqa_wrong_group_target", "h = g // G\n", "h = g % Hkv\n"),
+    ("gqa_wrong_group_lse", "kh = q[s:s + L, g, :], k[s:s + L, g // G, :]",
+     "kh = q[s:s + L, g, :], k[s:s + L, g % Hkv, :]"),
+    ("scale_dropped", "S = scale * (qg[r0:r1] @ kh[:r1].T)", "S = (qg[r0:r1] @ kh[:r1].T)"),
+    ("operands_transposed", "S = scale * (qg[r0:r1] @ kh[:r1].T)", "S = scale * (kh[r0:r1] @ qg[:r1].T)"),
+    ("group_mean_not_sum", "col_sum = F.sum(axis=0)", "col_sum = F.sum(axis=0) / G"),
+    ("lse_max_dropped", "lse = (m + np.log(Z))[:, 0]", "lse = (np.log(Z))[:, 0]"),
+    ("softmax_unnormalised", "A = P / Z", "A = P"),
+    ("keep_tie_break_reversed", "np.lexsort((pos, -sc))", "np.lexsort((-pos, -sc))"),
+    ("keep_smallest_not_largest", "np.lexsort((pos, -sc))", "np.lexsort((pos, sc))"),
+    ("keep_window_short", "keep[h, s + L - W:s + L] = 1", "keep[h, s + L - W + 1:s + L] = 1"),
+    ("keep_no_sinks", "keep[h, s:s + S] = 1", "pass"),
+    ("keep_off_by_one_k", "order[:k_top]", "order[:k_top - 1]"),
+    ("keep_all_when_short_dropped", "if L <= B:", "if L < 0:"),
+]
+
+
+def _load_mutant(name, old, new, tmp_path):
+    src = open(ORACLE_SRC).read()
+    assert old in src, f"mutant {name}: text not found in the oracle"
+    path = tmp_path / f"oracle_mutant_{name}.py"
+    path.write_text(src.replace(old, new))
+    spec = importlib.util.spec_from_file_location(f"oracle_mutant_{name}", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_oracle_mutants_are_caught(name, old, new, tmp_path):
+    mod = _load_mutant(name, old, new, tmp_path)
+    caught = []
+    for pin in ALL_PINS:
+        try:
+            pin(mod)
+        except Exception:  # an assertion, or the mutant crashing on the pin's input
+            caught.append(pin.__name__)
+    assert caught, f"planted mistake {name} passed every pin"
