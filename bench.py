@@ -1,0 +1,381 @@
+"""Throughput of the future-attention-target hot path on B200.
+
+One step = row logsumexp + transposed future-target pass + keep mask over one
+synthetic Qwen3-8B-shaped layer at 16,384 tokens (32 query / 8 KV heads,
+head_dim 128, W = 256, 4 sinks, budget 4,032 per KV head), inputs resident
+in HBM.  The metric is algorithmic tensor TFLOP/s: 2 * head_dim flops per
+unmasked (query, key) pair per query head, for both passes.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (under torchrun) every rank runs its own independent layer (its
+own seed): weak scaling, no data-path collective.  `--impl reference` times
+the CPU float64 oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from future_attention_targets_b200.workloads import WORKLOADS, algorithmic_flops, make_inputs  # noqa: E402
+
+METRIC = "future-attn target TFLOP/s & % BF16 tensor peak, Qwen3-8B shape, 16k ctx"
+UNIT = "TFLOP/s"
+WORKLOAD = "qwen3_8b_16k"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["attn_kernels.cu", "kvpop_device.cuh", "kvpop_sched.h"]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "future_attention_targets_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{WORKLOAD}.traffic.txt")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, cuda_index: int):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = self._handle_for(cuda_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: report no clocks rather than guess
+            self.nvml, self.error = None, str(e)
+
+    def _handle_for(self, idx):
+        import torch
+        pynvml = self.nvml
+        try:
+            props = torch.cuda.get_device_properties(idx)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(idx)
+
+    def _run(self):
+        pynvml = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(pynvml.nvmlDeviceGetClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+                r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(0.02)
+
+    def __enter__(self):
+        if self.nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if self.nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples)}
+
+
+def threads_in_use() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads", 1) for p in threadpool_info() if p.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(d, rows: int | None, kv_head: int = 0):
+    """Runs the oracle on one KV-head group (all rows, or the last `rows` query rows).
+
+    Returns (seconds, algorithmic flops of the sample, description)."""
+    import oracle
+    w = d["workload"]
+    G, L, W = w.group, w.seqlen, w.window
+    qh = d["q_bits"][:, kv_head * G:(kv_head + 1) * G]
+    kh = d["k_bits"][:, kv_head:kv_head + 1]
+    cu = d["cu_seqlens"]
+    t0 = time.perf_counter()
+    if rows is None:
+        oracle.future_target(qh, kh, cu, W, d["scale"], return_lse=True)
+        fl = algorithmic_flops([L], G, w.head_dim, W)["total"]
+        desc = f"KV head {kv_head} with its {G} query heads, all {L} positions, both passes (1/{w.n_kv_heads} of a step)"
+    else:
+        key_lo = L - W - rows
+        oracle.future_target(qh, kh, cu, W, d["scale"], key_lo=key_lo, return_lse=True)
+        # rows i >= L - rows: their full causal rows (lse) and their future pairs with keys >= key_lo
+        n_lse = sum(i + 1 for i in range(L - rows, L))
+        n_tgt = sum(i - W - key_lo + 1 for i in range(L - rows, L) if i - W >= key_lo)
+        fl = 2 * w.head_dim * G * (n_lse + n_tgt)
+        desc = f"KV head {kv_head}, last {rows} query rows of {L}, both passes"
+    return time.perf_counter() - t0, fl, desc
+
+
+# ------------------------------------------------------------------ reference arm (CPU oracle)
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    d = make_inputs(WORKLOAD)
+    w = d["workload"]
+    rows = 256
+    for _ in range(args.warmup):
+        oracle_sample(d, rows)
+    total_t, total_f = 0.0, 0
+    desc = ""
+    for _ in range(args.steps):
+        t, f, desc = oracle_sample(d, rows)
+        total_t += t
+        total_f += f
+    value = total_f / total_t / 1e12
+    cores = threads_in_use()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": WORKLOAD, "seq_len": w.seqlen, "n_q_heads": w.n_q_heads,
+                   "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "window": w.window,
+                   "sinks": w.sinks, "budget": w.budget, "parallelism": "single host process"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {desc}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from future_attention_targets_b200 import (HostPipeline, check_status, future_target, keep_mask, lib,
+                                               row_lse)
+    from future_attention_targets_b200.build import build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.barrier()
+    lib()
+
+    d = make_inputs(WORKLOAD, seed=rank)   # an independent layer per rank
+    w = d["workload"]
+    cu, W, S, budgets, scale = d["cu_seqlens"], d["window"], d["sinks"], d["budgets"], d["scale"]
+    q = torch.from_numpy(d["q_bits"].view(np.int16)).view(torch.bfloat16).to(dev)
+    k = torch.from_numpy(d["k_bits"].view(np.int16)).view(torch.bfloat16).to(dev)
+    T = q.shape[0]
+    lse = torch.empty((w.n_q_heads, T), dtype=torch.float32, device=dev)
+    tgt = torch.empty((w.n_kv_heads, T), dtype=torch.float32, device=dev)
+    keep = torch.empty((w.n_kv_heads, T), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        row_lse(q, k, cu, scale, out=lse, status=status, stream=stream)
+        if evs is not None:
+            evs[1].record(stream)
+        future_target(q, k, cu, W, lse, scale, out=tgt, status=status, stream=stream)
+        if evs is not None:
+            evs[2].record(stream)
+        keep_mask(tgt, cu, W, S, budgets, out=keep, stream=stream)
+        if evs is not None:
+            evs[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    check_status(status, stream)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    check_status(status, stream)
+    elapsed_ms = t_start.elapsed_time(t_end)
+    per_kernel = {name: [e[j].elapsed_time(e[j + 1]) for e in evs]
+                  for j, name in enumerate(["row_lse", "future_target", "keep_mask"])}
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    fl = algorithmic_flops([w.seqlen], w.n_q_heads, w.head_dim, w.window)
+    ms_per_step = elapsed_ms / args.steps
+    value = fl["total"] * world / (ms_per_step * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    peak_sus = float(peaks.get("bf16_tflops_sustained", peak))
+
+    avg = {n: statistics.mean(v) for n, v in per_kernel.items()}
+    dom = max(("row_lse", "future_target"), key=lambda n: avg[n])
+    dom_flops = fl["lse"] if dom == "row_lse" else fl["target"]
+    achieved = dom_flops / (avg[dom] * 1e-3) / 1e12
+
+    # End to end through the host-buffer C entry point: H2D of q and k, the
+    # three kernels, D2H of target and keep, every step.
+    e2e = None
+    if not args.no_e2e:
+        pipe = HostPipeline(cu, w.n_q_heads, w.n_kv_heads, w.head_dim, W, S, budgets, scale, device=dev)
+        qh = torch.from_numpy(d["q_bits"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        kh = torch.from_numpy(d["k_bits"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        for _ in range(2):
+            pipe(qh, kh, stream)
+        n_e2e = max(3, min(args.steps, 10))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            pipe(qh, kh, stream)   # synchronises the stream after each step (results on the host)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": fl["total"] * world / (e_ms / n_e2e * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": pipe.h2d_bytes, "d2h_bytes_per_step": pipe.d2h_bytes,
+               "ms_per_step": e_ms / n_e2e, "steps": n_e2e}
+        del pipe
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t, f, desc = oracle_sample(d, None)
+        cpu = {"value": f / t / 1e12, "unit": UNIT, "cores": threads_in_use(), "kind": "oracle",
+               "sample": desc, "seconds": t}
+
+    if rank == 0:
+        keys = sum(int(L) for L in np.diff(cu)) * w.n_kv_heads * world
+        attn_ms = avg["row_lse"] + avg["future_target"]
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "seq_len": w.seqlen, "n_q_heads": w.n_q_heads,
+                       "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "window": w.window,
+                       "sinks": w.sinks, "budget": w.budget, "input": "1% heavy-hitter keys, seed = rank",
+                       "l2": "inputs larger than L2 (160 MiB of Q and K vs 126 MB L2); no flush",
+                       "parallelism": f"independent layer per GPU x{world}"},
+            "pct_of_bf16_peak": 100.0 * value / world / peak,
+            "pct_of_bf16_peak_sustained": 100.0 * value / world / peak_sus,
+            "keys_per_s": keys / (attn_ms * 1e-3),
+            "kernel_ms": {n: round(v, 4) for n, v in avg.items()},
+            "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": f"{peak_kind} bf16 burst",
+                         "traffic": recorded_traffic(dom),
+                         "algorithmic_flops_per_launch": dom_flops},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 3 * args.steps,
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: at least 3 warm-up steps are used", file=sys.stderr)
+        args.warmup = 3
+    return run_reference(args) if args.impl == "reference" else run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,20 @@
+"""KVpop future-attention targets on NVIDIA B200 (sm_100a).
+
+The compute lives in libkvpop.so (C ABI in include/kvpop.h, CUDA kernels in
+csrc/); this package is its Python binding plus the seeded workload
+generators.  See ``_binding`` for the entry points.
+"""
+from ._binding import (  # noqa: F401
+    HostPipeline,
+    KvpopError,
+    check_status,
+    future_target,
+    future_targets,
+    keep_mask,
+    lib,
+    row_lse,
+    selftest_bounded_wait,
+)
+
+__all__ = ["HostPipeline", "KvpopError", "check_status", "future_target", "future_targets", "keep_mask", "lib",
+           "row_lse", "selftest_bounded_wait"]

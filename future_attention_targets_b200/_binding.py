@@ -1,0 +1,250 @@
+"""ctypes binding of libkvpop.so (include/kvpop.h): argument marshalling only.
+
+Every step of the computation runs in the library's CUDA kernels; PyTorch is
+used here only to allocate device memory and to supply the current stream.
+There is no CPU fallback: without the built library every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+import threading
+
+import numpy as np
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libkvpop.so")
+HEADER_PATH = os.path.join(os.path.dirname(PKG_DIR), "include", "kvpop.h")
+
+OK, INVALID_ARG, UNSUPPORTED, CUDA_ERROR, TIMEOUT = 0, 1, 2, 3, 4
+STATUS_NAMES = {OK: "KVPOP_OK", INVALID_ARG: "KVPOP_ERR_INVALID_ARG", UNSUPPORTED: "KVPOP_ERR_UNSUPPORTED",
+                CUDA_ERROR: "KVPOP_ERR_CUDA", TIMEOUT: "KVPOP_ERR_TIMEOUT"}
+
+
+class KvpopError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("total_tokens", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
+                ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+
+
+_P = ctypes.c_void_p
+_I32P = ctypes.POINTER(ctypes.c_int32)
+_SIGS = {
+    "kvpop_row_lse": (ctypes.c_int, [_P, _P, _I32P, Shape, ctypes.c_float, _P, _P, _P]),
+    "kvpop_future_target": (ctypes.c_int, [_P, _P, _I32P, Shape, ctypes.c_float, ctypes.c_int32, _P, _P, _P, _P]),
+    "kvpop_keep_mask": (ctypes.c_int, [_P, _I32P, Shape, ctypes.c_int32, ctypes.c_int32, _I32P, _P, _P]),
+    "kvpop_future_targets": (ctypes.c_int, [_P, _P, _I32P, Shape, ctypes.c_float, ctypes.c_int32, ctypes.c_int32,
+                                            _I32P, _P, _P, _P, _P, _P]),
+    "kvpop_host_workspace_bytes": (ctypes.c_size_t, [Shape]),
+    "kvpop_future_targets_host": (ctypes.c_int, [_P, _P, _I32P, Shape, ctypes.c_float, ctypes.c_int32,
+                                                 ctypes.c_int32, _I32P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
+    "kvpop_check_device_status": (ctypes.c_int, [_P, _P]),
+    "kvpop_selftest_bounded_wait": (ctypes.c_int, [_P, ctypes.c_uint64, _P]),
+    "kvpop_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "kvpop_last_error": (ctypes.c_char_p, []),
+    "kvpop_abi_version": (ctypes.c_int32, []),
+}
+
+_lock = threading.Lock()
+_handle = None
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libkvpop.so (once).  Raises if it has not been built."""
+    global _handle
+    with _lock:
+        if _handle is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                   "`python -m future_attention_targets_b200.build` (needs nvcc)")
+            h = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in _SIGS.items():
+                fn = getattr(h, name)
+                fn.restype = res
+                fn.argtypes = args
+            _handle = h
+    return _handle
+
+
+def header_symbols() -> list[str]:
+    """Entry points declared in include/kvpop.h."""
+    with open(HEADER_PATH) as f:
+        return re.findall(r"KVPOP_API\s+[\w\s\*]+?\b(kvpop_\w+)\s*\(", f.read())
+
+
+def _check(status: int) -> None:
+    if status != OK:
+        raise KvpopError(status, lib().kvpop_last_error().decode())
+
+
+def _i32_host(values) -> ctypes.Array:
+    arr = np.ascontiguousarray(np.asarray(values, dtype=np.int64))
+    if arr.size and (arr.min() < -2**31 or arr.max() >= 2**31):
+        raise ValueError("value out of int32 range")
+    return (ctypes.c_int32 * arr.size)(*arr.astype(np.int32).tolist())
+
+
+def _cu_host(cu_seqlens):
+    try:
+        import torch
+        if isinstance(cu_seqlens, torch.Tensor):
+            cu_seqlens = cu_seqlens.detach().cpu().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    cu = np.asarray(cu_seqlens, dtype=np.int64).reshape(-1)
+    return cu, _i32_host(cu)
+
+
+def _stream_ptr(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _shape(q, k, cu) -> Shape:
+    T, Hq, d = q.shape
+    Hkv = k.shape[1]
+    return Shape(len(cu) - 1, T, Hq, Hkv, d)
+
+
+def _check_qk(q, k):
+    import torch
+    for name, t in (("q", q), ("k", k)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or not t.is_cuda or t.dim() != 3:
+            raise TypeError(f"{name} must be a 3-D bf16 CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if q.shape[0] != k.shape[0] or q.shape[2] != k.shape[2]:
+        raise ValueError("q [T, H_q, d] and k [T, H_kv, d] disagree on T or d")
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+# ------------------------------------------------------------------ entry points
+
+def row_lse(q, k, cu_seqlens, scale: float | None = None, out=None, status=None, stream=None):
+    """lse [H_q, T] fp32 (natural log) of the causal softmax rows."""
+    import torch
+    _check_qk(q, k)
+    cu, cu_c = _cu_host(cu_seqlens)
+    sh = _shape(q, k, cu)
+    scale = 1.0 / math.sqrt(sh.head_dim) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((sh.n_q_heads, sh.total_tokens), dtype=torch.float32, device=q.device)
+    _check(lib().kvpop_row_lse(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, out.data_ptr(), _ptr(status),
+                               _stream_ptr(stream)))
+    return out
+
+
+def future_target(q, k, cu_seqlens, window: int, lse, scale: float | None = None, out=None, status=None,
+                  stream=None):
+    """target [H_kv, T] fp32: mass each key receives from queries i >= j + W, summed over its GQA group."""
+    import torch
+    _check_qk(q, k)
+    cu, cu_c = _cu_host(cu_seqlens)
+    sh = _shape(q, k, cu)
+    scale = 1.0 / math.sqrt(sh.head_dim) if scale is None else float(scale)
+    if lse.dtype != torch.float32 or not lse.is_cuda or tuple(lse.shape) != (sh.n_q_heads, sh.total_tokens):
+        raise ValueError("lse must be a fp32 CUDA tensor [H_q, T]")
+    if out is None:
+        out = torch.empty((sh.n_kv_heads, sh.total_tokens), dtype=torch.float32, device=q.device)
+    _check(lib().kvpop_future_target(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, int(window),
+                                     lse.contiguous().data_ptr(), out.data_ptr(), _ptr(status), _stream_ptr(stream)))
+    return out
+
+
+def keep_mask(score, cu_seqlens, window: int, sinks: int, budgets, out=None, stream=None):
+    """keep [H_kv, T] uint8: sinks + recent window + top-(budget - sinks - window) scores."""
+    import torch
+    if score.dtype != torch.float32 or not score.is_cuda or score.dim() != 2 or not score.is_contiguous():
+        raise TypeError("score must be a contiguous 2-D fp32 CUDA tensor [H_kv, T]")
+    cu, cu_c = _cu_host(cu_seqlens)
+    Hkv, T = score.shape
+    sh = Shape(len(cu) - 1, T, Hkv, Hkv, 128)
+    bud = _i32_host(budgets)
+    if len(bud) != sh.batch:
+        raise ValueError("one budget per sequence is needed")
+    if out is None:
+        out = torch.empty((Hkv, T), dtype=torch.uint8, device=score.device)
+    _check(lib().kvpop_keep_mask(score.data_ptr(), cu_c, sh, int(window), int(sinks), bud, out.data_ptr(),
+                                 _stream_ptr(stream)))
+    return out
+
+
+def future_targets(q, k, cu_seqlens, window: int, sinks: int, budgets, scale: float | None = None,
+                   lse=None, target=None, keep=None, status=None, stream=None):
+    """The whole hot path on device tensors: returns (lse, target, keep)."""
+    import torch
+    _check_qk(q, k)
+    cu, cu_c = _cu_host(cu_seqlens)
+    sh = _shape(q, k, cu)
+    scale = 1.0 / math.sqrt(sh.head_dim) if scale is None else float(scale)
+    dev = q.device
+    if lse is None:
+        lse = torch.empty((sh.n_q_heads, sh.total_tokens), dtype=torch.float32, device=dev)
+    if target is None:
+        target = torch.empty((sh.n_kv_heads, sh.total_tokens), dtype=torch.float32, device=dev)
+    if keep is None:
+        keep = torch.empty((sh.n_kv_heads, sh.total_tokens), dtype=torch.uint8, device=dev)
+    bud = _i32_host(budgets)
+    _check(lib().kvpop_future_targets(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, int(window), int(sinks), bud,
+                                      lse.data_ptr(), target.data_ptr(), keep.data_ptr(), _ptr(status),
+                                      _stream_ptr(stream)))
+    return lse, target, keep
+
+
+class HostPipeline:
+    """The hot path on host buffers through kvpop_future_targets_host.
+
+    Owns one device workspace (allocated once by torch) and pinned host
+    outputs; each call copies q and k in, runs the three passes and copies
+    target and keep out, all on one stream.
+    """
+
+    def __init__(self, cu_seqlens, n_q_heads: int, n_kv_heads: int, head_dim: int, window: int, sinks: int,
+                 budgets, scale: float | None = None, device=None):
+        import torch
+        self.cu, self.cu_c = _cu_host(cu_seqlens)
+        T = int(self.cu[-1])
+        self.shape = Shape(len(self.cu) - 1, T, n_q_heads, n_kv_heads, head_dim)
+        self.window, self.sinks = int(window), int(sinks)
+        self.budgets = _i32_host(budgets)
+        self.scale = 1.0 / math.sqrt(head_dim) if scale is None else float(scale)
+        self.device = torch.device("cuda") if device is None else torch.device(device)
+        nbytes = int(lib().kvpop_host_workspace_bytes(self.shape))
+        self.workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self.target = torch.empty((n_kv_heads, T), dtype=torch.float32, pin_memory=True)
+        self.keep = torch.empty((n_kv_heads, T), dtype=torch.uint8, pin_memory=True)
+        self.h2d_bytes = T * (n_q_heads + n_kv_heads) * head_dim * 2
+        self.d2h_bytes = T * n_kv_heads * 5
+
+    def __call__(self, q_host, k_host, stream=None):
+        """q_host, k_host: pinned CPU bf16 tensors.  Returns (target, keep) host tensors after syncing."""
+        import torch
+        s = torch.cuda.current_stream(self.device) if stream is None else stream
+        _check(lib().kvpop_future_targets_host(
+            q_host.data_ptr(), k_host.data_ptr(), self.cu_c, self.shape, self.scale, self.window, self.sinks,
+            self.budgets, self.target.data_ptr(), self.keep.data_ptr(), self.workspace.data_ptr(),
+            self.workspace.numel(), self.status.data_ptr(), _stream_ptr(s)))
+        s.synchronize()
+        return self.target, self.keep
+
+
+def check_status(status, stream=None) -> None:
+    """Raises KvpopError(TIMEOUT) when a kernel recorded a wait that ran out."""
+    _check(lib().kvpop_check_device_status(status.data_ptr(), _stream_ptr(stream)))
+
+
+def selftest_bounded_wait(status, limit_ns: int, stream=None) -> None:
+    _check(lib().kvpop_selftest_bounded_wait(status.data_ptr(), int(limit_ns), _stream_ptr(stream)))

@@ -1,0 +1,396 @@
+// Host side of the C ABI declared in include/kvpop.h: argument validation,
+// TMA descriptor encoding, the longest-first work schedule, and launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "kvpop.h"
+#include "kvpop_sched.h"
+
+namespace kvpop {
+cudaError_t launch_row_lse(const AttnParams& p, int head_dim, int grid, cudaStream_t stream);
+cudaError_t launch_future_target(const AttnParams& p, int head_dim, int grid, cudaStream_t stream);
+cudaError_t launch_keep_mask(const KeepParams& p, int n_kv_heads, cudaStream_t stream);
+cudaError_t launch_selftest_wait(int32_t* status, uint64_t limit_ns, cudaStream_t stream);
+}  // namespace kvpop
+
+using namespace kvpop;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+kvpop_status fail(kvpop_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+kvpop_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(KVPOP_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+// ---------------------------------------------------------------- device info
+
+struct DeviceInfo {
+  int sm_count = 0;
+  int major = 0, minor = 0;
+};
+
+kvpop_status device_info(DeviceInfo* out) {
+  static std::mutex mu;
+  static std::vector<DeviceInfo> cache;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lock(mu);
+  if (static_cast<int>(cache.size()) <= dev) cache.resize(dev + 1);
+  DeviceInfo& d = cache[dev];
+  if (d.sm_count == 0) {
+    if ((e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess) {
+      d.sm_count = 0;
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    }
+  }
+  *out = d;
+  if (d.major != 10 || d.minor != 0)
+    return fail(KVPOP_ERR_UNSUPPORTED, "device compute capability %d.%d; this library is built for sm_100a only",
+                d.major, d.minor);
+  return KVPOP_OK;
+}
+
+// ---------------------------------------------------------------- tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 matrix [rows, cols] (row-major, cols contiguous) read as boxes of
+// 64 columns x box_rows rows with 128-byte swizzle; rows past the end read as 0.
+kvpop_status make_map(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return fail(KVPOP_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KVPOP_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+  return KVPOP_OK;
+}
+
+// ---------------------------------------------------------------- validation
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+kvpop_status check_shape(const int32_t* cu, const kvpop_shape& sh, bool need_heads) {
+  if (cu == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "cu_seqlens is NULL");
+  if (sh.batch < 1) return fail(KVPOP_ERR_INVALID_ARG, "batch must be >= 1 (got %d)", sh.batch);
+  if (sh.batch > kMaxSeqs) return fail(KVPOP_ERR_UNSUPPORTED, "batch %d exceeds the %d-sequence limit", sh.batch, kMaxSeqs);
+  if (sh.total_tokens < 0) return fail(KVPOP_ERR_INVALID_ARG, "total_tokens must be >= 0");
+  if (sh.n_kv_heads < 1) return fail(KVPOP_ERR_INVALID_ARG, "n_kv_heads must be >= 1");
+  if (need_heads) {
+    if (sh.n_q_heads < 1) return fail(KVPOP_ERR_INVALID_ARG, "n_q_heads must be >= 1");
+    if (sh.n_q_heads % sh.n_kv_heads != 0)
+      return fail(KVPOP_ERR_INVALID_ARG, "n_q_heads (%d) is not a multiple of n_kv_heads (%d)", sh.n_q_heads,
+                  sh.n_kv_heads);
+    if (sh.head_dim != 64 && sh.head_dim != 128)
+      return fail(KVPOP_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", sh.head_dim);
+    if (static_cast<int64_t>(sh.n_q_heads) * sh.head_dim > (1 << 24))
+      return fail(KVPOP_ERR_UNSUPPORTED, "n_q_heads * head_dim too large");
+  }
+  if (cu[0] != 0) return fail(KVPOP_ERR_INVALID_ARG, "cu_seqlens[0] must be 0 (got %d)", cu[0]);
+  for (int b = 0; b < sh.batch; ++b) {
+    const int64_t L = static_cast<int64_t>(cu[b + 1]) - cu[b];
+    if (L < 0) return fail(KVPOP_ERR_INVALID_ARG, "cu_seqlens decreases at %d", b);
+    if (L > static_cast<int64_t>(kMaxLevels) * kTileRows)
+      return fail(KVPOP_ERR_UNSUPPORTED, "sequence %d has %lld tokens (limit %d)", b, static_cast<long long>(L),
+                  kMaxLevels * kTileRows);
+  }
+  if (cu[sh.batch] != sh.total_tokens)
+    return fail(KVPOP_ERR_INVALID_ARG, "cu_seqlens[batch] (%d) != total_tokens (%d)", cu[sh.batch],
+                sh.total_tokens);
+  return KVPOP_OK;
+}
+
+kvpop_status check_qk(const void* q, const void* k, float scale) {
+  if (q == nullptr || k == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "q or k is NULL");
+  if (!aligned16(q) || !aligned16(k)) return fail(KVPOP_ERR_INVALID_ARG, "q and k must be 16-byte aligned");
+  if (!isfinite(scale)) return fail(KVPOP_ERR_INVALID_ARG, "scale must be finite");
+  return KVPOP_OK;
+}
+
+// ---------------------------------------------------------------- schedule
+
+// Items (level, sequence, head), heaviest level first.  Sequences with t
+// 128-row tiles take part in levels 0 .. t-1.
+void build_schedule(const int32_t* cu, int batch, int n_heads, LevelSchedule* s) {
+  std::vector<std::pair<int, int>> seqs;  // (tiles, index)
+  for (int b = 0; b < batch; ++b) {
+    const int L = cu[b + 1] - cu[b];
+    const int t = (L + kTileRows - 1) / kTileRows;
+    if (t > 0) seqs.emplace_back(t, b);
+  }
+  std::stable_sort(seqs.begin(), seqs.end(), [](const std::pair<int, int>& a, const std::pair<int, int>& b) {
+    return a.first > b.first;
+  });
+  memset(s, 0, sizeof(*s));
+  s->n_seqs = static_cast<int32_t>(seqs.size());
+  s->n_heads = n_heads;
+  s->n_levels = seqs.empty() ? 0 : seqs[0].first;
+  for (size_t r = 0; r < seqs.size(); ++r) {
+    s->seq_start[r] = cu[seqs[r].second];
+    s->seq_len[r] = cu[seqs[r].second + 1] - cu[seqs[r].second];
+  }
+  int32_t running = 0;
+  size_t active = 0;  // sequences with a tile at this level form a prefix of the sorted list
+  for (int k = 0; k < s->n_levels; ++k) {
+    const int level = s->n_levels - 1 - k;
+    while (active < seqs.size() && seqs[active].first > level) ++active;
+    s->level_base[k] = running;
+    running += static_cast<int32_t>(active) * n_heads;
+  }
+  s->level_base[s->n_levels] = running;
+  s->total_items = running;
+}
+
+int grid_for(int items, int sm_count) { return std::max(1, std::min(items, sm_count)); }
+
+kvpop_status fill_attn_common(AttnParams* p, const void* q, const void* k, const int32_t* cu,
+                              const kvpop_shape& sh, float scale, bool target_pass) {
+  memset(p, 0, sizeof(*p));
+  const int64_t T = sh.total_tokens;
+  kvpop_status st;
+  // Resident (A) tiles are 128 rows, streamed (B) tiles 256 rows.
+  if ((st = make_map(&p->tmap_q, q, static_cast<int64_t>(sh.n_q_heads) * sh.head_dim, T,
+                     target_pass ? kStreamRows : kTileRows)) != KVPOP_OK)
+    return st;
+  if ((st = make_map(&p->tmap_k, k, static_cast<int64_t>(sh.n_kv_heads) * sh.head_dim, T,
+                     target_pass ? kTileRows : kStreamRows)) != KVPOP_OK)
+    return st;
+  p->wait_ns = kDefaultWaitNs;
+  p->total_tokens = sh.total_tokens;
+  p->n_q_heads = sh.n_q_heads;
+  p->n_kv_heads = sh.n_kv_heads;
+  p->group = sh.n_q_heads / sh.n_kv_heads;
+  p->scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  build_schedule(cu, sh.batch, target_pass ? sh.n_kv_heads : sh.n_q_heads, &p->sched);
+  return KVPOP_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+
+extern "C" {
+
+int32_t kvpop_abi_version(void) { return KVPOP_ABI_VERSION; }
+
+const char* kvpop_last_error(void) { return g_last_error.c_str(); }
+
+const char* kvpop_status_string(kvpop_status s) {
+  switch (s) {
+    case KVPOP_OK: return "ok";
+    case KVPOP_ERR_INVALID_ARG: return "invalid argument";
+    case KVPOP_ERR_UNSUPPORTED: return "unsupported";
+    case KVPOP_ERR_CUDA: return "CUDA error";
+    case KVPOP_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+kvpop_status kvpop_row_lse(const void* q, const void* k, const int32_t* cu_seqlens, kvpop_shape shape, float scale,
+                           float* lse, int32_t* dev_status, void* stream) {
+  kvpop_status st;
+  if ((st = check_qk(q, k, scale)) != KVPOP_OK) return st;
+  if (lse == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "lse is NULL");
+  if ((st = check_shape(cu_seqlens, shape, true)) != KVPOP_OK) return st;
+  if (shape.total_tokens == 0) return KVPOP_OK;
+  DeviceInfo dev;
+  if ((st = device_info(&dev)) != KVPOP_OK) return st;
+  AttnParams p;
+  if ((st = fill_attn_common(&p, q, k, cu_seqlens, shape, scale, false)) != KVPOP_OK) return st;
+  p.out = lse;
+  p.status = dev_status;
+  if (p.sched.total_items == 0) return KVPOP_OK;
+  cudaError_t e = launch_row_lse(p, shape.head_dim, grid_for(p.sched.total_items, dev.sm_count),
+                                 static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "row_lse launch");
+}
+
+kvpop_status kvpop_future_target(const void* q, const void* k, const int32_t* cu_seqlens, kvpop_shape shape,
+                                 float scale, int32_t window, const float* lse, float* target,
+                                 int32_t* dev_status, void* stream) {
+  kvpop_status st;
+  if ((st = check_qk(q, k, scale)) != KVPOP_OK) return st;
+  if (lse == nullptr || target == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "lse or target is NULL");
+  if (window < 0) return fail(KVPOP_ERR_INVALID_ARG, "window must be >= 0 (got %d)", window);
+  if ((st = check_shape(cu_seqlens, shape, true)) != KVPOP_OK) return st;
+  if (shape.total_tokens == 0) return KVPOP_OK;
+  DeviceInfo dev;
+  if ((st = device_info(&dev)) != KVPOP_OK) return st;
+  AttnParams p;
+  if ((st = fill_attn_common(&p, q, k, cu_seqlens, shape, scale, true)) != KVPOP_OK) return st;
+  // A window longer than any sequence leaves every target at zero; clamp it
+  // so the tile arithmetic stays in range.
+  p.window = std::min<int32_t>(window, kMaxLevels * kTileRows + 1);
+  p.lse_in = lse;
+  p.out = target;
+  p.status = dev_status;
+  if (p.sched.total_items == 0) return KVPOP_OK;
+  cudaError_t e = launch_future_target(p, shape.head_dim, grid_for(p.sched.total_items, dev.sm_count),
+                                       static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "future_target launch");
+}
+
+kvpop_status kvpop_keep_mask(const float* score, const int32_t* cu_seqlens, kvpop_shape shape, int32_t window,
+                             int32_t sinks, const int32_t* budgets, uint8_t* keep, void* stream) {
+  kvpop_status st;
+  if (score == nullptr || keep == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "score or keep is NULL");
+  if (budgets == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "budgets is NULL");
+  if (window < 0 || sinks < 0) return fail(KVPOP_ERR_INVALID_ARG, "window and sinks must be >= 0");
+  if ((st = check_shape(cu_seqlens, shape, false)) != KVPOP_OK) return st;
+  for (int b = 0; b < shape.batch; ++b) {
+    if (static_cast<int64_t>(budgets[b]) < static_cast<int64_t>(sinks) + window)
+      return fail(KVPOP_ERR_INVALID_ARG, "budget[%d] = %d is below sinks + window = %lld", b, budgets[b],
+                  static_cast<long long>(sinks) + window);
+  }
+  if (shape.total_tokens == 0) return KVPOP_OK;
+  DeviceInfo dev;
+  if ((st = device_info(&dev)) != KVPOP_OK) return st;
+  KeepParams p;
+  memset(&p, 0, sizeof(p));
+  p.score = score;
+  p.keep = keep;
+  p.total_tokens = shape.total_tokens;
+  p.window = window;
+  p.sinks = sinks;
+  p.n_seqs = shape.batch;
+  for (int b = 0; b < shape.batch; ++b) {
+    p.seq_start[b] = cu_seqlens[b];
+    p.seq_len[b] = cu_seqlens[b + 1] - cu_seqlens[b];
+    p.budget[b] = budgets[b];
+  }
+  cudaError_t e = launch_keep_mask(p, shape.n_kv_heads, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "keep_mask launch");
+}
+
+kvpop_status kvpop_future_targets(const void* q, const void* k, const int32_t* cu_seqlens, kvpop_shape shape,
+                                  float scale, int32_t window, int32_t sinks, const int32_t* budgets, float* lse,
+                                  float* target, uint8_t* keep, int32_t* dev_status, void* stream) {
+  kvpop_status st;
+  // Validate everything before the first launch.
+  if ((st = check_qk(q, k, scale)) != KVPOP_OK) return st;
+  if (lse == nullptr || target == nullptr || keep == nullptr || budgets == nullptr)
+    return fail(KVPOP_ERR_INVALID_ARG, "lse, target, keep or budgets is NULL");
+  if (window < 0 || sinks < 0) return fail(KVPOP_ERR_INVALID_ARG, "window and sinks must be >= 0");
+  if ((st = check_shape(cu_seqlens, shape, true)) != KVPOP_OK) return st;
+  for (int b = 0; b < shape.batch; ++b)
+    if (static_cast<int64_t>(budgets[b]) < static_cast<int64_t>(sinks) + window)
+      return fail(KVPOP_ERR_INVALID_ARG, "budget[%d] = %d is below sinks + window", b, budgets[b]);
+  if ((st = kvpop_row_lse(q, k, cu_seqlens, shape, scale, lse, dev_status, stream)) != KVPOP_OK) return st;
+  if ((st = kvpop_future_target(q, k, cu_seqlens, shape, scale, window, lse, target, dev_status, stream)) !=
+      KVPOP_OK)
+    return st;
+  return kvpop_keep_mask(target, cu_seqlens, shape, window, sinks, budgets, keep, stream);
+}
+
+size_t kvpop_host_workspace_bytes(kvpop_shape shape) {
+  if (shape.total_tokens <= 0 || shape.n_q_heads <= 0 || shape.n_kv_heads <= 0 || shape.head_dim <= 0) return 0;
+  const size_t T = static_cast<size_t>(shape.total_tokens);
+  return align256(T * shape.n_q_heads * shape.head_dim * 2) + align256(T * shape.n_kv_heads * shape.head_dim * 2) +
+         align256(T * shape.n_q_heads * 4) + align256(T * shape.n_kv_heads * 4) + align256(T * shape.n_kv_heads);
+}
+
+kvpop_status kvpop_future_targets_host(const void* q_host, const void* k_host, const int32_t* cu_seqlens,
+                                       kvpop_shape shape, float scale, int32_t window, int32_t sinks,
+                                       const int32_t* budgets, float* target_host, uint8_t* keep_host,
+                                       void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  kvpop_status st;
+  if (q_host == nullptr || k_host == nullptr || target_host == nullptr || keep_host == nullptr)
+    return fail(KVPOP_ERR_INVALID_ARG, "a host buffer is NULL");
+  if ((st = check_shape(cu_seqlens, shape, true)) != KVPOP_OK) return st;
+  if (shape.total_tokens == 0) return KVPOP_OK;
+  const size_t need = kvpop_host_workspace_bytes(shape);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(KVPOP_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu required", workspace_bytes,
+                need);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(KVPOP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const size_t T = static_cast<size_t>(shape.total_tokens);
+  const size_t qb = T * shape.n_q_heads * shape.head_dim * 2, kb = T * shape.n_kv_heads * shape.head_dim * 2;
+  const size_t lb = T * shape.n_q_heads * 4, tb = T * shape.n_kv_heads * 4, mb = T * shape.n_kv_heads;
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  void* q = w;
+  void* k = w + align256(qb);
+  float* lse = reinterpret_cast<float*>(w + align256(qb) + align256(kb));
+  float* target = reinterpret_cast<float*>(w + align256(qb) + align256(kb) + align256(lb));
+  uint8_t* keep = w + align256(qb) + align256(kb) + align256(lb) + align256(tb);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if ((e = cudaMemcpyAsync(q, q_host, qb, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy q");
+  if ((e = cudaMemcpyAsync(k, k_host, kb, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy k");
+  if ((st = kvpop_future_targets(q, k, cu_seqlens, shape, scale, window, sinks, budgets, lse, target, keep,
+                                 dev_status, stream)) != KVPOP_OK)
+    return st;
+  if ((e = cudaMemcpyAsync(target_host, target, tb, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
+    return cuda_fail(e, "copy target");
+  if ((e = cudaMemcpyAsync(keep_host, keep, mb, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
+    return cuda_fail(e, "copy keep");
+  return KVPOP_OK;
+}
+
+kvpop_status kvpop_check_device_status(const int32_t* dev_status, void* stream) {
+  if (dev_status == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "dev_status is NULL");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int32_t v = 0;
+  e = cudaMemcpy(&v, dev_status, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read dev_status");
+  if (v == 0) return KVPOP_OK;
+  if ((v & 0xff) == KVPOP_ERR_TIMEOUT)
+    return fail(KVPOP_ERR_TIMEOUT, "a kernel wait timed out (site %d)", (v >> 8) & 0xff);
+  return fail(KVPOP_ERR_CUDA, "device status word holds %d", v);
+}
+
+kvpop_status kvpop_selftest_bounded_wait(int32_t* dev_status, uint64_t limit_ns, void* stream) {
+  if (dev_status == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "dev_status is NULL");
+  if (limit_ns < 1 || limit_ns > 1000000000ull) return fail(KVPOP_ERR_INVALID_ARG, "limit_ns out of range");
+  DeviceInfo dev;
+  kvpop_status st;
+  if ((st = device_info(&dev)) != KVPOP_OK) return st;
+  cudaError_t e = launch_selftest_wait(dev_status, limit_ns, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "selftest launch");
+}
+
+}  // extern "C"

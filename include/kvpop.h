@@ -1,0 +1,165 @@
+/*
+ * kvpop.h -- C ABI for KVpop future-attention targets on NVIDIA B200 (sm_100a).
+ *
+ * KVpop trains a per-KV-head token scorer against a "future-attention
+ * target": the attention mass a token will receive from later queries once it
+ * has left a small protected recent window, computed during training with a
+ * transposed attention pass so that the dense attention map is never formed
+ * (aiweekly article "KVpop shrinks Qwen3 KV cache 88%", second paragraph;
+ * KVpop paper summary; French article, second paragraph).  At inference the
+ * cache keeps sink tokens, the protected recent window and the scored top-k
+ * of the older tokens (Qwen3-8B-KVpop-4x model card, introduction:
+ * 4 sink + 3,772 scored + 256 recent = 4,032 entries per head).
+ *
+ * Definitions used by every call (one packed sequence of length L; positions
+ * i, j relative to the sequence's start; G = n_q_heads / n_kv_heads; query
+ * head g reads KV head g / G; s = the softmax scale):
+ *
+ *   lse[g, i]    = ln sum_{j <= i} exp(s * q[i, g, :] . k[j, g/G, :])
+ *   target[h, j] = sum_{g : g/G = h} sum_{i = j+W}^{L-1} exp(s * q[i,g,:] . k[j,h,:] - lse[g, i])
+ *
+ * Key j has left the recent window of W positions exactly when the query is
+ * at i >= j + W; target[h, j] = 0 for j >= L - W.
+ *
+ * Memory layouts (row-major, no padding, element strides as written):
+ *   q       bf16  [T, n_q_heads,  head_dim]      T = cu_seqlens[batch]
+ *   k       bf16  [T, n_kv_heads, head_dim]
+ *   lse     fp32  [n_q_heads,  T]                natural logarithm
+ *   target  fp32  [n_kv_heads, T]
+ *   keep    uint8 [n_kv_heads, T]                1 = kept, 0 = evicted
+ *
+ * Ownership: every pointer is owned by the caller.  Device pointers must stay
+ * valid until the enqueued work has finished.  Calls are stream-ordered: they
+ * validate on the host, enqueue on `stream` (a cudaStream_t, NULL = legacy
+ * default stream) on the current device and return without synchronising.
+ * The library allocates no device memory and keeps no mutable state besides
+ * per-device caches (SM count, capability, kernel attributes).
+ *
+ * Errors: a call returns KVPOP_ERR_INVALID_ARG or KVPOP_ERR_UNSUPPORTED before
+ * touching the device when an argument is bad; KVPOP_ERR_CUDA when the CUDA
+ * runtime reports an error (cudaGetLastError after the launch).  Kernels that
+ * wait on on-chip barriers give every wait a time limit; when one runs out the
+ * kernel writes a nonzero code into *dev_status, stops its work early and
+ * exits cleanly; kvpop_check_device_status() maps that word to
+ * KVPOP_ERR_TIMEOUT.  kvpop_last_error() gives a one-line description of the
+ * last failure on the calling thread.
+ */
+#ifndef KVPOP_H_
+#define KVPOP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KVPOP_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define KVPOP_API __attribute__((visibility("default")))
+#else
+#define KVPOP_API
+#endif
+
+typedef enum {
+  KVPOP_OK = 0,
+  KVPOP_ERR_INVALID_ARG = 1,   /* null pointer, bad size, inconsistent cu_seqlens, ... */
+  KVPOP_ERR_UNSUPPORTED = 2,   /* head_dim not 64/128, too many sequences or tokens, non-sm_100 device */
+  KVPOP_ERR_CUDA = 3,          /* CUDA runtime error (launch, copy, device query) */
+  KVPOP_ERR_TIMEOUT = 4        /* a kernel's bounded on-chip wait ran out (from kvpop_check_device_status) */
+} kvpop_status;
+
+/* Problem shape.  cu_seqlens (host memory, int32 [batch + 1]) holds the packed
+ * sequence offsets: cu_seqlens[0] = 0, non-decreasing, cu_seqlens[batch] =
+ * total_tokens.  Zero-length sequences are allowed. */
+typedef struct {
+  int32_t batch;          /* number of packed sequences, 1 .. 512 */
+  int32_t total_tokens;   /* T, >= 0; every sequence at most 131072 tokens */
+  int32_t n_q_heads;      /* >= 1, a multiple of n_kv_heads */
+  int32_t n_kv_heads;     /* >= 1 */
+  int32_t head_dim;       /* 64 or 128 */
+} kvpop_shape;
+
+/* Row logsumexp, the normaliser of every causal softmax row (first of the two
+ * passes; the transposed pass below needs it to normalise without the row).
+ *   q, k        device, bf16, 16-byte aligned, layouts above
+ *   cu_seqlens  HOST int32 [batch + 1]
+ *   scale       softmax scale s (finite; 1/sqrt(head_dim) for the workloads)
+ *   lse         device fp32 [n_q_heads, T], written for every (g, i)
+ *   dev_status  device int32 or NULL; receives a nonzero code if a wait times out
+ */
+KVPOP_API kvpop_status kvpop_row_lse(const void* q, const void* k, const int32_t* cu_seqlens,
+                           kvpop_shape shape, float scale, float* lse,
+                           int32_t* dev_status, void* stream);
+
+/* Future-attention target: the transposed pass.  Each CTA owns a tile of 128
+ * keys of one KV head and streams the query tiles i >= j + W of all G query
+ * heads of its group, so the sum over queries and over the GQA group stays
+ * inside one thread per key (KVpop: "transposed-attention pass", aiweekly
+ * article, second paragraph).
+ *   window      W >= 0, the protected recent window
+ *   lse         device fp32 [n_q_heads, T] from kvpop_row_lse with the same q, k, scale
+ *   target      device fp32 [n_kv_heads, T], written for every (h, j)
+ * other arguments as for kvpop_row_lse. */
+KVPOP_API kvpop_status kvpop_future_target(const void* q, const void* k, const int32_t* cu_seqlens,
+                                 kvpop_shape shape, float scale, int32_t window,
+                                 const float* lse, float* target,
+                                 int32_t* dev_status, void* stream);
+
+/* Sink + top-k + recent-window keep set (model card, introduction; French
+ * article, second paragraph).  Per sequence b and KV head h: keep p < sinks,
+ * keep p >= L - window, and among p in [sinks, L - window) keep the
+ * budget[b] - sinks - window largest scores, equal scores going to the
+ * smaller position first and NaN ranking below every number (-0 equals +0).
+ * Everything is kept when L <= budget[b].
+ *   score    device fp32 [n_kv_heads, T] (any values; normally the target)
+ *   budgets  HOST int32 [batch], each >= sinks + window
+ *   keep     device uint8 [n_kv_heads, T]
+ * This kernel has no on-chip waits and takes no status word. */
+KVPOP_API kvpop_status kvpop_keep_mask(const float* score, const int32_t* cu_seqlens, kvpop_shape shape,
+                             int32_t window, int32_t sinks, const int32_t* budgets,
+                             uint8_t* keep, void* stream);
+
+/* The whole hot path on device buffers: row logsumexp, transposed pass, keep
+ * mask, enqueued back to back on `stream`.  lse is written as a by-product. */
+KVPOP_API kvpop_status kvpop_future_targets(const void* q, const void* k, const int32_t* cu_seqlens,
+                                  kvpop_shape shape, float scale, int32_t window, int32_t sinks,
+                                  const int32_t* budgets, float* lse, float* target,
+                                  uint8_t* keep, int32_t* dev_status, void* stream);
+
+/* Device workspace (bytes) that kvpop_future_targets_host needs for `shape`. */
+KVPOP_API size_t kvpop_host_workspace_bytes(kvpop_shape shape);
+
+/* The whole hot path on HOST buffers: copies q and k (host, preferably pinned)
+ * into `workspace` (device, at least kvpop_host_workspace_bytes(shape) bytes,
+ * 256-byte aligned), runs the three passes and copies target and keep back to
+ * host memory, all enqueued on `stream`.  The results are valid once the
+ * stream has been synchronised. */
+KVPOP_API kvpop_status kvpop_future_targets_host(const void* q_host, const void* k_host,
+                                       const int32_t* cu_seqlens, kvpop_shape shape,
+                                       float scale, int32_t window, int32_t sinks,
+                                       const int32_t* budgets, float* target_host,
+                                       uint8_t* keep_host, void* workspace,
+                                       size_t workspace_bytes, int32_t* dev_status,
+                                       void* stream);
+
+/* Synchronises `stream`, reads *dev_status and maps it: 0 -> KVPOP_OK, a
+ * kernel wait that ran out -> KVPOP_ERR_TIMEOUT.  The word is not cleared. */
+KVPOP_API kvpop_status kvpop_check_device_status(const int32_t* dev_status, void* stream);
+
+/* Self-test of the bounded wait: one CTA waits on an on-chip barrier that
+ * nothing ever completes, gives up after `limit_ns` nanoseconds (1 .. 1e9)
+ * and writes its timeout code into *dev_status.  Used by the tests to show a
+ * wait that runs out ends in an error status, not a hang. */
+KVPOP_API kvpop_status kvpop_selftest_bounded_wait(int32_t* dev_status, uint64_t limit_ns, void* stream);
+
+KVPOP_API const char* kvpop_status_string(kvpop_status status);
+KVPOP_API const char* kvpop_last_error(void);
+KVPOP_API int32_t kvpop_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVPOP_H_ */

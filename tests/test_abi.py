@@ -1,0 +1,127 @@
+"""The C-ABI library on the CPU: it loads, exports every declared symbol, and
+rejects bad arguments before any device call (no GPU needed)."""
+import ctypes
+
+import numpy as np
+import pytest
+
+from future_attention_targets_b200 import _binding as B
+from future_attention_targets_b200.build import build
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return B.lib()
+
+
+def test_exports_every_header_symbol(lib):
+    names = B.header_symbols()
+    assert len(names) == 11, names
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in kvpop.h but not exported"
+    assert set(names) == set(B._SIGS), "binding signatures and header disagree"
+
+
+def test_version_and_strings(lib):
+    assert lib.kvpop_abi_version() == 1
+    for code, word in [(0, b"ok"), (1, b"invalid argument"), (2, b"unsupported"), (3, b"CUDA error"),
+                       (4, b"device wait timed out")]:
+        assert lib.kvpop_status_string(code) == word
+
+
+FAKE = 0x10000  # never dereferenced: every call below fails validation first
+
+
+def _shape(batch=1, T=100, hq=4, hkv=2, d=128):
+    return B.Shape(batch, T, hq, hkv, d)
+
+
+def _cu(*v):
+    return B._i32_host(v)
+
+
+def _row_lse(lib, q=FAKE, k=FAKE, cu=None, shape=None, scale=0.1, lse=FAKE):
+    cu = _cu(0, 100) if cu is None else cu
+    shape = _shape() if shape is None else shape
+    return lib.kvpop_row_lse(q, k, cu, shape, scale, lse, None, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), B.INVALID_ARG),
+    (dict(k=None), B.INVALID_ARG),
+    (dict(lse=None), B.INVALID_ARG),
+    (dict(q=FAKE + 2), B.INVALID_ARG),                       # misaligned
+    (dict(scale=float("nan")), B.INVALID_ARG),
+    (dict(scale=float("inf")), B.INVALID_ARG),
+    (dict(shape=_shape(hq=3, hkv=2)), B.INVALID_ARG),         # H_q not a multiple of H_kv
+    (dict(shape=_shape(hkv=0)), B.INVALID_ARG),
+    (dict(shape=_shape(d=96)), B.UNSUPPORTED),
+    (dict(shape=_shape(d=256)), B.UNSUPPORTED),
+    (dict(shape=_shape(batch=0)), B.INVALID_ARG),
+    (dict(shape=_shape(batch=513), cu=_cu(*([0] * 514))), B.UNSUPPORTED),
+    (dict(shape=_shape(T=99)), B.INVALID_ARG),               # cu[batch] != T
+    (dict(cu=_cu(1, 100)), B.INVALID_ARG),                    # cu[0] != 0
+    (dict(shape=_shape(batch=2), cu=_cu(0, 60, 50)), B.INVALID_ARG),   # decreasing
+    (dict(shape=_shape(T=131073), cu=_cu(0, 131073)), B.UNSUPPORTED),  # sequence too long
+])
+def test_row_lse_rejects(lib, kw, code):
+    assert _row_lse(lib, **kw) == code
+    assert lib.kvpop_last_error()
+
+
+def test_cu_seqlens_null(lib):
+    assert lib.kvpop_row_lse(FAKE, FAKE, None, _shape(), 0.1, FAKE, None, None) == B.INVALID_ARG
+
+
+def test_future_target_rejects(lib):
+    cu, sh = _cu(0, 100), _shape()
+    assert lib.kvpop_future_target(FAKE, FAKE, cu, sh, 0.1, -1, FAKE, FAKE, None, None) == B.INVALID_ARG
+    assert lib.kvpop_future_target(FAKE, FAKE, cu, sh, 0.1, 4, None, FAKE, None, None) == B.INVALID_ARG
+    assert lib.kvpop_future_target(FAKE, FAKE, cu, sh, 0.1, 4, FAKE, None, None, None) == B.INVALID_ARG
+
+
+def test_keep_mask_rejects(lib):
+    cu, sh = _cu(0, 100), _shape()
+    bud = _cu(50)
+    assert lib.kvpop_keep_mask(None, cu, sh, 16, 4, bud, FAKE, None) == B.INVALID_ARG
+    assert lib.kvpop_keep_mask(FAKE, cu, sh, 16, 4, None, FAKE, None) == B.INVALID_ARG
+    assert lib.kvpop_keep_mask(FAKE, cu, sh, 16, 4, _cu(19), FAKE, None) == B.INVALID_ARG   # < sinks + window
+    assert lib.kvpop_keep_mask(FAKE, cu, sh, -1, 4, bud, FAKE, None) == B.INVALID_ARG
+    assert lib.kvpop_keep_mask(FAKE, cu, sh, 16, -4, bud, FAKE, None) == B.INVALID_ARG
+
+
+def test_pipeline_rejects(lib):
+    cu, sh = _cu(0, 100), _shape()
+    bud = _cu(50)
+    assert lib.kvpop_future_targets(FAKE, FAKE, cu, sh, 0.1, 16, 4, _cu(10), FAKE, FAKE, FAKE, None,
+                                    None) == B.INVALID_ARG
+    need = lib.kvpop_host_workspace_bytes(sh)
+    assert lib.kvpop_future_targets_host(FAKE, FAKE, cu, sh, 0.1, 16, 4, bud, FAKE, FAKE, FAKE, need - 1, None,
+                                         None) == B.INVALID_ARG
+    assert lib.kvpop_future_targets_host(FAKE, FAKE, cu, sh, 0.1, 16, 4, bud, FAKE, FAKE, FAKE + 16, need, None,
+                                         None) == B.INVALID_ARG
+    assert lib.kvpop_check_device_status(None, None) == B.INVALID_ARG
+    assert lib.kvpop_selftest_bounded_wait(FAKE, 0, None) == B.INVALID_ARG
+    assert lib.kvpop_selftest_bounded_wait(None, 1000, None) == B.INVALID_ARG
+
+
+def test_workspace_bytes(lib):
+    sh = B.Shape(1, 16384, 32, 8, 128)
+    r = lambda x: (x + 255) // 256 * 256
+    T = 16384
+    want = r(T * 32 * 128 * 2) + r(T * 8 * 128 * 2) + r(T * 32 * 4) + r(T * 8 * 4) + r(T * 8)
+    assert lib.kvpop_host_workspace_bytes(sh) == want
+    assert lib.kvpop_host_workspace_bytes(B.Shape(1, 0, 32, 8, 128)) == 0
+
+
+def test_empty_input_is_a_no_op(lib):
+    # T = 0: valid, nothing to enqueue, no device call.
+    assert lib.kvpop_row_lse(FAKE, FAKE, _cu(0, 0), B.Shape(1, 0, 4, 2, 128), 0.1, FAKE, None, None) == B.OK
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(B, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(B, "_handle", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        B.lib()

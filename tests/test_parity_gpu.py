@@ -1,0 +1,275 @@
+"""CUDA path (through the C ABI) against the CPU float64 oracle.
+
+Targets must satisfy max_j |gpu - oracle| / max(|oracle_j|, 1e-3) <= 2e-3;
+the keep mask must equal, bit for bit, the oracle's keep mask computed from
+the same fp32 scores (the GPU's targets).  Small shapes are compared
+element by element; the full-size workloads on sampled outputs the oracle
+can compute (key blocks near the end of each sequence, whose targets need
+only the last rows; logsumexp of sampled rows), plus closed forms and
+invariants that hold at any size.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from future_attention_targets_b200 import (KvpopError, check_status, future_target, future_targets, keep_mask,
+                                           row_lse, selftest_bounded_wait)
+from future_attention_targets_b200 import _binding as B
+from future_attention_targets_b200.workloads import WORKLOADS, make_inputs, random_qk
+
+pytestmark = pytest.mark.gpu
+
+TARGET_TOL = 2e-3       # elementwise relative error bound on the targets (floor 1e-3)
+LSE_TOL = 1e-4          # absolute error on the natural-log row logsumexp
+
+
+def rel_err(gpu, ref):
+    gpu, ref = np.asarray(gpu, np.float64), np.asarray(ref, np.float64)
+    if gpu.size == 0:
+        return 0.0
+    return float(np.max(np.abs(gpu - ref) / np.maximum(np.abs(ref), 1e-3)))
+
+
+def dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def run_gpu(q_bits, k_bits, cu, W, S, budgets, scale):
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lse, tgt, keep = future_targets(dev(q_bits), dev(k_bits), cu, W, S, budgets, scale=scale, status=status)
+    check_status(status)
+    return lse.cpu().numpy(), tgt.cpu().numpy(), keep.cpu().numpy()
+
+
+_CACHE = {}
+
+
+def workload(name):
+    if name not in _CACHE:
+        d = make_inputs(name)
+        lse, tgt, keep = run_gpu(d["q_bits"], d["k_bits"], d["cu_seqlens"], d["window"], d["sinks"], d["budgets"],
+                                 d["scale"])
+        _CACHE[name] = (d, lse, tgt, keep)
+    return _CACHE[name]
+
+
+def assert_keep_exact(d, tgt, keep):
+    ref = oracle.keep_mask(tgt, d["cu_seqlens"], d["window"], d["sinks"], d["budgets"])
+    np.testing.assert_array_equal(keep, ref)
+    cu = d["cu_seqlens"]
+    for b in range(len(cu) - 1):
+        L = int(cu[b + 1] - cu[b])
+        assert np.all(keep[:, cu[b]:cu[b + 1]].sum(axis=1) == min(int(d["budgets"][b]), L))
+
+
+# ------------------------------------------------------------------ full comparisons
+
+@pytest.mark.parametrize("name", ["tiny", "qwen3_4b_4k"])
+def test_full_parity(name):
+    d, lse, tgt, keep = workload(name)
+    ref_tgt, ref_lse = oracle.future_target(d["q_bits"], d["k_bits"], d["cu_seqlens"], d["window"], d["scale"],
+                                            return_lse=True)
+    assert rel_err(tgt, ref_tgt) <= TARGET_TOL
+    assert np.max(np.abs(lse - ref_lse)) <= LSE_TOL
+    assert np.all(tgt[:, -d["window"]:] == 0)
+    assert_keep_exact(d, tgt, keep)
+
+
+EDGE = [
+    # seqlens, H_q, H_kv, d, W, gain
+    ((1,), 2, 1, 128, 0, 1.0),
+    ((1,), 2, 1, 64, 4, 1.0),
+    ((127, 129, 255, 257, 300), 4, 2, 128, 16, 2.0),
+    ((255, 256, 257), 8, 1, 64, 255, 2.0),
+    ((600,), 4, 4, 128, 0, 3.0),
+    ((1000, 0, 513), 8, 2, 128, 700, 2.0),
+    ((384, 640), 16, 2, 128, 128, 2.0),
+    ((2000,), 2, 1, 64, 2000, 1.0),
+    ((1537, 90, 4), 4, 1, 128, 37, 4.0),
+]
+
+
+@pytest.mark.parametrize("case", EDGE, ids=[f"L{c[0]}-G{c[1] // c[2]}-d{c[3]}-W{c[4]}" for c in EDGE])
+def test_edge_shapes(case):
+    seqlens, hq, hkv, d, W, gain = case
+    T = sum(seqlens)
+    q_bits, k_bits = random_qk(T, hq, hkv, d, seed=T + W, gain=gain)
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    budgets = [W + 4 + 7] * len(seqlens)
+    scale = 1.0 / math.sqrt(d)
+    lse, tgt, keep = run_gpu(q_bits, k_bits, cu, W, 4, budgets, scale)
+    ref_tgt, ref_lse = oracle.future_target(q_bits, k_bits, cu, W, scale, return_lse=True)
+    assert rel_err(tgt, ref_tgt) <= TARGET_TOL
+    assert np.max(np.abs(lse - ref_lse), initial=0.0) <= LSE_TOL
+    np.testing.assert_array_equal(keep, oracle.keep_mask(tgt, cu, W, 4, budgets))
+
+
+# ------------------------------------------------------------------ full size: closed forms, invariants
+
+def _harmonic_tail(L):
+    inv = 1.0 / np.arange(1, L + 1, dtype=np.float64)
+    return np.concatenate([np.cumsum(inv[::-1])[::-1], [0.0]])
+
+
+def test_zero_keys_closed_form_16k():
+    """All-zero keys: A[i, j] = 1/(i+1), so target_j = G sum_{i >= j+W} 1/(i+1) and lse_i = ln(i+1)."""
+    w = WORKLOADS["qwen3_8b_16k"]
+    L = w.seqlen
+    q_bits, k_bits = random_qk(L, w.n_q_heads, w.n_kv_heads, w.head_dim, seed=3, k_zero=True)
+    cu = np.array([0, L], dtype=np.int32)
+    lse, tgt, _ = run_gpu(q_bits, k_bits, cu, w.window, w.sinks, [w.budget], 1.0 / math.sqrt(w.head_dim))
+    tail = _harmonic_tail(L)
+    expect = w.group * tail[np.minimum(np.arange(L) + w.window, L)]
+    assert rel_err(tgt, np.broadcast_to(expect, tgt.shape)) <= TARGET_TOL
+    assert np.max(np.abs(lse - np.log(np.arange(1, L + 1))[None, :])) <= LSE_TOL
+
+
+def test_row_stochastic_16k():
+    """W = 0: every query row sums to one, so sum_j target[h, j] = G * L (at the full 16k size)."""
+    d = make_inputs("qwen3_8b_16k")
+    w = d["workload"]
+    lse, tgt, _ = run_gpu(d["q_bits"], d["k_bits"], d["cu_seqlens"], 0, 0, [w.seqlen], d["scale"])
+    sums = tgt.astype(np.float64).sum(axis=1)
+    np.testing.assert_allclose(sums, w.group * w.seqlen, rtol=1e-4)
+
+
+# ------------------------------------------------------------------ full size: sampled outputs
+
+def _sampled_check(name, tail_keys, n_lse_rows, kv_heads=None, mid_block=False):
+    d, lse, tgt, keep = workload(name)
+    w = d["workload"]
+    G = w.group
+    heads = range(w.n_kv_heads) if kv_heads is None else kv_heads
+    cu = d["cu_seqlens"]
+    rng = np.random.default_rng(7)
+    for h in heads:
+        for b in range(len(cu) - 1):
+            s0, s1 = int(cu[b]), int(cu[b + 1])
+            L = s1 - s0
+            qh = d["q_bits"][s0:s1, h * G:(h + 1) * G]
+            kh = d["k_bits"][s0:s1, h:h + 1]
+            key_lo = max(0, L - w.window - tail_keys)
+            ref = oracle.future_target(qh, kh, np.array([0, L], dtype=np.int32), w.window, d["scale"],
+                                       key_lo=key_lo)
+            assert rel_err(tgt[h, s0 + key_lo:s1], ref[0, key_lo:]) <= TARGET_TOL, f"KV head {h}, sequence {b}"
+        rows = np.sort(rng.choice(int(cu[-1]), size=n_lse_rows, replace=False))
+        qh = d["q_bits"][:, h * G:(h + 1) * G]
+        kh = d["k_bits"][:, h:h + 1]
+        ref_l = oracle.row_lse(qh, kh, cu, d["scale"], rows=rows)
+        assert np.max(np.abs(lse[h * G:(h + 1) * G][:, rows] - ref_l[:, rows])) <= LSE_TOL
+    if mid_block:
+        # A block of keys in the middle of the sequence, one KV head.
+        L = int(cu[1])
+        j_lo = L // 2
+        qh, kh = d["q_bits"][:, :G], d["k_bits"][:, :1]
+        ref = oracle.future_target(qh, kh, cu, w.window, d["scale"], key_lo=j_lo)
+        assert rel_err(tgt[0, j_lo:L], ref[0, j_lo:L]) <= TARGET_TOL
+    assert_keep_exact(d, tgt, keep)
+
+
+def test_16k_sampled():
+    _sampled_check("qwen3_8b_16k", tail_keys=512, n_lse_rows=48, mid_block=True)
+
+
+def test_varlen_sampled():
+    _sampled_check("varlen_8x", tail_keys=256, n_lse_rows=32, kv_heads=[0, 5])
+
+
+def test_64k_sampled():
+    _sampled_check("long_64k", tail_keys=192, n_lse_rows=16, kv_heads=[2, 7])
+
+
+def test_64k_invariants():
+    """Targets are non-negative, zero in the last W positions, and no key gets more than G * (L - j - W)."""
+    d, lse, tgt, keep = workload("long_64k")
+    w = d["workload"]
+    L = w.seqlen
+    assert np.all(np.isfinite(tgt)) and np.all(tgt >= 0)
+    assert np.all(tgt[:, L - w.window:] == 0)
+    cap = w.group * np.maximum(L - np.arange(L) - w.window, 0)
+    assert np.all(tgt <= cap[None, :] * (1 + 1e-5) + 1e-6)
+    assert np.all(np.isfinite(lse))
+
+
+# ------------------------------------------------------------------ keep mask alone
+
+def test_keep_mask_edge_cases():
+    rng = np.random.default_rng(5)
+    seqlens = (12, 400, 37, 250, 300, 5000)
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    T = int(cu[-1])
+    W, S = 16, 4
+    budgets = [30, 100, 60, 250, 20, 1000]
+    score = rng.random((3, T)).astype(np.float32)
+    score[0, ::7] = 0.5
+    score[1, 12 + 50:12 + 150] = 2.0
+    score[2, 30] = np.nan
+    score[2, 31] = -0.0
+    score[2, 32] = 0.0
+    score[2, 33] = np.inf
+    score[2, 34] = -np.inf
+    score[1, 1000:2000] = -1.5
+    score[0, 2000:] = 0.25        # the whole long sequence of head 0 ties
+    out = keep_mask(torch.from_numpy(score).cuda(), cu, W, S, budgets).cpu().numpy()
+    np.testing.assert_array_equal(out, oracle.keep_mask(score, cu, W, S, budgets))
+
+
+# ------------------------------------------------------------------ determinism, errors, host path
+
+def test_deterministic():
+    d = make_inputs("qwen3_4b_4k")
+    a = run_gpu(d["q_bits"], d["k_bits"], d["cu_seqlens"], d["window"], d["sinks"], d["budgets"], d["scale"])
+    for _ in range(3):
+        b = run_gpu(d["q_bits"], d["k_bits"], d["cu_seqlens"], d["window"], d["sinks"], d["budgets"], d["scale"])
+        for x, y in zip(a, b):
+            np.testing.assert_array_equal(x, y)
+
+
+def test_separate_calls_match_pipeline():
+    d, lse, tgt, keep = workload("qwen3_4b_4k")
+    q, k = dev(d["q_bits"]), dev(d["k_bits"])
+    l2 = row_lse(q, k, d["cu_seqlens"], d["scale"])
+    t2 = future_target(q, k, d["cu_seqlens"], d["window"], l2, d["scale"])
+    k2 = keep_mask(t2, d["cu_seqlens"], d["window"], d["sinks"], d["budgets"])
+    np.testing.assert_array_equal(l2.cpu().numpy(), lse)
+    np.testing.assert_array_equal(t2.cpu().numpy(), tgt)
+    np.testing.assert_array_equal(k2.cpu().numpy(), keep)
+
+
+def test_host_pipeline_matches_device():
+    d, lse, tgt, keep = workload("qwen3_4b_4k")
+    w = d["workload"]
+    pipe = B.HostPipeline(d["cu_seqlens"], w.n_q_heads, w.n_kv_heads, w.head_dim, w.window, w.sinks, d["budgets"],
+                          d["scale"])
+    qh = torch.from_numpy(d["q_bits"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    kh = torch.from_numpy(d["k_bits"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    t_h, k_h = pipe(qh, kh)
+    np.testing.assert_array_equal(t_h.numpy(), tgt)
+    np.testing.assert_array_equal(k_h.numpy(), keep)
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    selftest_bounded_wait(status, 50_000_000)          # 50 ms on a barrier nothing completes
+    with pytest.raises(KvpopError) as ei:
+        check_status(status)
+    assert ei.value.status == B.TIMEOUT
+    # The context is still usable afterwards.
+    d = make_inputs("tiny")
+    lse, tgt, keep = run_gpu(d["q_bits"], d["k_bits"], d["cu_seqlens"], d["window"], d["sinks"], d["budgets"],
+                             d["scale"])
+    ref = oracle.future_target(d["q_bits"], d["k_bits"], d["cu_seqlens"], d["window"], d["scale"])
+    assert rel_err(tgt, ref) <= TARGET_TOL
+
+
+def test_binding_rejects_bad_tensors():
+    q = torch.zeros((10, 4, 128), dtype=torch.float16, device="cuda")
+    k = torch.zeros((10, 2, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(TypeError):
+        row_lse(q, k, [0, 10])
+    with pytest.raises(KvpopError) as ei:
+        row_lse(q.bfloat16(), k, [0, 9])                 # cu_seqlens[batch] != T
+    assert ei.value.status == B.INVALID_ARG
