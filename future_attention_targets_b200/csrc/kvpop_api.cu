@@ -146,7 +146,7 @@ kvpop_status check_shape(const int32_t* cu, const kvpop_shape& sh, bool need_hea
 kvpop_status check_qk(const void* q, const void* k, float scale) {
   if (q == nullptr || k == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "q or k is NULL");
   if (!aligned16(q) || !aligned16(k)) return fail(KVPOP_ERR_INVALID_ARG, "q and k must be 16-byte aligned");
-  if (!isfinite(scale)) return fail(KVPOP_ERR_INVALID_ARG, "scale must be finite");
+  if (!isfinite(scale) || !(scale > 0.f)) return fail(KVPOP_ERR_INVALID_ARG, "scale must be finite and > 0");
   return KVPOP_OK;
 }
 
@@ -204,6 +204,7 @@ kvpop_status fill_attn_common(AttnParams* p, const void* q, const void* k, const
   p->n_kv_heads = sh.n_kv_heads;
   p->group = sh.n_q_heads / sh.n_kv_heads;
   p->scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p->inv_scale = static_cast<float>(1.0 / static_cast<double>(scale));
   build_schedule(cu, sh.batch, target_pass ? sh.n_kv_heads : sh.n_q_heads, &p->sched);
   return KVPOP_OK;
 }

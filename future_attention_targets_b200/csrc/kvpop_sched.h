@@ -42,6 +42,7 @@ struct AttnParams {
   int32_t group;
   int32_t window;
   float scale_log2;       // softmax scale * log2(e)
+  float inv_scale;        // 1 / softmax scale (pass 2 normaliser slab)
   LevelSchedule sched;
 };
 

@@ -85,7 +85,7 @@ typedef struct {
  * passes; the transposed pass below needs it to normalise without the row).
  *   q, k        device, bf16, 16-byte aligned, layouts above
  *   cu_seqlens  HOST int32 [batch + 1]
- *   scale       softmax scale s (finite; 1/sqrt(head_dim) for the workloads)
+ *   scale       softmax scale s (finite, > 0; 1/sqrt(head_dim) for the workloads)
  *   lse         device fp32 [n_q_heads, T], written for every (g, i)
  *   dev_status  device int32 or NULL; receives a nonzero code if a wait times out
  */

@@ -54,6 +54,8 @@ def _row_lse(lib, q=FAKE, k=FAKE, cu=None, shape=None, scale=0.1, lse=FAKE):
     (dict(q=FAKE + 2), B.INVALID_ARG),                       # misaligned
     (dict(scale=float("nan")), B.INVALID_ARG),
     (dict(scale=float("inf")), B.INVALID_ARG),
+    (dict(scale=0.0), B.INVALID_ARG),
+    (dict(scale=-0.1), B.INVALID_ARG),
     (dict(shape=_shape(hq=3, hkv=2)), B.INVALID_ARG),         # H_q not a multiple of H_kv
     (dict(shape=_shape(hkv=0)), B.INVALID_ARG),
     (dict(shape=_shape(d=96)), B.UNSUPPORTED),
