@@ -173,6 +173,29 @@ def oracle_sample(d, rows: int | None, kv_head: int = 0):
     return time.perf_counter() - t0, fl, desc
 
 
+# ------------------------------------------------------------------ multi-rank helpers
+
+def rank_seed(rank: int) -> int:
+    """Each rank runs its own independent layer: the workload seed is the rank."""
+    return int(rank)
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank number over the process group (identity without one)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_throughput(flops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: the work of every rank over the slowest rank's step time."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ reference arm (CPU oracle)
 
 def run_reference(args):
@@ -232,7 +255,7 @@ def run_ours(args):
         dist.barrier()
     lib()
 
-    d = make_inputs(WORKLOAD, seed=rank)   # an independent layer per rank
+    d = make_inputs(WORKLOAD, seed=rank_seed(rank))   # an independent layer per rank
     w = d["workload"]
     cu, W, S, budgets, scale = d["cu_seqlens"], d["window"], d["sinks"], d["budgets"], d["scale"]
     q = torch.from_numpy(d["q_bits"].view(np.int16)).view(torch.bfloat16).to(dev)
@@ -279,14 +302,11 @@ def run_ours(args):
     elapsed_ms = t_start.elapsed_time(t_end)
     per_kernel = {name: [e[j].elapsed_time(e[j + 1]) for e in evs]
                   for j, name in enumerate(["row_lse", "future_target", "keep_mask"])}
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dev)
 
     fl = algorithmic_flops([w.seqlen], w.n_q_heads, w.head_dim, w.window)
     ms_per_step = elapsed_ms / args.steps
-    value = fl["total"] * world / (ms_per_step * 1e-3) / 1e12
+    value = weak_throughput(fl["total"], world, ms_per_step)
     peaks, peak_kind = load_peaks()
     peak = float(peaks["bf16_tflops"])
     peak_sus = float(peaks.get("bf16_tflops_sustained", peak))
@@ -315,12 +335,8 @@ def run_ours(args):
             pipe(qh, kh, stream)   # synchronises the stream after each step (results on the host)
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": fl["total"] * world / (e_ms / n_e2e * 1e-3) / 1e12, "unit": UNIT,
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+        e2e = {"value": weak_throughput(fl["total"], world, e_ms / n_e2e), "unit": UNIT,
                "h2d_bytes_per_step": pipe.h2d_bytes, "d2h_bytes_per_step": pipe.d2h_bytes,
                "ms_per_step": e_ms / n_e2e, "steps": n_e2e}
         del pipe
