@@ -227,7 +227,7 @@ struct TileCursor {
 // Every lane waits; the outcome is made warp-uniform so that warp-collective
 // instructions that follow never run in a partial warp.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl, int32_t site) {
-  const bool ok = wait_bounded(bar, parity, ctl, site);
+  const bool ok = mbar_try_wait(bar, parity) || wait_bounded(bar, parity, ctl, site);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -459,32 +459,68 @@ __device__ __forceinline__ uint64_t exp2_poly_pair(uint64_t y) {
   return f2_pack(__uint_as_float(b0), __uint_as_float(b1));
 }
 
+// 2^(c x) for a pair with the scale folded into the range reduction:
+// x is clamped so that c x >= -126, then t = rm(c x + 1.5 * 2^23) in one
+// fused multiply-add, n = t - 1.5 * 2^23 = floor(c x), f = c x - n (exact).
+__device__ __forceinline__ uint64_t exp2_poly_pair_scaled(uint64_t x, uint64_t c2, float xmin) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, xmin), fmaxf(x1, xmin));
+  uint64_t t;
+  asm("fma.rm.ftz.f32x2 %0, %1, %2, %3;" : "=l"(t) : "l"(xc), "l"(c2), "l"(f2_pack(kRoundMagic, kRoundMagic)));
+  const uint64_t n = f2_add(t, f2_pack(-kRoundMagic, -kRoundMagic));
+  float n0, n1;
+  f2_unpack(n, n0, n1);
+  const uint64_t f = f2_fma(xc, c2, f2_pack(-n0, -n1));
+  uint64_t q = f2_fma(f, f2_pack(kP4, kP4), f2_pack(kP3, kP3));
+  q = f2_fma(q, f, f2_pack(kP2, kP2));
+  q = f2_fma(q, f, f2_pack(kP1, kP1));
+  q = f2_fma(q, f, f2_pack(1.f, 1.f));
+  float t0, t1, q0, q1;
+  f2_unpack(t, t0, t1);
+  f2_unpack(q, q0, q1);
+  const uint32_t b0 = __float_as_uint(q0) + __float_as_uint(t0) * (1u << 23);
+  const uint32_t b1 = __float_as_uint(q1) + __float_as_uint(t1) * (1u << 23);
+  return f2_pack(__uint_as_float(b0), __uint_as_float(b1));
+}
+
 __device__ __forceinline__ uint64_t exp2_mufu_pair(uint64_t y) {
   float y0, y1;
   f2_unpack(y, y0, y1);
   return f2_pack(ex2_approx(y0), ex2_approx(y1));
 }
 
-// Split between the exponent paths, pairs per 8 on the polynomial (measured
-// best on B200 for each pass at the Qwen3-8B 16k shape).
-#ifndef KVPOP_POLY_PAIRS_LSE
-#define KVPOP_POLY_PAIRS_LSE 3
+// Split between the exponent paths: pairs (of the 16 in a 32-column chunk)
+// evaluated by the polynomial, spread evenly over the chunk (measured on
+// B200 for each pass at the Qwen3-8B 16k shape).
+#ifndef KVPOP_POLY16_LSE
+#define KVPOP_POLY16_LSE 4
 #endif
-#ifndef KVPOP_POLY_PAIRS_TARGET
-#define KVPOP_POLY_PAIRS_TARGET 2
+#ifndef KVPOP_POLY16_TARGET
+#define KVPOP_POLY16_TARGET 4
 #endif
 
-// acc += exp2(x * c + nb) over one 32-column chunk (nb: one negated offset
-// for the whole chunk); in every group of 8 pairs the first kPoly go through
-// the polynomial, the rest through MUFU.
 template <int kPoly>
-__device__ __forceinline__ void chunk_exp_sum(const uint32_t (&r)[32], uint64_t c2, uint64_t nb,
+__device__ __forceinline__ constexpr bool poly_pair(int q) {
+  return ((q * kPoly) & 15) < kPoly;
+}
+
+// acc += exp2(x * c + nb) over one 32-column chunk (nb: one negated offset
+// for the whole chunk); kPoly of the 16 pairs go through the polynomial, the
+// rest through MUFU.  kBiasFree: nb is zero (pass 2), the scale is folded
+// into the polynomial's range reduction and x >= xmin keeps c x >= -126.
+template <int kPoly, bool kBiasFree>
+__device__ __forceinline__ void chunk_exp_sum(const uint32_t (&r)[32], uint64_t c2, uint64_t nb, float xmin,
                                               uint64_t (&acc)[4]) {
 #pragma unroll
   for (int q = 0; q < 16; ++q) {
     const uint64_t x = f2_pack(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
-    const uint64_t y = f2_fma(x, c2, nb);
-    const uint64_t e = ((q & 7) < kPoly) ? exp2_poly_pair(y) : exp2_mufu_pair(y);
+    uint64_t e;
+    if (poly_pair<kPoly>(q)) {
+      e = kBiasFree ? exp2_poly_pair_scaled(x, c2, xmin) : exp2_poly_pair(f2_fma(x, c2, nb));
+    } else {
+      e = exp2_mufu_pair(f2_fma(x, c2, nb));
+    }
     acc[q & 3] = f2_add(acc[q & 3], e);
   }
 }
@@ -515,27 +551,28 @@ __device__ __forceinline__ float acc_total(uint64_t (&acc)[4]) {
 // Sum of exp2(x * c - off) over the 128 columns of this thread's TMEM lane
 // starting at taddr: four chunks of 32, the load of chunk c+1 in flight
 // while chunk c is summed.  kMasked: column m counts iff lo <= m < hi.
-template <bool kMasked, int kPoly>
-__device__ __forceinline__ float half_tile_exp_sum(uint32_t taddr, uint64_t c2, uint64_t nb, int lo, int hi) {
+template <bool kMasked, int kPoly, bool kBiasFree = false>
+__device__ __forceinline__ float half_tile_exp_sum(uint32_t taddr, uint64_t c2, uint64_t nb, int lo, int hi,
+                                                   float xmin = 0.f) {
   uint32_t ra[32], rb[32];
   uint64_t acc[4] = {0, 0, 0, 0};
   auto run = [&](const uint32_t (&r)[32], int ch) {
     if constexpr (kMasked)
       chunk_exp_sum_masked(r, c2, nb, lo - 32 * ch, hi - 32 * ch, acc);
     else
-      chunk_exp_sum<kPoly>(r, c2, nb, acc);
+      chunk_exp_sum<kPoly, kBiasFree>(r, c2, nb, xmin, acc);
   };
-  tmem_load32(taddr, ra);
-  tmem_load_wait(ra);
-  tmem_load32(taddr + 32, rb);
+  tmem_load<32>(taddr, ra);
+  tmem_load_wait<32>(ra);
+  tmem_load<32>(taddr + 32, rb);
   run(ra, 0);
-  tmem_load_wait(rb);
-  tmem_load32(taddr + 64, ra);
+  tmem_load_wait<32>(rb);
+  tmem_load<32>(taddr + 64, ra);
   run(rb, 1);
-  tmem_load_wait(ra);
-  tmem_load32(taddr + 96, rb);
+  tmem_load_wait<32>(ra);
+  tmem_load<32>(taddr + 96, rb);
   run(ra, 2);
-  tmem_load_wait(rb);
+  tmem_load_wait<32>(rb);
   run(rb, 3);
   return acc_total(acc);
 }
@@ -546,8 +583,8 @@ __device__ __forceinline__ float half_tile_max(uint32_t taddr, float c, int lo, 
 #pragma unroll 1
   for (int ch = 0; ch < 4; ++ch) {
     uint32_t r[32];
-    tmem_load32(taddr + 32 * ch, r);
-    tmem_load_wait(r);
+    tmem_load<32>(taddr + 32 * ch, r);
+    tmem_load_wait<32>(r);
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       const int col = 32 * ch + e;
@@ -601,7 +638,7 @@ __device__ void lse_softmax_role(const AttnParams& p, uint8_t* smem, const Bars&
         if (!rescale) {
           const uint64_t nb = f2_pack(-off, -off);
           ts = masked ? half_tile_exp_sum<true, 0>(taddr, c2, nb, 0, hi)
-                      : half_tile_exp_sum<false, KVPOP_POLY_PAIRS_LSE>(taddr, c2, nb, 0, 128);
+                      : half_tile_exp_sum<false, KVPOP_POLY16_LSE>(taddr, c2, nb, 0, 128);
           rescale = !(ts < kBig);
         }
         // Warp-uniform: the rescale path issues warp-collective TMEM loads.
@@ -614,7 +651,7 @@ __device__ void lse_softmax_role(const AttnParams& p, uint8_t* smem, const Bars&
           }
           const uint64_t nb = f2_pack(-off, -off);
           ts = masked ? half_tile_exp_sum<true, 0>(taddr, c2, nb, 0, hi)
-                      : half_tile_exp_sum<false, KVPOP_POLY_PAIRS_LSE>(taddr, c2, nb, 0, 128);
+                      : half_tile_exp_sum<false, KVPOP_POLY16_LSE>(taddr, c2, nb, 0, 128);
           if (!(off > -INFINITY)) ts = 0.f;
         }
         sum += ts;
@@ -666,6 +703,7 @@ __device__ void target_softmax_role(const AttnParams& p, uint8_t* smem, const Ba
   float* comb = reinterpret_cast<float*>(smem + L::OFF_COMB);
   const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
   const uint64_t zero2 = f2_pack(0.f, 0.f);
+  const float xmin = -126.f / p.scale_log2;   // below it exp2(c x) < 2^-126: clamp for the polynomial
   const int32_t total = p.sched.total_items;
   uint32_t acc_cnt = 0, item_cnt = 0;
   bool ok = true;
@@ -690,7 +728,8 @@ __device__ void target_softmax_role(const AttnParams& p, uint8_t* smem, const Ba
         const bool ragged = (qt == it.nq - 1) && ragged_end;
         const float ts = (diag || ragged)
                              ? half_tile_exp_sum<true, 0>(taddr, c2, zero2, diag ? row : 0, 128)
-                             : half_tile_exp_sum<false, KVPOP_POLY_PAIRS_TARGET>(taddr, c2, zero2, 0, 128);
+                             : half_tile_exp_sum<false, KVPOP_POLY16_TARGET, true>(taddr, c2, zero2, 0, 128,
+                                                                                      xmin);
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.acc_empty[acc]);
