@@ -28,6 +28,15 @@ materialised causal softmax (one block of query rows at a time):
   keep the k = budget - S - W largest scores; equal scores go to the
   smaller position first.  Everything is kept when L <= budget.
 
+* Prefix top-k thresholds (model card, "Usage" note: the scorer's "prefix
+  top-k thresholds").  At decoding step t the tokens p in [S, t - W] have
+  left the recent window and compete for the k = budget - S - W scored
+  slots.  The threshold of step t is the k-th best of them under the
+  keep-set order (higher score first, then smaller position); a token is
+  kept at step t iff it ranks at or above the threshold.  With fixed scores
+  this is exactly online eviction of the worst token whenever the scored
+  slots overflow, and at the last step it gives the keep mask above.
+
 Readings taken where the pages are silent: the window condition is
 ``i >= j + W``; the GQA group is summed (not averaged) with consecutive
 grouping ``g // G``; the softmax normaliser is the full causal row (sinks
@@ -42,7 +51,7 @@ from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["as_f64", "row_lse", "future_target", "keep_mask", "ROW_BLOCK"]
+__all__ = ["as_f64", "row_lse", "future_target", "keep_mask", "prefix_topk_thresholds", "ROW_BLOCK"]
 
 ROW_BLOCK = 256  # query rows materialised at once
 
@@ -183,3 +192,42 @@ def keep_mask(score, cu_seqlens, window: int, sinks: int, budgets) -> np.ndarray
             order = np.lexsort((pos, -sc))                      # -score ascending, then position
             keep[h, s + pos[order[:k_top]]] = 1
     return keep
+
+
+def prefix_topk_thresholds(score, cu_seqlens, window: int, sinks: int, budgets):
+    """Per-step eviction thresholds, (thr_score float32 [H_kv, T], thr_pos int32 [H_kv, T]).
+
+    For step t of a sequence (t relative to its start) the candidates are the
+    positions p in [S, t - W].  With k = budget - S - W:
+      * fewer than k candidates (or none): no eviction yet, thr = (-inf, -1);
+      * k = 0 and at least one candidate: nothing is kept, thr = (+inf, -1);
+      * otherwise thr = (score, position) of the k-th best candidate in the
+        order (-score, position), NaN scores last.
+    """
+    score = np.asarray(score, dtype=np.float32)
+    Hkv, T = score.shape
+    thr_s = np.full((Hkv, T), -np.inf, dtype=np.float32)
+    thr_p = np.full((Hkv, T), -1, dtype=np.int32)
+    budgets = np.asarray(budgets, dtype=np.int64)
+    W, S = int(window), int(sinks)
+    for b, (s0, L) in enumerate(_sequences(cu_seqlens)):
+        k_top = int(budgets[b]) - S - W
+        if k_top < 0:
+            raise ValueError("budget below sinks + window")
+        for h in range(Hkv):
+            for t in range(L):
+                hi = t - W                                     # last candidate position
+                if hi < S:
+                    continue
+                pos = np.arange(S, hi + 1)
+                if k_top == 0:
+                    thr_s[h, s0 + t] = np.inf
+                    continue
+                if len(pos) < k_top:
+                    continue
+                sc = score[h, s0 + S:s0 + hi + 1].astype(np.float64)
+                order = np.lexsort((pos, -sc))
+                kth = order[k_top - 1]
+                thr_s[h, s0 + t] = score[h, s0 + pos[kth]]
+                thr_p[h, s0 + t] = pos[kth]
+    return thr_s, thr_p

@@ -270,3 +270,87 @@ ALL_PINS = [
     pin_budget_from_pages,
     pin_restrictions,
 ]
+
+
+# ------------------------------------------------------------ prefix top-k thresholds
+
+def online_eviction(score_row, L, W, S, k_top):
+    """Token-by-token online eviction with a heap (independent of the oracle):
+    the scored slots hold at most k_top of the tokens that have left the
+    window; when they overflow, the worst (lowest score, then larger position,
+    NaN lowest) is evicted.  Returns the kept set after each step."""
+    import heapq
+    heap, kept, evicted, out = [], set(), set(), []
+    for t in range(L):
+        p = t - W
+        if p >= S:
+            x = float(score_row[p])
+            # heap entry orders "worse" first: (nan flag inverted, score, -position)
+            key = (0 if math.isnan(x) else 1, 0.0 if math.isnan(x) else x, -p)
+            heapq.heappush(heap, (key, p))
+            kept.add(p)
+            while len(kept) > k_top:
+                _, q = heapq.heappop(heap)
+                kept.discard(q)
+                evicted.add(q)
+        out.append(set(kept))
+    return out
+
+
+def _rank_at_or_above(x, p, ts, tp):
+    """(x, p) ranks at or above the threshold (ts, tp) in the keep-set order."""
+    xn, tn = math.isnan(x), math.isnan(ts)
+    if tn and xn:
+        return p <= tp
+    if tn:
+        return True
+    if xn:
+        return False
+    return x > ts or (x == ts and p <= tp)
+
+
+def pin_prefix_thresholds(orc):
+    rng = np.random.default_rng(31)
+    seqlens = (70, 9, 130, 45)
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    T = int(cu[-1])
+    W, S = 6, 3
+    budgets = [W + S + 10, W + S + 3, W + S + 25, W + S]          # last: k = 0
+    score = rng.random((2, T)).astype(np.float32)
+    score[0, ::5] = 0.25                                          # ties
+    score[1, 20:40] = 0.75
+    score[1, 50] = np.nan
+    thr_s, thr_p = orc.prefix_topk_thresholds(score, cu, W, S, budgets)
+    keep_final = orc.keep_mask(score, cu, W, S, budgets)
+    for b, L in enumerate(seqlens):
+        s0 = int(cu[b])
+        k_top = budgets[b] - S - W
+        for h in range(2):
+            sets = online_eviction(score[h, s0:s0 + L], L, W, S, k_top)
+            for t in range(L):
+                ts, tp = float(thr_s[h, s0 + t]), int(thr_p[h, s0 + t])
+                cand = range(S, t - W + 1) if t - W >= S else range(0)
+                if tp == -1 and ts == -np.inf:
+                    assert sets[t] == set(cand)                  # nothing evicted yet
+                    continue
+                kept = {p for p in cand if _rank_at_or_above(float(score[h, s0 + p]), p, ts, tp)}
+                assert kept == sets[t], (b, h, t)
+                if k_top > 0:
+                    assert len(kept) == k_top and tp in kept
+            # monotone: once defined, the threshold never gets worse
+            prev = None
+            for t in range(L):
+                ts, tp = float(thr_s[h, s0 + t]), int(thr_p[h, s0 + t])
+                if tp < 0:
+                    continue
+                if prev is not None:
+                    assert _rank_at_or_above(ts, tp, *prev)
+                prev = (ts, tp)
+            # the last step agrees with the keep mask's scored slots
+            if L > budgets[b] and L - 1 - W >= S:
+                ts, tp = float(thr_s[h, s0 + L - 1]), int(thr_p[h, s0 + L - 1])
+                mid = [p for p in range(S, L - W) if keep_final[h, s0 + p]]
+                assert set(mid) == sets[L - 1]
+
+
+ALL_PINS.append(pin_prefix_thresholds)

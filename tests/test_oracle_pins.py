@@ -43,6 +43,11 @@ MUTANTS = [
     ("keep_no_sinks", "keep[h, s:s + S] = 1", "pass"),
     ("keep_off_by_one_k", "order[:k_top]", "order[:k_top - 1]"),
     ("keep_all_when_short_dropped", "if L <= B:", "if L < 0:"),
+    ("threshold_window_off_by_one", "hi = t - W                                     # last candidate position",
+     "hi = t - W - 1"),
+    ("threshold_kth_off_by_one", "kth = order[k_top - 1]", "kth = order[k_top]"),
+    ("threshold_tie_reversed", "order = np.lexsort((pos, -sc))\n                kth", "order = np.lexsort((-pos, -sc))\n                kth"),
+    ("threshold_sinks_included", "pos = np.arange(S, hi + 1)", "pos = np.arange(0, hi + 1)"),
 ]
 
 
