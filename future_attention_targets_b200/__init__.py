@@ -12,9 +12,10 @@ from ._binding import (  # noqa: F401
     future_targets,
     keep_mask,
     lib,
+    prefix_topk_thresholds,
     row_lse,
     selftest_bounded_wait,
 )
 
 __all__ = ["HostPipeline", "KvpopError", "check_status", "future_target", "future_targets", "keep_mask", "lib",
-           "row_lse", "selftest_bounded_wait"]
+           "prefix_topk_thresholds", "row_lse", "selftest_bounded_wait"]

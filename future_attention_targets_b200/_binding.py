@@ -40,6 +40,8 @@ _SIGS = {
     "kvpop_row_lse": (ctypes.c_int, [_P, _P, _I32P, Shape, ctypes.c_float, _P, _P, _P]),
     "kvpop_future_target": (ctypes.c_int, [_P, _P, _I32P, Shape, ctypes.c_float, ctypes.c_int32, _P, _P, _P, _P]),
     "kvpop_keep_mask": (ctypes.c_int, [_P, _I32P, Shape, ctypes.c_int32, ctypes.c_int32, _I32P, _P, _P]),
+    "kvpop_prefix_topk_thresholds": (ctypes.c_int, [_P, _I32P, Shape, ctypes.c_int32, ctypes.c_int32, _I32P, _P,
+                                                    _P, _P]),
     "kvpop_future_targets": (ctypes.c_int, [_P, _P, _I32P, Shape, ctypes.c_float, ctypes.c_int32, ctypes.c_int32,
                                             _I32P, _P, _P, _P, _P, _P]),
     "kvpop_host_workspace_bytes": (ctypes.c_size_t, [Shape]),
@@ -179,6 +181,26 @@ def keep_mask(score, cu_seqlens, window: int, sinks: int, budgets, out=None, str
     _check(lib().kvpop_keep_mask(score.data_ptr(), cu_c, sh, int(window), int(sinks), bud, out.data_ptr(),
                                  _stream_ptr(stream)))
     return out
+
+
+def prefix_topk_thresholds(score, cu_seqlens, window: int, sinks: int, budgets, out=None, stream=None):
+    """Per-step eviction thresholds: (thr_score fp32 [H_kv, T], thr_pos int32 [H_kv, T])."""
+    import torch
+    if score.dtype != torch.float32 or not score.is_cuda or score.dim() != 2 or not score.is_contiguous():
+        raise TypeError("score must be a contiguous 2-D fp32 CUDA tensor [H_kv, T]")
+    cu, cu_c = _cu_host(cu_seqlens)
+    Hkv, T = score.shape
+    sh = Shape(len(cu) - 1, T, Hkv, Hkv, 128)
+    bud = _i32_host(budgets)
+    if len(bud) != sh.batch:
+        raise ValueError("one budget per sequence is needed")
+    if out is None:
+        out = (torch.empty((Hkv, T), dtype=torch.float32, device=score.device),
+               torch.empty((Hkv, T), dtype=torch.int32, device=score.device))
+    thr_s, thr_p = out
+    _check(lib().kvpop_prefix_topk_thresholds(score.data_ptr(), cu_c, sh, int(window), int(sinks), bud,
+                                              thr_s.data_ptr(), thr_p.data_ptr(), _stream_ptr(stream)))
+    return thr_s, thr_p
 
 
 def future_targets(q, k, cu_seqlens, window: int, sinks: int, budgets, scale: float | None = None,

@@ -20,6 +20,7 @@ cudaError_t launch_row_lse(const AttnParams& p, int head_dim, int grid, cudaStre
 cudaError_t launch_future_target(const AttnParams& p, int head_dim, int grid, cudaStream_t stream);
 cudaError_t launch_keep_mask(const KeepParams& p, int n_kv_heads, cudaStream_t stream);
 cudaError_t launch_selftest_wait(int32_t* status, uint64_t limit_ns, cudaStream_t stream);
+cudaError_t launch_prefix_thresholds(const ThresholdParams& p, int n_kv_heads, cudaStream_t stream);
 }  // namespace kvpop
 
 using namespace kvpop;
@@ -304,6 +305,45 @@ kvpop_status kvpop_keep_mask(const float* score, const int32_t* cu_seqlens, kvpo
   }
   cudaError_t e = launch_keep_mask(p, shape.n_kv_heads, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "keep_mask launch");
+}
+
+kvpop_status kvpop_prefix_topk_thresholds(const float* score, const int32_t* cu_seqlens, kvpop_shape shape,
+                                          int32_t window, int32_t sinks, const int32_t* budgets, float* thr_score,
+                                          int32_t* thr_pos, void* stream) {
+  kvpop_status st;
+  if (score == nullptr || thr_score == nullptr || thr_pos == nullptr)
+    return fail(KVPOP_ERR_INVALID_ARG, "score, thr_score or thr_pos is NULL");
+  if (budgets == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "budgets is NULL");
+  if (window < 0 || sinks < 0) return fail(KVPOP_ERR_INVALID_ARG, "window and sinks must be >= 0");
+  if ((st = check_shape(cu_seqlens, shape, false)) != KVPOP_OK) return st;
+  for (int b = 0; b < shape.batch; ++b) {
+    const int64_t k = static_cast<int64_t>(budgets[b]) - sinks - window;
+    if (k < 0)
+      return fail(KVPOP_ERR_INVALID_ARG, "budget[%d] = %d is below sinks + window = %lld", b, budgets[b],
+                  static_cast<long long>(sinks) + window);
+    if (k > kMaxScored)
+      return fail(KVPOP_ERR_UNSUPPORTED, "budget[%d] leaves %lld scored slots (limit %d)", b,
+                  static_cast<long long>(k), kMaxScored);
+  }
+  if (shape.total_tokens == 0) return KVPOP_OK;
+  DeviceInfo dev;
+  if ((st = device_info(&dev)) != KVPOP_OK) return st;
+  ThresholdParams p;
+  memset(&p, 0, sizeof(p));
+  p.score = score;
+  p.thr_score = thr_score;
+  p.thr_pos = thr_pos;
+  p.total_tokens = shape.total_tokens;
+  p.window = window;
+  p.sinks = sinks;
+  p.n_seqs = shape.batch;
+  for (int b = 0; b < shape.batch; ++b) {
+    p.seq_start[b] = cu_seqlens[b];
+    p.seq_len[b] = cu_seqlens[b + 1] - cu_seqlens[b];
+    p.budget[b] = budgets[b];
+  }
+  cudaError_t e = launch_prefix_thresholds(p, shape.n_kv_heads, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "prefix thresholds launch");
 }
 
 kvpop_status kvpop_future_targets(const void* q, const void* k, const int32_t* cu_seqlens, kvpop_shape shape,

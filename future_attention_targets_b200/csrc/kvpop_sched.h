@@ -58,4 +58,19 @@ struct KeepParams {
   int32_t budget[kMaxSeqs];
 };
 
+constexpr int kMaxScored = 8192;   // largest scored-slot count k for the prefix thresholds
+
+struct ThresholdParams {
+  const float* score;     // [H_kv, T]
+  float* thr_score;       // [H_kv, T]
+  int32_t* thr_pos;       // [H_kv, T]
+  int32_t total_tokens;
+  int32_t window;
+  int32_t sinks;
+  int32_t n_seqs;
+  int32_t seq_start[kMaxSeqs];
+  int32_t seq_len[kMaxSeqs];
+  int32_t budget[kMaxSeqs];
+};
+
 }  // namespace kvpop

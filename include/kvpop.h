@@ -121,6 +121,30 @@ KVPOP_API kvpop_status kvpop_keep_mask(const float* score, const int32_t* cu_seq
                              int32_t window, int32_t sinks, const int32_t* budgets,
                              uint8_t* keep, void* stream);
 
+/* Prefix top-k eviction thresholds (model card, "Usage" note: the scorer's
+ * "prefix top-k thresholds").  At decoding step t (relative to the sequence
+ * start) the tokens p in [sinks, t - window] have left the recent window and
+ * compete for the k = budget[b] - sinks - window scored slots.  Per sequence
+ * b, KV head h and step t the threshold is the k-th best of them in the keep
+ * order (higher score first, then smaller position; NaN below every number,
+ * -0 equal to +0); a token is kept at step t iff it ranks at or above it.
+ * With fixed scores this equals online eviction of the worst token whenever
+ * the scored slots overflow, and at the last step it selects the same tokens
+ * as kvpop_keep_mask.
+ *   score      device fp32 [n_kv_heads, T]
+ *   budgets    HOST int32 [batch], each >= sinks + window, and
+ *              budget - sinks - window <= 8192 (else KVPOP_ERR_UNSUPPORTED)
+ *   thr_score  device fp32 [n_kv_heads, T]: the threshold token's score
+ *              (-0 reported as +0); -inf while fewer than k tokens compete
+ *              (nothing evicted yet); +inf when k = 0 (nothing kept)
+ *   thr_pos    device int32 [n_kv_heads, T]: its position relative to the
+ *              sequence start, or -1 in the two cases above
+ * No on-chip waits, no status word. */
+KVPOP_API kvpop_status kvpop_prefix_topk_thresholds(const float* score, const int32_t* cu_seqlens,
+                                                    kvpop_shape shape, int32_t window, int32_t sinks,
+                                                    const int32_t* budgets, float* thr_score,
+                                                    int32_t* thr_pos, void* stream);
+
 /* The whole hot path on device buffers: row logsumexp, transposed pass, keep
  * mask, enqueued back to back on `stream`.  lse is written as a by-product. */
 KVPOP_API kvpop_status kvpop_future_targets(const void* q, const void* k, const int32_t* cu_seqlens,

@@ -194,8 +194,11 @@ def keep_mask(score, cu_seqlens, window: int, sinks: int, budgets) -> np.ndarray
     return keep
 
 
-def prefix_topk_thresholds(score, cu_seqlens, window: int, sinks: int, budgets):
+def prefix_topk_thresholds(score, cu_seqlens, window: int, sinks: int, budgets, steps=None):
     """Per-step eviction thresholds, (thr_score float32 [H_kv, T], thr_pos int32 [H_kv, T]).
+
+    ``steps`` (optional, step indices relative to each sequence's start)
+    restricts the work to those steps; other entries are NaN / -2.
 
     For step t of a sequence (t relative to its start) the candidates are the
     positions p in [S, t - W].  With k = budget - S - W:
@@ -214,8 +217,13 @@ def prefix_topk_thresholds(score, cu_seqlens, window: int, sinks: int, budgets):
         k_top = int(budgets[b]) - S - W
         if k_top < 0:
             raise ValueError("budget below sinks + window")
+        ts_all = range(L) if steps is None else [int(t) for t in steps if 0 <= int(t) < L]
+        if steps is not None:
+            thr_s[:, s0:s0 + L] = np.nan
+            thr_p[:, s0:s0 + L] = -2
         for h in range(Hkv):
-            for t in range(L):
+            for t in ts_all:
+                thr_s[h, s0 + t], thr_p[h, s0 + t] = -np.inf, -1
                 hi = t - W                                     # last candidate position
                 if hi < S:
                     continue

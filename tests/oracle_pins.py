@@ -354,3 +354,24 @@ def pin_prefix_thresholds(orc):
 
 
 ALL_PINS.append(pin_prefix_thresholds)
+
+
+def pin_threshold_steps(orc):
+    """The steps= restriction agrees with the full computation."""
+    rng = np.random.default_rng(8)
+    cu = np.array([0, 60, 200], dtype=np.int32)
+    score = rng.random((2, 200)).astype(np.float32)
+    full_s, full_p = orc.prefix_topk_thresholds(score, cu, 5, 2, [17, 40])
+    steps = [0, 6, 7, 30, 59, 100, 139]
+    part_s, part_p = orc.prefix_topk_thresholds(score, cu, 5, 2, [17, 40], steps=steps)
+    for b in range(2):
+        s0, L = int(cu[b]), int(cu[b + 1] - cu[b])
+        for t in range(L):
+            if t in steps:
+                assert part_p[0, s0 + t] == full_p[0, s0 + t] and part_p[1, s0 + t] == full_p[1, s0 + t]
+                np.testing.assert_array_equal(part_s[:, s0 + t], full_s[:, s0 + t])
+            else:
+                assert np.all(part_p[:, s0 + t] == -2)
+
+
+ALL_PINS.append(pin_threshold_steps)

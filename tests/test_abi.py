@@ -17,7 +17,7 @@ def lib():
 
 def test_exports_every_header_symbol(lib):
     names = B.header_symbols()
-    assert len(names) == 11, names
+    assert len(names) == 12, names
     for name in names:
         assert hasattr(lib, name), f"{name} declared in kvpop.h but not exported"
     assert set(names) == set(B._SIGS), "binding signatures and header disagree"
@@ -91,6 +91,19 @@ def test_keep_mask_rejects(lib):
     assert lib.kvpop_keep_mask(FAKE, cu, sh, 16, 4, _cu(19), FAKE, None) == B.INVALID_ARG   # < sinks + window
     assert lib.kvpop_keep_mask(FAKE, cu, sh, -1, 4, bud, FAKE, None) == B.INVALID_ARG
     assert lib.kvpop_keep_mask(FAKE, cu, sh, 16, -4, bud, FAKE, None) == B.INVALID_ARG
+
+
+def test_thresholds_reject(lib):
+    cu, sh = _cu(0, 100), _shape()
+    bud = _cu(50)
+    T = lib.kvpop_prefix_topk_thresholds
+    assert T(None, cu, sh, 16, 4, bud, FAKE, FAKE, None) == B.INVALID_ARG
+    assert T(FAKE, cu, sh, 16, 4, bud, None, FAKE, None) == B.INVALID_ARG
+    assert T(FAKE, cu, sh, 16, 4, bud, FAKE, None, None) == B.INVALID_ARG
+    assert T(FAKE, cu, sh, 16, 4, None, FAKE, FAKE, None) == B.INVALID_ARG
+    assert T(FAKE, cu, sh, 16, 4, _cu(19), FAKE, FAKE, None) == B.INVALID_ARG        # below sinks + window
+    assert T(FAKE, cu, sh, 16, 4, _cu(20 + 8193), FAKE, FAKE, None) == B.UNSUPPORTED  # too many scored slots
+    assert T(FAKE, _cu(0, 0), B.Shape(1, 0, 4, 2, 128), 16, 4, bud, FAKE, FAKE, None) == B.OK
 
 
 def test_pipeline_rejects(lib):
