@@ -341,6 +341,30 @@ def run_ours(args):
                "ms_per_step": e_ms / n_e2e, "steps": n_e2e}
         del pipe
 
+    # Rows beyond the hot path, timed on this step's own targets (outside the timed region above).
+    extras = {}
+    if not args.no_extras:
+        from future_attention_targets_b200 import prefix_topk_thresholds
+        thr = (torch.empty_like(tgt), torch.empty(tgt.shape, dtype=torch.int32, device=dev))
+        for _ in range(3):
+            prefix_topk_thresholds(tgt, cu, W, S, budgets, out=thr, stream=stream)
+        n_rep = 20
+        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        x0.record(stream)
+        for _ in range(n_rep):
+            prefix_topk_thresholds(tgt, cu, W, S, budgets, out=thr, stream=stream)
+        x1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = x0.elapsed_time(x1) / n_rep
+        steps_total = sum(int(L) for L in np.diff(cu)) * w.n_kv_heads
+        moved = tgt.numel() * 4 + thr[0].numel() * 4 + thr[1].numel() * 4   # score in, threshold score + position out
+        peaks_x, _ = load_peaks()
+        extras["prefix_topk_thresholds"] = {
+            "ms": ms, "steps_per_s": steps_total / (ms * 1e-3),
+            "bound": "latency", "hbm_gbs": moved / (ms * 1e-3) / 1e9,
+            "frac_of_hbm": moved / (ms * 1e-3) / 1e9 / float(peaks_x["hbm_gbs"]),
+            "launch": f"{len(cu) - 1} x {w.n_kv_heads} CTAs of 1024 threads, one per (sequence, KV head)"}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t, f, desc = oracle_sample(d, None)
@@ -370,6 +394,7 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 3 * args.steps,
+            "next_rows": extras,
             "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)
@@ -386,6 +411,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("note: at least 3 warm-up steps are used", file=sys.stderr)

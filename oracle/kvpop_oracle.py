@@ -37,6 +37,12 @@ materialised causal softmax (one block of query rows at a time):
   this is exactly online eviction of the worst token whenever the scored
   slots overflow, and at the last step it gives the keep mask above.
 
+* Static sparse cache (model card, "Cache backends": fixed-size buffers
+  holding the same sink + scored top-k + sliding-window budget).  Compaction
+  gathers, per sequence and KV head, the kept positions in increasing order
+  into fixed slots; a decode step attends one new query per query head over
+  the filled slots of its KV head: ``out = sum_s softmax_s(s q.k_s) v_s``.
+
 Readings taken where the pages are silent: the window condition is
 ``i >= j + W``; the GQA group is summed (not averaged) with consecutive
 grouping ``g // G``; the softmax normaliser is the full causal row (sinks
@@ -51,7 +57,8 @@ from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["as_f64", "row_lse", "future_target", "keep_mask", "prefix_topk_thresholds", "ROW_BLOCK"]
+__all__ = ["as_f64", "row_lse", "future_target", "keep_mask", "prefix_topk_thresholds", "compact_kv",
+           "decode_attention", "ROW_BLOCK"]
 
 ROW_BLOCK = 256  # query rows materialised at once
 
@@ -239,3 +246,58 @@ def prefix_topk_thresholds(score, cu_seqlens, window: int, sinks: int, budgets, 
                 thr_s[h, s0 + t] = score[h, s0 + pos[kth]]
                 thr_p[h, s0 + t] = pos[kth]
     return thr_s, thr_p
+
+
+def compact_kv(k, v, keep, cu_seqlens, capacity: int):
+    """Gather kept K/V rows into fixed slots.
+
+    Returns (k_cache [B, H_kv, C, d], v_cache [B, H_kv, C, d], pos [B, H_kv, C]
+    int32 with -1 in unused slots, count [B, H_kv] int32).  Slots hold the
+    kept positions (relative to the sequence start) in increasing order; a row
+    with more kept positions than C keeps its first C and reports the full
+    count.  K and V keep their input dtype (bf16 bits stay bits).
+    """
+    k, v, keep = np.asarray(k), np.asarray(v), np.asarray(keep)
+    seqs = _sequences(cu_seqlens)
+    B, Hkv, d = len(seqs), k.shape[1], k.shape[2]
+    kc = np.zeros((B, Hkv, capacity, d), dtype=k.dtype)
+    vc = np.zeros((B, Hkv, capacity, d), dtype=v.dtype)
+    pos = np.full((B, Hkv, capacity), -1, dtype=np.int32)
+    cnt = np.zeros((B, Hkv), dtype=np.int32)
+    for b, (s0, L) in enumerate(seqs):
+        for h in range(Hkv):
+            p = np.nonzero(keep[h, s0:s0 + L])[0]
+            cnt[b, h] = len(p)
+            p = p[:capacity]
+            pos[b, h, :len(p)] = p
+            kc[b, h, :len(p)] = k[s0 + p, h]
+            vc[b, h, :len(p)] = v[s0 + p, h]
+    return kc, vc, pos, cnt
+
+
+def decode_attention(q, k_cache, v_cache, count, scale: float):
+    """One decode step over the compacted cache, float64.
+
+    q [B, H_q, d]; k_cache, v_cache [B, H_kv, C, d]; count [B, H_kv].
+    Returns (out [B, H_q, d], lse [B, H_q]) with query head g reading KV head
+    g // G over its first count[b, g // G] slots.
+    """
+    q, kc, vc = as_f64(q), as_f64(k_cache), as_f64(v_cache)
+    B, Hq, d = q.shape
+    Hkv = kc.shape[1]
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, d))
+    lse = np.full((B, Hq), -np.inf)
+    for b in range(B):
+        for g in range(Hq):
+            h = g // G
+            n = int(count[b, h])
+            if n == 0:
+                continue
+            logits = scale * (kc[b, h, :n] @ q[b, g])
+            m = logits.max()
+            w = np.exp(logits - m)
+            Z = w.sum()
+            out[b, g] = (w / Z) @ vc[b, h, :n]
+            lse[b, g] = m + np.log(Z)
+    return out, lse

@@ -375,3 +375,60 @@ def pin_threshold_steps(orc):
 
 
 ALL_PINS.append(pin_threshold_steps)
+
+
+# ------------------------------------------------------------ static cache: compaction + decode attention
+
+def pin_compact_kv(orc):
+    rng = np.random.default_rng(12)
+    seqlens = (30, 0, 45)
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    T, Hkv, d = int(cu[-1]), 2, 4
+    k = rng.integers(0, 2**16, size=(T, Hkv, d)).astype(np.uint16)
+    v = rng.integers(0, 2**16, size=(T, Hkv, d)).astype(np.uint16)
+    keep = (rng.random((Hkv, T)) < 0.4).astype(np.uint8)
+    kc, vc, pos, cnt = orc.compact_kv(k, v, keep, cu, capacity=15)
+    for b, L in enumerate(seqlens):
+        s0 = int(cu[b])
+        for h in range(Hkv):
+            kept = [p for p in range(L) if keep[h, s0 + p]]          # scalar walk, position order
+            assert cnt[b, h] == len(kept)
+            for slot in range(15):
+                if slot < len(kept):
+                    p = kept[slot]
+                    assert pos[b, h, slot] == p
+                    assert list(kc[b, h, slot]) == list(k[s0 + p, h]) and list(vc[b, h, slot]) == list(v[s0 + p, h])
+                else:
+                    assert pos[b, h, slot] == -1 and not kc[b, h, slot].any() and not vc[b, h, slot].any()
+
+
+def pin_decode_attention(orc):
+    rng = np.random.default_rng(13)
+    B, Hq, Hkv, C, d = 2, 4, 2, 9, 5
+    q = rng.standard_normal((B, Hq, d))
+    kc = rng.standard_normal((B, Hkv, C, d))
+    vc = rng.standard_normal((B, Hkv, C, d))
+    cnt = np.array([[9, 4], [1, 0]], dtype=np.int32)
+    out, lse = orc.decode_attention(q, kc, vc, cnt, 0.6)
+    for b in range(B):
+        for g in range(Hq):
+            h, n = g // 2, int(cnt[b, g // 2])
+            if n == 0:
+                assert np.all(out[b, g] == 0) and lse[b, g] == -np.inf
+                continue
+            logits = [0.6 * math.fsum(q[b, g, t] * kc[b, h, s, t] for t in range(d)) for s in range(n)]
+            m = max(logits)
+            Z = math.fsum(math.exp(x - m) for x in logits)
+            for t in range(d):
+                ref = math.fsum(math.exp(logits[s] - m) / Z * vc[b, h, s, t] for s in range(n))
+                assert abs(out[b, g, t] - ref) < 1e-12
+            assert abs(lse[b, g] - (m + math.log(Z))) < 1e-12
+    # zero keys: uniform weights, the output is the mean of the filled value rows
+    out0, _ = orc.decode_attention(q, np.zeros_like(kc), vc, cnt, 0.6)
+    np.testing.assert_allclose(out0[0, 0], vc[0, 0, :9].mean(axis=0), rtol=1e-13)
+    np.testing.assert_allclose(out0[0, 2], vc[0, 1, :4].mean(axis=0), rtol=1e-13)
+    # one filled slot: the output is that value row
+    np.testing.assert_allclose(out[1, 0], vc[1, 0, 0], rtol=1e-13)
+
+
+ALL_PINS.extend([pin_compact_kv, pin_decode_attention])

@@ -48,6 +48,10 @@ MUTANTS = [
     ("threshold_kth_off_by_one", "kth = order[k_top - 1]", "kth = order[k_top]"),
     ("threshold_tie_reversed", "order = np.lexsort((pos, -sc))\n                kth", "order = np.lexsort((-pos, -sc))\n                kth"),
     ("threshold_sinks_included", "pos = np.arange(S, hi + 1)", "pos = np.arange(0, hi + 1)"),
+    ("compact_drops_last", "p = p[:capacity]", "p = p[:capacity - 1]"),
+    ("decode_wrong_group", "            h = g // G\n            n = int(count[b, h])", "            h = g % Hkv\n            n = int(count[b, h])"),
+    ("decode_unnormalised", "out[b, g] = (w / Z) @ vc[b, h, :n]", "out[b, g] = w @ vc[b, h, :n]"),
+    ("decode_scale_dropped", "logits = scale * (kc[b, h, :n] @ q[b, g])", "logits = (kc[b, h, :n] @ q[b, g])"),
 ]
 
 
