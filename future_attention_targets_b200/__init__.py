@@ -8,6 +8,9 @@ from ._binding import (  # noqa: F401
     HostPipeline,
     KvpopError,
     check_status,
+    compact_kv,
+    decode_attention,
+    decode_workspace_bytes,
     future_target,
     future_targets,
     keep_mask,
@@ -17,5 +20,6 @@ from ._binding import (  # noqa: F401
     selftest_bounded_wait,
 )
 
-__all__ = ["HostPipeline", "KvpopError", "check_status", "future_target", "future_targets", "keep_mask", "lib",
+__all__ = ["HostPipeline", "KvpopError", "check_status", "compact_kv", "decode_attention",
+           "decode_workspace_bytes", "future_target", "future_targets", "keep_mask", "lib",
            "prefix_topk_thresholds", "row_lse", "selftest_bounded_wait"]

@@ -34,6 +34,11 @@ class Shape(ctypes.Structure):
                 ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
 
 
+class CacheShape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("capacity", ctypes.c_int32)]
+
+
 _P = ctypes.c_void_p
 _I32P = ctypes.POINTER(ctypes.c_int32)
 _SIGS = {
@@ -42,6 +47,10 @@ _SIGS = {
     "kvpop_keep_mask": (ctypes.c_int, [_P, _I32P, Shape, ctypes.c_int32, ctypes.c_int32, _I32P, _P, _P]),
     "kvpop_prefix_topk_thresholds": (ctypes.c_int, [_P, _I32P, Shape, ctypes.c_int32, ctypes.c_int32, _I32P, _P,
                                                     _P, _P]),
+    "kvpop_compact_kv": (ctypes.c_int, [_P, _P, _P, _I32P, Shape, ctypes.c_int32, _P, _P, _P, _P, _P]),
+    "kvpop_decode_workspace_bytes": (ctypes.c_size_t, [CacheShape]),
+    "kvpop_decode_attention": (ctypes.c_int, [_P, _P, _P, _P, CacheShape, ctypes.c_float, _P, _P, _P, ctypes.c_size_t,
+                                              _P]),
     "kvpop_future_targets": (ctypes.c_int, [_P, _P, _I32P, Shape, ctypes.c_float, ctypes.c_int32, ctypes.c_int32,
                                             _I32P, _P, _P, _P, _P, _P]),
     "kvpop_host_workspace_bytes": (ctypes.c_size_t, [Shape]),
@@ -201,6 +210,56 @@ def prefix_topk_thresholds(score, cu_seqlens, window: int, sinks: int, budgets, 
     _check(lib().kvpop_prefix_topk_thresholds(score.data_ptr(), cu_c, sh, int(window), int(sinks), bud,
                                               thr_s.data_ptr(), thr_p.data_ptr(), _stream_ptr(stream)))
     return thr_s, thr_p
+
+
+def compact_kv(k, v, keep, cu_seqlens, capacity: int, out=None, stream=None):
+    """Static cache: (k_cache, v_cache [B, H_kv, C, d] bf16, pos [B, H_kv, C] int32, count [B, H_kv] int32)."""
+    import torch
+    for name, t in (("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or t.dim() != 3 or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous 3-D bf16 CUDA tensor [T, H_kv, d]")
+    if keep.dtype != torch.uint8 or not keep.is_cuda or not keep.is_contiguous():
+        raise TypeError("keep must be a contiguous uint8 CUDA tensor [H_kv, T]")
+    cu, cu_c = _cu_host(cu_seqlens)
+    T, Hkv, d = k.shape
+    B = len(cu) - 1
+    sh = Shape(B, T, Hkv, Hkv, d)
+    if out is None:
+        out = (torch.empty((B, Hkv, capacity, d), dtype=torch.bfloat16, device=k.device),
+               torch.empty((B, Hkv, capacity, d), dtype=torch.bfloat16, device=k.device),
+               torch.empty((B, Hkv, capacity), dtype=torch.int32, device=k.device),
+               torch.empty((B, Hkv), dtype=torch.int32, device=k.device))
+    kc, vc, pos, cnt = out
+    _check(lib().kvpop_compact_kv(k.data_ptr(), v.data_ptr(), keep.data_ptr(), cu_c, sh, int(capacity),
+                                  kc.data_ptr(), vc.data_ptr(), pos.data_ptr(), cnt.data_ptr(), _stream_ptr(stream)))
+    return kc, vc, pos, cnt
+
+
+def decode_workspace_bytes(batch, n_q_heads, n_kv_heads, head_dim, capacity) -> int:
+    return int(lib().kvpop_decode_workspace_bytes(CacheShape(batch, n_q_heads, n_kv_heads, head_dim, capacity)))
+
+
+def decode_attention(q, k_cache, v_cache, count, scale: float | None = None, out=None, lse=None, workspace=None,
+                     stream=None):
+    """One decode step over the compacted cache: (out [B, H_q, d] fp32, lse [B, H_q] fp32)."""
+    import torch
+    if q.dtype != torch.bfloat16 or not q.is_cuda or q.dim() != 3 or not q.is_contiguous():
+        raise TypeError("q must be a contiguous 3-D bf16 CUDA tensor [B, H_q, d]")
+    B, Hq, d = q.shape
+    _, Hkv, C, _ = k_cache.shape
+    sh = CacheShape(B, Hq, Hkv, d, C)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    need = int(lib().kvpop_decode_workspace_bytes(sh))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(lib().kvpop_decode_attention(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), count.data_ptr(), sh,
+                                        scale, out.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
+                                        workspace.numel(), _stream_ptr(stream)))
+    return out, lse
 
 
 def future_targets(q, k, cu_seqlens, window: int, sinks: int, budgets, scale: float | None = None,

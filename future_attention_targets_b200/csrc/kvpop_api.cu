@@ -21,6 +21,8 @@ cudaError_t launch_future_target(const AttnParams& p, int head_dim, int grid, cu
 cudaError_t launch_keep_mask(const KeepParams& p, int n_kv_heads, cudaStream_t stream);
 cudaError_t launch_selftest_wait(int32_t* status, uint64_t limit_ns, cudaStream_t stream);
 cudaError_t launch_prefix_thresholds(const ThresholdParams& p, int n_kv_heads, cudaStream_t stream);
+cudaError_t launch_compact_kv(const CompactParams& p, cudaStream_t stream);
+cudaError_t launch_decode_attention(const DecodeParams& p, int batch, cudaStream_t stream);
 }  // namespace kvpop
 
 using namespace kvpop;
@@ -344,6 +346,98 @@ kvpop_status kvpop_prefix_topk_thresholds(const float* score, const int32_t* cu_
   }
   cudaError_t e = launch_prefix_thresholds(p, shape.n_kv_heads, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "prefix thresholds launch");
+}
+
+kvpop_status kvpop_compact_kv(const void* k, const void* v, const uint8_t* keep, const int32_t* cu_seqlens,
+                              kvpop_shape shape, int32_t capacity, void* k_cache, void* v_cache, int32_t* pos,
+                              int32_t* count, void* stream) {
+  kvpop_status st;
+  if (k == nullptr || v == nullptr || keep == nullptr || k_cache == nullptr || v_cache == nullptr ||
+      pos == nullptr || count == nullptr)
+    return fail(KVPOP_ERR_INVALID_ARG, "a pointer argument is NULL");
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache))
+    return fail(KVPOP_ERR_INVALID_ARG, "k, v, k_cache and v_cache must be 16-byte aligned");
+  if (capacity < 1) return fail(KVPOP_ERR_INVALID_ARG, "capacity must be >= 1");
+  if (shape.head_dim != 64 && shape.head_dim != 128)
+    return fail(KVPOP_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", shape.head_dim);
+  if ((st = check_shape(cu_seqlens, shape, false)) != KVPOP_OK) return st;
+  DeviceInfo dev;
+  if ((st = device_info(&dev)) != KVPOP_OK) return st;
+  CompactParams p;
+  memset(&p, 0, sizeof(p));
+  p.k = static_cast<const uint16_t*>(k);
+  p.v = static_cast<const uint16_t*>(v);
+  p.keep = keep;
+  p.k_cache = static_cast<uint16_t*>(k_cache);
+  p.v_cache = static_cast<uint16_t*>(v_cache);
+  p.pos = pos;
+  p.count = count;
+  p.total_tokens = shape.total_tokens;
+  p.n_kv_heads = shape.n_kv_heads;
+  p.head_dim = shape.head_dim;
+  p.capacity = capacity;
+  p.n_seqs = shape.batch;
+  int max_len = 0;
+  for (int b = 0; b < shape.batch; ++b) {
+    p.seq_start[b] = cu_seqlens[b];
+    p.seq_len[b] = cu_seqlens[b + 1] - cu_seqlens[b];
+    max_len = std::max(max_len, p.seq_len[b]);
+  }
+  p.n_ranges = std::max(1, (max_len + kCompactRange - 1) / kCompactRange);
+  cudaError_t e = launch_compact_kv(p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "compact_kv launch");
+}
+
+static bool check_cache_shape(const kvpop_cache_shape& sh) {
+  if (sh.batch < 1 || sh.batch > kMaxSeqs || sh.n_kv_heads < 1 || sh.n_q_heads < 1 || sh.capacity < 1) return false;
+  if (sh.n_q_heads % sh.n_kv_heads != 0) return false;
+  const int G = sh.n_q_heads / sh.n_kv_heads;
+  if (G > 16 || (G & (G - 1)) != 0) return false;
+  return sh.head_dim == 64 || sh.head_dim == 128;
+}
+
+size_t kvpop_decode_workspace_bytes(kvpop_cache_shape shape) {
+  if (!check_cache_shape(shape)) return 0;
+  const size_t n_split = (static_cast<size_t>(shape.capacity) + kDecSplit - 1) / kDecSplit;
+  return static_cast<size_t>(shape.batch) * shape.n_q_heads * n_split * (shape.head_dim + 2) * sizeof(float);
+}
+
+kvpop_status kvpop_decode_attention(const void* q, const void* k_cache, const void* v_cache, const int32_t* count,
+                                    kvpop_cache_shape shape, float scale, float* out, float* lse, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  kvpop_status st;
+  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || count == nullptr || out == nullptr)
+    return fail(KVPOP_ERR_INVALID_ARG, "a pointer argument is NULL");
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(workspace))
+    return fail(KVPOP_ERR_INVALID_ARG, "k_cache, v_cache and workspace must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(q) & 7u) != 0) return fail(KVPOP_ERR_INVALID_ARG, "q must be 8-byte aligned");
+  if (!isfinite(scale) || !(scale > 0.f)) return fail(KVPOP_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (!check_cache_shape(shape))
+    return fail(KVPOP_ERR_UNSUPPORTED,
+                "cache shape not supported (head_dim 64/128, group size a power of two <= 16, 1..512 sequences)");
+  const size_t need = kvpop_decode_workspace_bytes(shape);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(KVPOP_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu required", workspace_bytes,
+                need);
+  DeviceInfo dev;
+  if ((st = device_info(&dev)) != KVPOP_OK) return st;
+  DecodeParams p;
+  memset(&p, 0, sizeof(p));
+  p.q = static_cast<const uint16_t*>(q);
+  p.k_cache = static_cast<const uint16_t*>(k_cache);
+  p.v_cache = static_cast<const uint16_t*>(v_cache);
+  p.count = count;
+  p.partial = static_cast<float*>(workspace);
+  p.out = out;
+  p.lse = lse;
+  p.n_q_heads = shape.n_q_heads;
+  p.n_kv_heads = shape.n_kv_heads;
+  p.head_dim = shape.head_dim;
+  p.capacity = shape.capacity;
+  p.n_split = (shape.capacity + kDecSplit - 1) / kDecSplit;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  cudaError_t e = launch_decode_attention(p, shape.batch, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "decode attention launch");
 }
 
 kvpop_status kvpop_future_targets(const void* q, const void* k, const int32_t* cu_seqlens, kvpop_shape shape,

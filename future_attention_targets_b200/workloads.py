@@ -24,6 +24,7 @@ __all__ = [
     "WORKLOADS",
     "get_workload",
     "make_inputs",
+    "make_decode_inputs",
     "f32_to_bf16_bits",
     "bf16_bits_to_f32",
     "causal_pairs",
@@ -214,6 +215,24 @@ def make_inputs(w: Workload | str, seed: int | None = None) -> dict:
         "sinks": w.sinks,
         "scale": 1.0 / math.sqrt(w.head_dim),
     }
+
+
+def make_decode_inputs(w: Workload | str, seed: int | None = None) -> dict:
+    """Values for the static cache and one decode query per sequence.
+
+    V rows are i.i.d. N(0,1) (bf16 bits, [T, H_kv, d]); the decode query is a
+    unit-RMS N(0,1) row per query head ([B, H_q, d]).  Drawn from a stream of
+    their own (seed + 1000), so the Q/K inputs stay unchanged.
+    """
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    s = w.seed if seed is None else seed
+    seqlens = seqlens_of(w, np.random.default_rng(s))
+    rng = np.random.default_rng(s + 1000)
+    T = int(seqlens.sum())
+    v = rng.standard_normal((T, w.n_kv_heads, w.head_dim), dtype=np.float32)
+    q_dec = _unit_rms(rng.standard_normal((len(seqlens), w.n_q_heads, w.head_dim), dtype=np.float32))
+    return {"v_bits": f32_to_bf16_bits(v), "q_dec_bits": f32_to_bf16_bits(q_dec)}
 
 
 def random_qk(T: int, n_q_heads: int, n_kv_heads: int, head_dim: int, seed: int,

@@ -145,6 +145,52 @@ KVPOP_API kvpop_status kvpop_prefix_topk_thresholds(const float* score, const in
                                                     const int32_t* budgets, float* thr_score,
                                                     int32_t* thr_pos, void* stream);
 
+/* Static fixed-budget cache (model card, "Cache backends": fixed-size buffers
+ * with the same sink + scored top-k + sliding-window budget). */
+typedef struct {
+  int32_t batch;          /* sequences, 1 .. 512 */
+  int32_t n_q_heads;      /* a multiple of n_kv_heads, at most 16 per KV head, group a power of two */
+  int32_t n_kv_heads;
+  int32_t head_dim;       /* 64 or 128 */
+  int32_t capacity;       /* cache slots per (sequence, KV head), >= 1 */
+} kvpop_cache_shape;
+
+/* Compaction: per sequence b and KV head h, the positions with keep = 1 (in
+ * increasing order) fill slots 0, 1, ... of the fixed cache.
+ *   k, v       device bf16 [T, n_kv_heads, head_dim], 16-byte aligned
+ *   keep       device uint8 [n_kv_heads, T] (normally from kvpop_keep_mask)
+ *   capacity   slots per (b, h); a row with more kept positions keeps its first
+ *              `capacity` and still reports its full count
+ *   k_cache, v_cache  device bf16 [batch, n_kv_heads, capacity, head_dim], 16-byte aligned;
+ *              unused slots are zero-filled
+ *   pos        device int32 [batch, n_kv_heads, capacity]: the source position
+ *              (relative to the sequence start) of each slot, -1 when unused
+ *   count      device int32 [batch, n_kv_heads]: kept positions per row
+ * shape.n_q_heads is ignored; no status word (no on-chip waits). */
+KVPOP_API kvpop_status kvpop_compact_kv(const void* k, const void* v, const uint8_t* keep,
+                                        const int32_t* cu_seqlens, kvpop_shape shape, int32_t capacity,
+                                        void* k_cache, void* v_cache, int32_t* pos, int32_t* count,
+                                        void* stream);
+
+/* Device workspace (bytes) kvpop_decode_attention needs for `shape`. */
+KVPOP_API size_t kvpop_decode_workspace_bytes(kvpop_cache_shape shape);
+
+/* One decode step over the compacted cache: for sequence b and query head g
+ * (KV head h = g / G),
+ *   out[b, g, :] = sum_{s < n} softmax_s(scale * q[b, g, :] . k_cache[b, h, s, :]) v_cache[b, h, s, :]
+ * with n = min(count[b, h], capacity); n = 0 gives out = 0 and lse = -inf.
+ *   q          device bf16 [batch, n_q_heads, head_dim]
+ *   k_cache, v_cache, count  as written by kvpop_compact_kv
+ *   out        device fp32 [batch, n_q_heads, head_dim]
+ *   lse        device fp32 [batch, n_q_heads] natural log, or NULL
+ *   workspace  device, >= kvpop_decode_workspace_bytes(shape) bytes, 16-byte aligned;
+ *              holds the per-split partial results (its contents on entry are ignored)
+ * Split-K over the cache slots, then one merge kernel; no on-chip waits. */
+KVPOP_API kvpop_status kvpop_decode_attention(const void* q, const void* k_cache, const void* v_cache,
+                                              const int32_t* count, kvpop_cache_shape shape, float scale,
+                                              float* out, float* lse, void* workspace, size_t workspace_bytes,
+                                              void* stream);
+
 /* The whole hot path on device buffers: row logsumexp, transposed pass, keep
  * mask, enqueued back to back on `stream`.  lse is written as a by-product. */
 KVPOP_API kvpop_status kvpop_future_targets(const void* q, const void* k, const int32_t* cu_seqlens,

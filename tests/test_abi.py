@@ -17,7 +17,7 @@ def lib():
 
 def test_exports_every_header_symbol(lib):
     names = B.header_symbols()
-    assert len(names) == 12, names
+    assert len(names) == 15, names
     for name in names:
         assert hasattr(lib, name), f"{name} declared in kvpop.h but not exported"
     assert set(names) == set(B._SIGS), "binding signatures and header disagree"
@@ -104,6 +104,25 @@ def test_thresholds_reject(lib):
     assert T(FAKE, cu, sh, 16, 4, _cu(19), FAKE, FAKE, None) == B.INVALID_ARG        # below sinks + window
     assert T(FAKE, cu, sh, 16, 4, _cu(20 + 8193), FAKE, FAKE, None) == B.UNSUPPORTED  # too many scored slots
     assert T(FAKE, _cu(0, 0), B.Shape(1, 0, 4, 2, 128), 16, 4, bud, FAKE, FAKE, None) == B.OK
+
+
+def test_static_cache_rejects(lib):
+    cu, sh = _cu(0, 100), _shape()
+    C = lib.kvpop_compact_kv
+    assert C(None, FAKE, FAKE, cu, sh, 8, FAKE, FAKE, FAKE, FAKE, None) == B.INVALID_ARG
+    assert C(FAKE, FAKE, FAKE, cu, sh, 0, FAKE, FAKE, FAKE, FAKE, None) == B.INVALID_ARG          # capacity
+    assert C(FAKE, FAKE + 8, FAKE, cu, sh, 8, FAKE, FAKE, FAKE, FAKE, None) == B.INVALID_ARG      # alignment
+    assert C(FAKE, FAKE, FAKE, cu, _shape(d=96), 8, FAKE, FAKE, FAKE, FAKE, None) == B.UNSUPPORTED
+    cs = B.CacheShape(1, 8, 2, 128, 1000)
+    need = lib.kvpop_decode_workspace_bytes(cs)
+    assert need == 1 * 8 * 4 * 130 * 4                                                             # 4 splits of 256 slots
+    assert lib.kvpop_decode_workspace_bytes(B.CacheShape(1, 6, 2, 128, 10)) == 0                    # group of 3
+    D = lib.kvpop_decode_attention
+    assert D(FAKE, FAKE, FAKE, FAKE, cs, 0.1, FAKE, None, FAKE, need - 1, None) == B.INVALID_ARG   # workspace
+    assert D(FAKE, FAKE, FAKE, FAKE, cs, 0.0, FAKE, None, FAKE, need, None) == B.INVALID_ARG       # scale
+    assert D(FAKE, FAKE, FAKE, None, cs, 0.1, FAKE, None, FAKE, need, None) == B.INVALID_ARG       # count
+    assert D(FAKE, FAKE, FAKE, FAKE, B.CacheShape(1, 64, 2, 128, 10), 0.1, FAKE, None, FAKE, need,
+             None) == B.UNSUPPORTED                                                                # group of 32
 
 
 def test_pipeline_rejects(lib):
