@@ -51,6 +51,7 @@ _SIGS = {
     "kvpop_decode_workspace_bytes": (ctypes.c_size_t, [CacheShape]),
     "kvpop_decode_attention": (ctypes.c_int, [_P, _P, _P, _P, CacheShape, ctypes.c_float, _P, _P, _P, ctypes.c_size_t,
                                               _P]),
+    "kvpop_decode_attention_noalloc": (ctypes.c_int, [_P, _P, _P, _P, CacheShape, ctypes.c_float, _P, _P, _P]),
     "kvpop_future_targets": (ctypes.c_int, [_P, _P, _I32P, Shape, ctypes.c_float, ctypes.c_int32, ctypes.c_int32,
                                             _I32P, _P, _P, _P, _P, _P]),
     "kvpop_host_workspace_bytes": (ctypes.c_size_t, [Shape]),

@@ -23,6 +23,8 @@ cudaError_t launch_selftest_wait(int32_t* status, uint64_t limit_ns, cudaStream_
 cudaError_t launch_prefix_thresholds(const ThresholdParams& p, int n_kv_heads, cudaStream_t stream);
 cudaError_t launch_compact_kv(const CompactParams& p, cudaStream_t stream);
 cudaError_t launch_decode_attention(const DecodeParams& p, int batch, cudaStream_t stream);
+size_t decode_scratch_bytes();
+cudaError_t decode_scratch_address(float** out);
 }  // namespace kvpop
 
 using namespace kvpop;
@@ -437,6 +439,49 @@ kvpop_status kvpop_decode_attention(const void* q, const void* k_cache, const vo
   p.n_split = (shape.capacity + kDecSplit - 1) / kDecSplit;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   cudaError_t e = launch_decode_attention(p, shape.batch, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "decode attention launch");
+}
+
+kvpop_status kvpop_decode_attention_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                            const int32_t* count, kvpop_cache_shape shape, float scale, float* out,
+                                            float* lse, void* stream) {
+  kvpop_status st;
+  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || count == nullptr || out == nullptr)
+    return fail(KVPOP_ERR_INVALID_ARG, "a pointer argument is NULL");
+  if (!aligned16(k_cache) || !aligned16(v_cache))
+    return fail(KVPOP_ERR_INVALID_ARG, "k_cache and v_cache must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(q) & 7u) != 0) return fail(KVPOP_ERR_INVALID_ARG, "q must be 8-byte aligned");
+  if (!isfinite(scale) || !(scale > 0.f)) return fail(KVPOP_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (!check_cache_shape(shape))
+    return fail(KVPOP_ERR_UNSUPPORTED,
+                "cache shape not supported (head_dim 64/128, group size a power of two <= 16, 1..512 sequences)");
+  const size_t need = kvpop_decode_workspace_bytes(shape);
+  if (need > decode_scratch_bytes())
+    return fail(KVPOP_ERR_UNSUPPORTED,
+                "this shape needs %zu bytes of split partials, more than the %zu-byte fixed scratch; "
+                "use kvpop_decode_attention with a workspace",
+                need, decode_scratch_bytes());
+  DeviceInfo dev;
+  if ((st = device_info(&dev)) != KVPOP_OK) return st;
+  float* scratch = nullptr;
+  cudaError_t e = decode_scratch_address(&scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the decode scratch");
+  DecodeParams p;
+  memset(&p, 0, sizeof(p));
+  p.q = static_cast<const uint16_t*>(q);
+  p.k_cache = static_cast<const uint16_t*>(k_cache);
+  p.v_cache = static_cast<const uint16_t*>(v_cache);
+  p.count = count;
+  p.partial = scratch;
+  p.out = out;
+  p.lse = lse;
+  p.n_q_heads = shape.n_q_heads;
+  p.n_kv_heads = shape.n_kv_heads;
+  p.head_dim = shape.head_dim;
+  p.capacity = shape.capacity;
+  p.n_split = (shape.capacity + kDecSplit - 1) / kDecSplit;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  e = launch_decode_attention(p, shape.batch, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "decode attention launch");
 }
 

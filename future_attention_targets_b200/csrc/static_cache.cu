@@ -9,6 +9,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "kvpop_sched.h"
 
 namespace kvpop {
@@ -267,6 +269,38 @@ cudaError_t launch_decode_attention(const DecodeParams& p, int batch, cudaStream
   if (e != cudaSuccess) return e;
   decode_combine_kernel<<<batch * p.n_q_heads, 128, 0, stream>>>(p);
   return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ fixed scratch for the allocation-free decode
+
+// Split partials of kvpop_decode_attention_noalloc live here instead of in a
+// caller workspace.  Every device on which this library's kernels run holds
+// these bytes until the process exits.
+constexpr size_t kDecodeScratchBytes = size_t(4) << 20;
+static __device__ __align__(256) float g_decode_scratch[kDecodeScratchBytes / sizeof(float)];
+
+size_t decode_scratch_bytes() { return kDecodeScratchBytes; }
+
+// Device address of g_decode_scratch on the current device.  In host code the
+// symbol's name is only a stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+cudaError_t decode_scratch_address(float** out) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = ptr;
+  }
+  *out = static_cast<float*>(addr[dev]);
+  return cudaSuccess;
 }
 
 }  // namespace kvpop

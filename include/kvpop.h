@@ -191,6 +191,33 @@ KVPOP_API kvpop_status kvpop_decode_attention(const void* q, const void* k_cache
                                               float* out, float* lse, void* workspace, size_t workspace_bytes,
                                               void* stream);
 
+/* kvpop_decode_attention without a workspace argument, for callers that may
+ * not allocate device memory when they run a decode step: for example code
+ * whose device memory is all owned by another framework's allocator or a
+ * pre-reserved pool (a stray cudaMalloc would fail or fragment it), decode
+ * loops where cudaMalloc's device-wide synchronisation costs too much, or
+ * plugin hooks whose interface hands them no scratch buffer.  The pages have
+ * no counterpart: this is a deployment variant, not part of the method.
+ *
+ * The split partials go to one fixed scratch array of 4 MiB that is part of
+ * the library's device image, so every GPU on which the library runs holds
+ * those 4 MiB until the process exits.  Shapes whose partials exceed it
+ * (batch * n_q_heads * ceil(capacity / 256) * (head_dim + 2) * 4 bytes)
+ * return KVPOP_ERR_UNSUPPORTED; use kvpop_decode_attention for them.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it; make that first call before any
+ * stream capture.  The call never calls cudaMalloc or cudaFree.  Every call
+ * uses the same array and leaves its partials there; nothing in it needs to
+ * start at zero, because each call writes every partial it later reads.
+ * Calls that overlap on the GPU (for example on two streams at once) race on
+ * the array, so issue them one after another, e.g. on one stream per device.
+ * Each process has its own copy of the array.
+ * Other arguments and results as for kvpop_decode_attention. */
+KVPOP_API kvpop_status kvpop_decode_attention_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                                      const int32_t* count, kvpop_cache_shape shape, float scale,
+                                                      float* out, float* lse, void* stream);
+
 /* The whole hot path on device buffers: row logsumexp, transposed pass, keep
  * mask, enqueued back to back on `stream`.  lse is written as a by-product. */
 KVPOP_API kvpop_status kvpop_future_targets(const void* q, const void* k, const int32_t* cu_seqlens,

@@ -17,7 +17,7 @@ def lib():
 
 def test_exports_every_header_symbol(lib):
     names = B.header_symbols()
-    assert len(names) == 15, names
+    assert len(names) == 16, names
     for name in names:
         assert hasattr(lib, name), f"{name} declared in kvpop.h but not exported"
     assert set(names) == set(B._SIGS), "binding signatures and header disagree"
@@ -123,6 +123,12 @@ def test_static_cache_rejects(lib):
     assert D(FAKE, FAKE, FAKE, None, cs, 0.1, FAKE, None, FAKE, need, None) == B.INVALID_ARG       # count
     assert D(FAKE, FAKE, FAKE, FAKE, B.CacheShape(1, 64, 2, 128, 10), 0.1, FAKE, None, FAKE, need,
              None) == B.UNSUPPORTED                                                                # group of 32
+    N = lib.kvpop_decode_attention_noalloc
+    assert N(FAKE, FAKE, FAKE, None, cs, 0.1, FAKE, None, None) == B.INVALID_ARG
+    assert N(FAKE, FAKE, FAKE, FAKE, cs, -1.0, FAKE, None, None) == B.INVALID_ARG
+    big = B.CacheShape(64, 64, 8, 128, 8192)                                                       # 68 MB of partials
+    assert N(FAKE, FAKE, FAKE, FAKE, big, 0.1, FAKE, None, None) == B.UNSUPPORTED
+    assert b"fixed scratch" in lib.kvpop_last_error()
 
 
 def test_pipeline_rejects(lib):
