@@ -345,17 +345,24 @@ def run_ours(args):
     extras = {}
     if not args.no_extras:
         from future_attention_targets_b200 import prefix_topk_thresholds
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # twice the 126 MB L2
+
+        def timed(fn, reps=20):
+            """Median device time of fn, with L2 flushed before every repetition."""
+            for _ in range(3):
+                fn()
+            evs_x = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                     for _ in range(reps)]
+            for a, z in evs_x:
+                flush.zero_()
+                a.record(stream)
+                fn()
+                z.record(stream)
+            torch.cuda.synchronize(dev)
+            return statistics.median(a.elapsed_time(z) for a, z in evs_x)
+
         thr = (torch.empty_like(tgt), torch.empty(tgt.shape, dtype=torch.int32, device=dev))
-        for _ in range(3):
-            prefix_topk_thresholds(tgt, cu, W, S, budgets, out=thr, stream=stream)
-        n_rep = 20
-        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        x0.record(stream)
-        for _ in range(n_rep):
-            prefix_topk_thresholds(tgt, cu, W, S, budgets, out=thr, stream=stream)
-        x1.record(stream)
-        torch.cuda.synchronize(dev)
-        ms = x0.elapsed_time(x1) / n_rep
+        ms = timed(lambda: prefix_topk_thresholds(tgt, cu, W, S, budgets, out=thr, stream=stream))
         steps_total = sum(int(L) for L in np.diff(cu)) * w.n_kv_heads
         moved = tgt.numel() * 4 + thr[0].numel() * 4 + thr[1].numel() * 4   # score in, threshold score + position out
         peaks_x, _ = load_peaks()
@@ -376,22 +383,14 @@ def run_ours(args):
         dec_out = decode_attention(q_dec, cache[0], cache[1], cache[3], scale, stream=stream)
         kept_rows = int(cache[3].sum().item())
 
-        def timed(fn, reps=20):
-            for _ in range(3):
-                fn()
-            a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for _ in range(reps):
-                fn()
-            z.record(stream)
-            torch.cuda.synchronize(dev)
-            return a.elapsed_time(z) / reps
-
         row_bytes = w.head_dim * 2
         ms_c = timed(lambda: compact_kv(k, v, keep, cu, C, out=cache, stream=stream))
         moved_c = keep.numel() + 2 * 2 * kept_rows * row_bytes + 4 * cache[2].numel()   # mask, K+V in and out, slots
+        from future_attention_targets_b200 import decode_workspace_bytes
+        ws1 = torch.empty(decode_workspace_bytes(1, w.n_q_heads, w.n_kv_heads, w.head_dim, C), dtype=torch.uint8,
+                          device=dev)
         ms_d = timed(lambda: decode_attention(q_dec, cache[0], cache[1], cache[3], scale, out=dec_out[0],
-                                              lse=dec_out[1], stream=stream))
+                                              lse=dec_out[1], workspace=ws1, stream=stream))
         moved_d = 2 * kept_rows * row_bytes + q_dec.numel() * 2 + dec_out[0].numel() * 4
         hbm = float(peaks_x["hbm_gbs"])
         extras["compact_kv"] = {"ms": ms_c, "bound": "hbm", "achieved_gbs": moved_c / (ms_c * 1e-3) / 1e9,
@@ -400,6 +399,54 @@ def run_ours(args):
         extras["decode_attention"] = {"ms": ms_d, "bound": "hbm", "achieved_gbs": moved_d / (ms_d * 1e-3) / 1e9,
                                       "peak_gbs": hbm, "frac": moved_d / (ms_d * 1e-3) / 1e9 / hbm,
                                       "bytes": moved_d, "cache_slots": C}
+        # The same decode step for 16 sequences at once (each a copy of this
+        # cache at its own address): 264 MB of K and V, past the L2.
+        nb = 16
+        kc16, vc16 = cache[0].repeat(nb, 1, 1, 1), cache[1].repeat(nb, 1, 1, 1)
+        cnt16, q16 = cache[3].repeat(nb, 1), q_dec.repeat(nb, 1, 1)
+        out16 = decode_attention(q16, kc16, vc16, cnt16, scale, stream=stream)
+        ws16 = torch.empty(decode_workspace_bytes(nb, w.n_q_heads, w.n_kv_heads, w.head_dim, C), dtype=torch.uint8,
+                           device=dev)
+        ms_d16 = timed(lambda: decode_attention(q16, kc16, vc16, cnt16, scale, out=out16[0], lse=out16[1],
+                                                workspace=ws16, stream=stream))
+        moved_d16 = nb * moved_d
+        extras["decode_attention_batch16"] = {
+            "ms": ms_d16, "bound": "hbm", "achieved_gbs": moved_d16 / (ms_d16 * 1e-3) / 1e9, "peak_gbs": hbm,
+            "frac": moved_d16 / (ms_d16 * 1e-3) / 1e9 / hbm, "bytes": moved_d16, "cache_slots": C, "batch": nb}
+        extras["timing"] = "median of 20 repetitions, L2 flushed (256 MiB write) before each"
+        del kc16, vc16, flush
+
+    # One problem (rank 0's layer) with its KV heads split over the ranks:
+    # two passes on H_kv / P heads, one NCCL all-gather of the targets, the
+    # keep mask on all heads.  Every rank takes the same collective steps.
+    if world > 1 and not args.no_extras and w.n_kv_heads % world == 0:
+        from future_attention_targets_b200.sharded import HeadShardedTargets, shard_heads
+        d0 = make_inputs(WORKLOAD, seed=rank_seed(0))
+        q0 = torch.from_numpy(d0["q_bits"].view(np.int16)).view(torch.bfloat16).to(dev)
+        k0 = torch.from_numpy(d0["k_bits"].view(np.int16)).view(torch.bfloat16).to(dev)
+        q_loc, k_loc = shard_heads(q0, k0, w.n_kv_heads, world, rank)
+        del q0, k0, d0
+        sharded = HeadShardedTargets(cu, w.n_q_heads, w.n_kv_heads, w.head_dim, W, S, budgets, scale, device=dev)
+        for _ in range(max(3, args.warmup)):
+            sharded(q_loc, k_loc, stream)
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        torch.cuda.synchronize(dev)
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            sharded(q_loc, k_loc, stream)
+        z.record(stream)
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        ms_sh = max_over_ranks(a.elapsed_time(z), dev) / args.steps
+        check_status(sharded.status, stream)
+        extras["head_sharded"] = {
+            "ms": ms_sh, "scaling": "strong", "value": fl["total"] / (ms_sh * 1e-3) / 1e12, "unit": UNIT,
+            "speedup_vs_one_gpu_step": ms_per_step / ms_sh, "kv_heads_per_rank": w.n_kv_heads // world,
+            "collective": "one all_gather_into_tensor (NCCL) of target [H_kv / P, T] fp32 per step",
+            "gathered_bytes": int(sharded.target.numel() * 4)}
+        del sharded, q_loc, k_loc
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

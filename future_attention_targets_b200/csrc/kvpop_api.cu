@@ -13,7 +13,7 @@
 #include <vector>
 
 #include "kvpop.h"
-#include "kvpop_sched.h"
+#include "kvpop_cache.h"
 
 namespace kvpop {
 cudaError_t launch_row_lse(const AttnParams& p, int head_dim, int grid, cudaStream_t stream);
@@ -379,13 +379,10 @@ kvpop_status kvpop_compact_kv(const void* k, const void* v, const uint8_t* keep,
   p.head_dim = shape.head_dim;
   p.capacity = capacity;
   p.n_seqs = shape.batch;
-  int max_len = 0;
   for (int b = 0; b < shape.batch; ++b) {
     p.seq_start[b] = cu_seqlens[b];
     p.seq_len[b] = cu_seqlens[b + 1] - cu_seqlens[b];
-    max_len = std::max(max_len, p.seq_len[b]);
   }
-  p.n_ranges = std::max(1, (max_len + kCompactRange - 1) / kCompactRange);
   cudaError_t e = launch_compact_kv(p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "compact_kv launch");
 }
@@ -412,7 +409,7 @@ kvpop_status kvpop_decode_attention(const void* q, const void* k_cache, const vo
     return fail(KVPOP_ERR_INVALID_ARG, "a pointer argument is NULL");
   if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(workspace))
     return fail(KVPOP_ERR_INVALID_ARG, "k_cache, v_cache and workspace must be 16-byte aligned");
-  if ((reinterpret_cast<uintptr_t>(q) & 7u) != 0) return fail(KVPOP_ERR_INVALID_ARG, "q must be 8-byte aligned");
+  if (!aligned16(q)) return fail(KVPOP_ERR_INVALID_ARG, "q must be 16-byte aligned");
   if (!isfinite(scale) || !(scale > 0.f)) return fail(KVPOP_ERR_INVALID_ARG, "scale must be finite and > 0");
   if (!check_cache_shape(shape))
     return fail(KVPOP_ERR_UNSUPPORTED,
@@ -450,7 +447,7 @@ kvpop_status kvpop_decode_attention_noalloc(const void* q, const void* k_cache, 
     return fail(KVPOP_ERR_INVALID_ARG, "a pointer argument is NULL");
   if (!aligned16(k_cache) || !aligned16(v_cache))
     return fail(KVPOP_ERR_INVALID_ARG, "k_cache and v_cache must be 16-byte aligned");
-  if ((reinterpret_cast<uintptr_t>(q) & 7u) != 0) return fail(KVPOP_ERR_INVALID_ARG, "q must be 8-byte aligned");
+  if (!aligned16(q)) return fail(KVPOP_ERR_INVALID_ARG, "q must be 16-byte aligned");
   if (!isfinite(scale) || !(scale > 0.f)) return fail(KVPOP_ERR_INVALID_ARG, "scale must be finite and > 0");
   if (!check_cache_shape(shape))
     return fail(KVPOP_ERR_UNSUPPORTED,

@@ -19,7 +19,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "kvpop_sched.h"
+#include "kvpop_cache.h"
 
 namespace kvpop {
 

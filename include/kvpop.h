@@ -179,13 +179,15 @@ KVPOP_API size_t kvpop_decode_workspace_bytes(kvpop_cache_shape shape);
  * (KV head h = g / G),
  *   out[b, g, :] = sum_{s < n} softmax_s(scale * q[b, g, :] . k_cache[b, h, s, :]) v_cache[b, h, s, :]
  * with n = min(count[b, h], capacity); n = 0 gives out = 0 and lse = -inf.
- *   q          device bf16 [batch, n_q_heads, head_dim]
+ *   q          device bf16 [batch, n_q_heads, head_dim], 16-byte aligned
  *   k_cache, v_cache, count  as written by kvpop_compact_kv
  *   out        device fp32 [batch, n_q_heads, head_dim]
  *   lse        device fp32 [batch, n_q_heads] natural log, or NULL
  *   workspace  device, >= kvpop_decode_workspace_bytes(shape) bytes, 16-byte aligned;
  *              holds the per-split partial results (its contents on entry are ignored)
- * Split-K over the cache slots, then one merge kernel; no on-chip waits. */
+ * Split-K over the cache slots (128 per CTA, staged in shared memory), then
+ * one merge kernel launched as a programmatic dependent of the first; no
+ * on-chip spin waits. */
 KVPOP_API kvpop_status kvpop_decode_attention(const void* q, const void* k_cache, const void* v_cache,
                                               const int32_t* count, kvpop_cache_shape shape, float scale,
                                               float* out, float* lse, void* workspace, size_t workspace_bytes,
@@ -202,7 +204,7 @@ KVPOP_API kvpop_status kvpop_decode_attention(const void* q, const void* k_cache
  * The split partials go to one fixed scratch array of 4 MiB that is part of
  * the library's device image, so every GPU on which the library runs holds
  * those 4 MiB until the process exits.  Shapes whose partials exceed it
- * (batch * n_q_heads * ceil(capacity / 256) * (head_dim + 2) * 4 bytes)
+ * (batch * n_q_heads * ceil(capacity / 128) * (head_dim + 2) * 4 bytes)
  * return KVPOP_ERR_UNSUPPORTED; use kvpop_decode_attention for them.
  *
  * The first call on each device looks up the array's device address

@@ -115,12 +115,13 @@ def test_static_cache_rejects(lib):
     assert C(FAKE, FAKE, FAKE, cu, _shape(d=96), 8, FAKE, FAKE, FAKE, FAKE, None) == B.UNSUPPORTED
     cs = B.CacheShape(1, 8, 2, 128, 1000)
     need = lib.kvpop_decode_workspace_bytes(cs)
-    assert need == 1 * 8 * 4 * 130 * 4                                                             # 4 splits of 256 slots
+    assert need == 1 * 8 * 8 * 130 * 4                                                             # 8 splits of 128 slots
     assert lib.kvpop_decode_workspace_bytes(B.CacheShape(1, 6, 2, 128, 10)) == 0                    # group of 3
     D = lib.kvpop_decode_attention
     assert D(FAKE, FAKE, FAKE, FAKE, cs, 0.1, FAKE, None, FAKE, need - 1, None) == B.INVALID_ARG   # workspace
     assert D(FAKE, FAKE, FAKE, FAKE, cs, 0.0, FAKE, None, FAKE, need, None) == B.INVALID_ARG       # scale
     assert D(FAKE, FAKE, FAKE, None, cs, 0.1, FAKE, None, FAKE, need, None) == B.INVALID_ARG       # count
+    assert D(FAKE + 8, FAKE, FAKE, FAKE, cs, 0.1, FAKE, None, FAKE, need, None) == B.INVALID_ARG   # q alignment
     assert D(FAKE, FAKE, FAKE, FAKE, B.CacheShape(1, 64, 2, 128, 10), 0.1, FAKE, None, FAKE, need,
              None) == B.UNSUPPORTED                                                                # group of 32
     N = lib.kvpop_decode_attention_noalloc

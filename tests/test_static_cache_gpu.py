@@ -50,18 +50,40 @@ def test_compaction_random_masks(seqlens, Hkv, d, C, p):
     check_compaction(k_bits, v_bits, keep, cu, C)
 
 
+@pytest.mark.parametrize("seqlens,C", [((16384,), 4032), ((3001, 17, 5000), 1000), ((70000,), 129)])
+def test_compaction_clustered_masks(seqlens, C):
+    """Kept positions packed at the front (as large targets of early keys give) and
+    unaligned sequence starts: the slot-range CTAs must still find every row."""
+    T, Hkv, d = sum(seqlens), 2, 128
+    k_bits, _ = random_qk(T, Hkv, Hkv, d, seed=5)
+    v_bits, _ = random_qk(T, Hkv, Hkv, d, seed=6)
+    keep = np.zeros((Hkv, T), dtype=np.uint8)
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    rng = np.random.default_rng(9)
+    for b, L in enumerate(seqlens):
+        s0 = cu[b]
+        keep[0, s0:s0 + min(L, 3 * C // 4)] = 1                        # a dense front block
+        keep[0, s0 + max(0, L - 256):s0 + L] = 1                       # and the recent window
+        keep[1, s0:s0 + L] = rng.random(L) < (C / max(L, 1)) * np.linspace(2, 0, L)   # density falling with p
+    check_compaction(k_bits, v_bits, keep, cu, C)
+
+
 @pytest.mark.parametrize("G,d,C,fill", [(4, 128, 1000, [1000, 3, 0, 517]), (2, 64, 300, [300, 1, 299, 0]),
                                         (1, 128, 40, [40, 40, 7, 1]), (16, 128, 600, [600, 256, 257, 255]),
-                                        (8, 64, 513, [513, 512, 1, 2])])
+                                        (8, 64, 513, [513, 512, 1, 2]),
+                                        # warp (32-slot) and CTA (128-slot) boundaries, several sequences
+                                        (4, 128, 300, [[129, 32, 33, 95], [1, 300, 128, 31], [0, 0, 0, 64]]),
+                                        (2, 64, 130, [[127, 128], [129, 130]])])
 def test_decode_attention_random_cache(G, d, C, fill):
-    B, Hkv = 1, len(fill)
+    fill = fill if isinstance(fill[0], list) else [fill]
+    B, Hkv = len(fill), len(fill[0])
     rng = np.random.default_rng(C + G)
     kc = rng.standard_normal((B, Hkv, C, d)).astype(np.float32) * 2.0
     vc = rng.standard_normal((B, Hkv, C, d)).astype(np.float32)
     q = rng.standard_normal((B, Hkv * G, d)).astype(np.float32)
     from future_attention_targets_b200.workloads import f32_to_bf16_bits
     kb, vb, qb = f32_to_bf16_bits(kc), f32_to_bf16_bits(vc), f32_to_bf16_bits(q)
-    cnt = np.array([fill], dtype=np.int32)
+    cnt = np.array(fill, dtype=np.int32)
     scale = 1.0 / math.sqrt(d)
     out, lse = decode_attention(dev(qb), dev(kb), dev(vb), torch.from_numpy(cnt).cuda(), scale)
     ro, rl = oracle.decode_attention(qb, kb, vb, cnt, scale)
