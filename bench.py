@@ -344,6 +344,33 @@ def run_ours(args):
     # Rows beyond the hot path, timed on this step's own targets (outside the timed region above).
     extras = {}
     if not args.no_extras:
+        # The same step with both attention passes in one cooperative launch.
+        from future_attention_targets_b200 import fused_workspace, future_targets_fused
+        ws_f = fused_workspace(cu, w.n_q_heads, w.n_kv_heads, w.head_dim, device=dev)
+        lse_f, tgt_f, keep_f = torch.empty_like(lse), torch.empty_like(tgt), torch.empty_like(keep)
+
+        def fused_step():
+            future_targets_fused(q, k, cu, W, S, budgets, scale, lse=lse_f, target=tgt_f, keep=keep_f,
+                                 workspace=ws_f, status=status, stream=stream)
+
+        for _ in range(max(3, args.warmup)):
+            fused_step()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            fused_step()
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        check_status(status, stream)
+        ms_f = f0.elapsed_time(f1) / args.steps
+        extras["fused_single_launch"] = {
+            "ms_per_step": ms_f, "value": fl["total"] / (ms_f * 1e-3) / 1e12, "unit": UNIT,
+            "vs_two_launch_step": ms_per_step / ms_f,
+            "identical_to_two_launch": bool(torch.equal(tgt_f, tgt) and torch.equal(keep_f, keep)
+                                            and torch.equal(lse_f, lse)),
+            "launches_per_step": 2}
+        del ws_f, lse_f, tgt_f, keep_f
+
         from future_attention_targets_b200 import prefix_topk_thresholds
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # twice the 126 MB L2
 

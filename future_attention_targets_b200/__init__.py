@@ -13,6 +13,8 @@ from ._binding import (  # noqa: F401
     decode_workspace_bytes,
     future_target,
     future_targets,
+    future_targets_fused,
+    fused_workspace,
     keep_mask,
     lib,
     prefix_topk_thresholds,
@@ -21,5 +23,6 @@ from ._binding import (  # noqa: F401
 )
 
 __all__ = ["HostPipeline", "KvpopError", "check_status", "compact_kv", "decode_attention",
-           "decode_workspace_bytes", "future_target", "future_targets", "keep_mask", "lib",
+           "decode_workspace_bytes", "future_target", "future_targets", "future_targets_fused", "fused_workspace",
+           "keep_mask", "lib",
            "prefix_topk_thresholds", "row_lse", "selftest_bounded_wait"]

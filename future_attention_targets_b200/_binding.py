@@ -54,6 +54,9 @@ _SIGS = {
     "kvpop_decode_attention_noalloc": (ctypes.c_int, [_P, _P, _P, _P, CacheShape, ctypes.c_float, _P, _P, _P]),
     "kvpop_future_targets": (ctypes.c_int, [_P, _P, _I32P, Shape, ctypes.c_float, ctypes.c_int32, ctypes.c_int32,
                                             _I32P, _P, _P, _P, _P, _P]),
+    "kvpop_fused_workspace_bytes": (ctypes.c_size_t, [_I32P, Shape]),
+    "kvpop_future_targets_fused": (ctypes.c_int, [_P, _P, _I32P, Shape, ctypes.c_float, ctypes.c_int32,
+                                                  ctypes.c_int32, _I32P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
     "kvpop_host_workspace_bytes": (ctypes.c_size_t, [Shape]),
     "kvpop_future_targets_host": (ctypes.c_int, [_P, _P, _I32P, Shape, ctypes.c_float, ctypes.c_int32,
                                                  ctypes.c_int32, _I32P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
@@ -282,6 +285,42 @@ def future_targets(q, k, cu_seqlens, window: int, sinks: int, budgets, scale: fl
     _check(lib().kvpop_future_targets(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, int(window), int(sinks), bud,
                                       lse.data_ptr(), target.data_ptr(), keep.data_ptr(), _ptr(status),
                                       _stream_ptr(stream)))
+    return lse, target, keep
+
+
+def fused_workspace(cu_seqlens, n_q_heads: int, n_kv_heads: int, head_dim: int, device=None):
+    """Zero-filled flag workspace for future_targets_fused (reusable: each completed call leaves it zeroed)."""
+    import torch
+    cu, cu_c = _cu_host(cu_seqlens)
+    sh = Shape(len(cu) - 1, int(cu[-1]), n_q_heads, n_kv_heads, head_dim)
+    n = int(lib().kvpop_fused_workspace_bytes(cu_c, sh))
+    if n == 0:
+        raise ValueError("cu_seqlens / head counts do not describe a valid problem")
+    return torch.zeros(n, dtype=torch.uint8, device=torch.device("cuda") if device is None else device)
+
+
+def future_targets_fused(q, k, cu_seqlens, window: int, sinks: int, budgets, scale: float | None = None,
+                         lse=None, target=None, keep=None, workspace=None, status=None, stream=None):
+    """future_targets with both attention passes in one cooperative launch: returns (lse, target, keep)."""
+    import torch
+    _check_qk(q, k)
+    cu, cu_c = _cu_host(cu_seqlens)
+    sh = _shape(q, k, cu)
+    scale = 1.0 / math.sqrt(sh.head_dim) if scale is None else float(scale)
+    dev = q.device
+    if lse is None:
+        lse = torch.empty((sh.n_q_heads, sh.total_tokens), dtype=torch.float32, device=dev)
+    if target is None:
+        target = torch.empty((sh.n_kv_heads, sh.total_tokens), dtype=torch.float32, device=dev)
+    if keep is None:
+        keep = torch.empty((sh.n_kv_heads, sh.total_tokens), dtype=torch.uint8, device=dev)
+    if workspace is None:
+        workspace = fused_workspace(cu, sh.n_q_heads, sh.n_kv_heads, sh.head_dim, device=dev)
+    bud = _i32_host(budgets)
+    _check(lib().kvpop_future_targets_fused(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, int(window), int(sinks),
+                                            bud, lse.data_ptr(), target.data_ptr(), keep.data_ptr(),
+                                            workspace.data_ptr(), workspace.numel(), _ptr(status),
+                                            _stream_ptr(stream)))
     return lse, target, keep
 
 

@@ -25,6 +25,14 @@
 //               columns (each warp reads its TMEM lane quadrant, warp % 4)
 // Two TMEM accumulators of 256 fp32 columns (all 512 columns) let the MMA of
 // tile t+1 run while the softmax warps read tile t.
+//
+// The single-launch variant runs both passes in one persistent cooperative
+// grid: every CTA walks its pass-1 items, then its pass-2 items, with the
+// pipeline state carried across.  Pass-1 writers publish each (query head,
+// 128-row tile) of lse with a release increment on a flag in global memory;
+// the pass-2 producer acquires the flags of a query tile before it reads that
+// tile's lse (through L2), with the same 1 s bound as every other wait.  The
+// last CTA to finish clears the flags for the next launch.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -114,14 +122,31 @@ __device__ __forceinline__ uint32_t slab_row_offset(int r) { return (r >> 3) * k
 
 // ------------------------------------------------------------------ policies
 
+// What a pass needs besides the common parameters: its schedule, tensor maps
+// (A tiles are 128 rows, B tiles 256, so each pass has its own boxes), its
+// output and, in the single-launch variant, the lse readiness flags.
+struct Phase {
+  const LevelSchedule* sched;
+  const CUtensorMap* tmap_q;
+  const CUtensorMap* tmap_k;
+  float* out;                  // pass 1: lse [H_q, T]; pass 2: target [H_kv, T]
+  int32_t* flags;              // single launch: [H_q, n_flag_tiles] counters (else unused)
+  const int32_t* tile_base;    // single launch: first flag tile of each scheduled sequence
+  int32_t n_flag_tiles;
+  int32_t* lse_done;           // single launch: softmax warps that have finished pass 1
+};
+
+// Pass-1 warps that write one item's lse rows; each adds 1 to the tile's flag.
+constexpr int32_t kLseFlagWriters = 4;
+
 // Pass 1: item = (sequence, query tile = level, query head).
 struct LsePass {
   static constexpr bool kSlab = false;
   struct Item {
-    int32_t s, L, g, h, i0, ntiles;
+    int32_t s, L, g, h, i0, ntiles, seq;
   };
-  static __device__ __forceinline__ Item item(const AttnParams& p, int32_t n) {
-    const WorkItem w = decode_item(p.sched, n);
+  static __device__ __forceinline__ Item item(const AttnParams& p, const LevelSchedule& sched, int32_t n) {
+    const WorkItem w = decode_item(sched, n);
     Item it;
     it.s = w.seq_start;
     it.L = w.seq_len;
@@ -129,21 +154,21 @@ struct LsePass {
     it.h = w.head / p.group;
     it.i0 = w.level * kTileRows;
     it.ntiles = it.i0 / kStreamRows + 1;  // key tiles [0,256), [256,512), ... up to the diagonal
+    it.seq = w.seq;
     return it;
   }
   template <int HD>
-  static __device__ __forceinline__ void load_a(const AttnParams& p, const Item& it, uint8_t* dst,
-                                                uint64_t* bar) {
+  static __device__ __forceinline__ void load_a(const Phase& ph, const Item& it, uint8_t* dst, uint64_t* bar) {
 #pragma unroll
     for (int kh = 0; kh < HD / 64; ++kh)
-      tma_load_2d(dst + kh * kTileRows * 128, &p.tmap_q, bar, it.g * HD + kh * 64, it.s + it.i0);
+      tma_load_2d(dst + kh * kTileRows * 128, ph.tmap_q, bar, it.g * HD + kh * 64, it.s + it.i0);
   }
   template <int HD>
-  static __device__ __forceinline__ void load_b(const AttnParams& p, const Item& it, int32_t t, uint8_t* dst,
+  static __device__ __forceinline__ void load_b(const Phase& ph, const Item& it, int32_t t, uint8_t* dst,
                                                 uint64_t* bar) {
 #pragma unroll
     for (int kh = 0; kh < HD / 64; ++kh)
-      tma_load_2d(dst + kh * kStreamRows * 128, &p.tmap_k, bar, it.h * HD + kh * 64, it.s + t * kStreamRows);
+      tma_load_2d(dst + kh * kStreamRows * 128, ph.tmap_k, bar, it.h * HD + kh * 64, it.s + t * kStreamRows);
   }
   // The last key tile holds the diagonal; when the query tile starts on a
   // 256-key boundary only its first 128 columns can be unmasked.
@@ -156,10 +181,10 @@ struct LsePass {
 struct TargetPass {
   static constexpr bool kSlab = true;
   struct Item {
-    int32_t s, L, h, j0, i0, nq, ntiles;
+    int32_t s, L, h, j0, i0, nq, ntiles, seq;
   };
-  static __device__ __forceinline__ Item item(const AttnParams& p, int32_t n) {
-    const WorkItem w = decode_item(p.sched, n);
+  static __device__ __forceinline__ Item item(const AttnParams& p, const LevelSchedule& sched, int32_t n) {
+    const WorkItem w = decode_item(sched, n);
     Item it;
     it.s = w.seq_start;
     it.L = w.seq_len;
@@ -169,23 +194,21 @@ struct TargetPass {
     it.i0 = it.j0 + p.window;
     it.nq = it.i0 < it.L ? (it.L - it.i0 + kStreamRows - 1) / kStreamRows : 0;
     it.ntiles = it.nq * p.group;
+    it.seq = w.seq;
     return it;
   }
   template <int HD>
-  static __device__ __forceinline__ void load_a(const AttnParams& p, const Item& it, uint8_t* dst,
-                                                uint64_t* bar) {
+  static __device__ __forceinline__ void load_a(const Phase& ph, const Item& it, uint8_t* dst, uint64_t* bar) {
 #pragma unroll
     for (int kh = 0; kh < HD / 64; ++kh)
-      tma_load_2d(dst + kh * kTileRows * 128, &p.tmap_k, bar, it.h * HD + kh * 64, it.s + it.j0);
+      tma_load_2d(dst + kh * kTileRows * 128, ph.tmap_k, bar, it.h * HD + kh * 64, it.s + it.j0);
   }
   template <int HD>
-  static __device__ __forceinline__ void load_b(const AttnParams& p, const Item& it, int32_t g, int32_t qt,
+  static __device__ __forceinline__ void load_b(const Phase& ph, const Item& it, int32_t qh, int32_t qt,
                                                 uint8_t* dst, uint64_t* bar) {
-    const int32_t qh = it.h * p.group + g;
 #pragma unroll
     for (int kh = 0; kh < HD / 64; ++kh)
-      tma_load_2d(dst + kh * kStreamRows * 128, &p.tmap_q, bar, qh * HD + kh * 64,
-                  it.s + it.i0 + qt * kStreamRows);
+      tma_load_2d(dst + kh * kStreamRows * 128, ph.tmap_q, bar, qh * HD + kh * 64, it.s + it.i0 + qt * kStreamRows);
   }
   static __device__ __forceinline__ bool half_tile(const Item&, int32_t) { return false; }
 };
@@ -196,12 +219,12 @@ struct TileCursor {
   TargetPass::Item it;
   int32_t g, qt;
   bool have;
-  __device__ __forceinline__ void next_item(const AttnParams& p) {
+  __device__ __forceinline__ void next_item(const AttnParams& p, const LevelSchedule& sched) {
     have = false;
     for (;;) {
       const int32_t n = cta_item(k++, blockIdx.x, gridDim.x);
-      if (n >= p.sched.total_items) return;
-      it = TargetPass::item(p, n);
+      if (n >= sched.total_items) return;
+      it = TargetPass::item(p, sched, n);
       if (it.ntiles > 0) {
         g = 0;
         qt = 0;
@@ -210,16 +233,30 @@ struct TileCursor {
       }
     }
   }
-  __device__ __forceinline__ void start(const AttnParams& p) {
+  __device__ __forceinline__ void start(const AttnParams& p, const LevelSchedule& sched) {
     k = 0;
-    next_item(p);
+    next_item(p, sched);
   }
-  __device__ __forceinline__ void advance(const AttnParams& p) {
+  __device__ __forceinline__ void advance(const AttnParams& p, const LevelSchedule& sched) {
     if (++qt == it.nq) {
       qt = 0;
-      if (++g == p.group) next_item(p);
+      if (++g == p.group) next_item(p, sched);
     }
   }
+};
+
+// Pipeline counters of each role, carried from one phase to the next.
+struct ProducerState {
+  uint32_t a_cnt = 0, b_cnt = 0;
+  bool ok = true;
+};
+struct MmaState {
+  uint32_t a_cnt = 0, b_cnt = 0, acc_cnt = 0;
+  bool ok = true, issued = false;
+};
+struct SoftmaxState {
+  uint32_t acc_cnt = 0, item_cnt = 0;
+  bool ok = true;
 };
 
 // ------------------------------------------------------------------ roles
@@ -238,8 +275,57 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity, const
   return wait_bounded(bar, parity, c2, SITE_TEARDOWN);
 }
 
+// Single launch: waits until every 128-row lse tile under the cursor's 256
+// query rows has been published.  Lanes 0..2 poll the (at most three) tile
+// flags and lane 31 the count of softmax warps that finished pass 1, all in
+// one round trip; once every CTA's pass 1 is done (*all_lse) no flag is read
+// again.  Bounded like every other wait; warp-uniform result.
+template <bool kFused>
+__device__ __forceinline__ bool norm_ready(const AttnParams& p, const Phase& ph, const TileCursor& cur, int lane,
+                                           const WaitCtl& ctl, bool& all_lse) {
+  if constexpr (!kFused) {
+    return true;
+  } else {
+    if (all_lse) return true;
+    const int32_t qh = cur.it.h * p.group + cur.g;
+    const int32_t a = cur.it.i0 + cur.qt * kStreamRows;
+    const int32_t b = min(a + kStreamRows, cur.it.L);
+    const int32_t t0 = a / kTileRows, nt = (b - 1) / kTileRows - t0 + 1;
+    const int32_t* f = ph.flags + static_cast<int64_t>(qh) * ph.n_flag_tiles + ph.tile_base[cur.it.seq] + t0;
+    const int32_t all_warps = kSoftmaxWarps * static_cast<int32_t>(gridDim.x);
+    uint64_t t_start = 0;
+    for (uint32_t it = 0;; ++it) {
+      bool mine = true;
+      if (lane < nt) mine = flag_acquire_load(f + lane) >= kLseFlagWriters;
+      const bool done_all = (lane == 31) && flag_acquire_load(ph.lse_done) >= all_warps;
+      if (__any_sync(0xffffffffu, done_all)) {
+        all_lse = true;
+        return true;
+      }
+      if (__all_sync(0xffffffffu, mine)) return true;
+      int give_up = 0;
+      if (lane == 0 && (it & 15u) == 0u) {
+        const uint64_t now = global_timer_ns();
+        if (it == 0) t_start = now;
+        if (*ctl.abort_flag) {
+          give_up = 1;
+        } else if (now - t_start > ctl.limit_ns) {
+          *ctl.abort_flag = 1;
+          if (ctl.status != nullptr) atomicCAS(ctl.status, 0, 4 | (SITE_LSE_FLAG << 8));
+          give_up = 1;
+        }
+      }
+      if (__shfl_sync(0xffffffffu, give_up, 0)) return false;
+      __nanosleep(64);
+    }
+  }
+}
+
 // Normaliser rows of one pass-2 B tile, this lane's 8 rows (lane + 32 m):
-// lse_i / s, or kPastEnd past the sequence end.
+// lse_i / s, or kPastEnd past the sequence end.  In the single launch the
+// lse rows were written by other CTAs during this launch, so they are read
+// through L2 (ld.global.cg), never from a possibly stale L1 line.
+template <bool kFused>
 __device__ __forceinline__ void load_norm_rows(const AttnParams& p, const TileCursor& cur, int lane,
                                                float (&v)[8]) {
   const int32_t qh = cur.it.h * p.group + cur.g;
@@ -247,7 +333,8 @@ __device__ __forceinline__ void load_norm_rows(const AttnParams& p, const TileCu
 #pragma unroll
   for (int m = 0; m < 8; ++m) {
     const int32_t i = cur.it.i0 + cur.qt * kStreamRows + lane + 32 * m;
-    v[m] = (i < cur.it.L) ? __ldg(src + i) * p.inv_scale : kPastEnd;
+    const float x = (i < cur.it.L) ? (kFused ? __ldcg(src + i) : __ldg(src + i)) : 0.f;
+    v[m] = (i < cur.it.L) ? x * p.inv_scale : kPastEnd;
   }
 }
 
@@ -269,109 +356,139 @@ __device__ __forceinline__ void store_norm_rows(uint8_t* slab, int lane, const f
   }
 }
 
-template <class Pass, int HD>
-__device__ void producer_role(const AttnParams& p, uint8_t* smem, const Bars& bars, const WaitCtl& ctl) {
-  using L = SmemLayout<HD, Pass::kSlab>;
+// One pass of the TMA producer warp.  kFused: the single launch, whose B
+// stages complete with 32 lane arrivals in both passes (pass 2 needs them
+// for the slab rows) and whose pass-2 normalisers wait for their lse flags.
+template <class Pass, int HD, bool kFused>
+__device__ void producer_phase(const AttnParams& p, const Phase& ph, uint8_t* smem, const Bars& bars,
+                               const WaitCtl& ctl, ProducerState& st) {
+  using L = SmemLayout<HD, Pass::kSlab || kFused>;
   const int lane = threadIdx.x & 31;
-  uint32_t a_cnt = 0, b_cnt = 0;
-  bool ok = true;
-  const int32_t total = p.sched.total_items;
+  const LevelSchedule& sched = *ph.sched;
+  const int32_t total = sched.total_items;
   // Pass 2: normaliser values of the next tile, loaded one tile ahead.
   TileCursor nxt;
   float norm[8];
+  bool all_lse = false;
   if constexpr (Pass::kSlab) {
-    nxt.start(p);
-    if (nxt.have) load_norm_rows(p, nxt, lane, norm);
+    nxt.start(p, sched);
+    if (nxt.have) {
+      if (!norm_ready<kFused>(p, ph, nxt, lane, ctl, all_lse)) {
+        st.ok = false;
+        return;
+      }
+      load_norm_rows<kFused>(p, nxt, lane, norm);
+    }
   }
-  for (int32_t k = 0; ok; ++k) {
+  for (int32_t k = 0; st.ok; ++k) {
     const int32_t n = cta_item(k, blockIdx.x, gridDim.x);
     if (n >= total) break;
-    const typename Pass::Item it = Pass::item(p, n);
+    const typename Pass::Item it = Pass::item(p, sched, n);
     if (it.ntiles == 0) continue;
-    const uint32_t ab = a_cnt & 1u;
-    if (!warp_wait(&bars.a_empty[ab], ((a_cnt >> 1) & 1u) ^ 1u, ctl, SITE_PRODUCER_A_EMPTY)) {
-      ok = false;
+    const uint32_t ab = st.a_cnt & 1u;
+    if (!warp_wait(&bars.a_empty[ab], ((st.a_cnt >> 1) & 1u) ^ 1u, ctl, SITE_PRODUCER_A_EMPTY)) {
+      st.ok = false;
       break;
     }
     if (lane == 0) {
       mbar_arrive_expect_tx(&bars.a_full[ab], L::A_BYTES);
-      Pass::template load_a<HD>(p, it, smem + L::OFF_A + ab * L::A_BYTES, &bars.a_full[ab]);
+      Pass::template load_a<HD>(ph, it, smem + L::OFF_A + ab * L::A_BYTES, &bars.a_full[ab]);
     }
-    ++a_cnt;
+    ++st.a_cnt;
     for (int32_t t = 0; t < it.ntiles; ++t) {
-      const uint32_t st = b_cnt % kStages;
-      if (!warp_wait(&bars.b_empty[st], ((b_cnt / kStages) & 1u) ^ 1u, ctl, SITE_PRODUCER_B_EMPTY)) {
-        ok = false;
+      const uint32_t sg = st.b_cnt % kStages;
+      if (!warp_wait(&bars.b_empty[sg], ((st.b_cnt / kStages) & 1u) ^ 1u, ctl, SITE_PRODUCER_B_EMPTY)) {
+        st.ok = false;
         break;
       }
-      uint8_t* stage = smem + L::OFF_B + st * L::B_STAGE;
+      uint8_t* stage = smem + L::OFF_B + sg * L::B_STAGE;
       if constexpr (Pass::kSlab) {
         // Tile bytes are expected before the loads are issued; the 32 lane
         // arrivals below (after their slab rows are written) complete the phase.
         const int32_t g = t / it.nq, qt = t - g * it.nq;
         if (lane == 0) {
-          mbar_expect_tx(&bars.b_full[st], L::B_TILE);
-          Pass::template load_b<HD>(p, it, g, qt, stage, &bars.b_full[st]);
+          mbar_expect_tx(&bars.b_full[sg], L::B_TILE);
+          Pass::template load_b<HD>(ph, it, it.h * p.group + g, qt, stage, &bars.b_full[sg]);
         }
         float cur[8];
 #pragma unroll
         for (int m = 0; m < 8; ++m) cur[m] = norm[m];
-        nxt.advance(p);
-        if (nxt.have) load_norm_rows(p, nxt, lane, norm);
+        nxt.advance(p, sched);
+        bool ready = true;
+        if (nxt.have) {
+          ready = norm_ready<kFused>(p, ph, nxt, lane, ctl, all_lse);
+          if (ready) load_norm_rows<kFused>(p, nxt, lane, norm);
+        }
         store_norm_rows(stage + L::B_TILE, lane, cur);
         fence_proxy_async_smem();
-        mbar_arrive(&bars.b_full[st]);
+        mbar_arrive(&bars.b_full[sg]);
+        ++st.b_cnt;
+        if (!ready) {
+          st.ok = false;
+          break;
+        }
+      } else if constexpr (kFused) {
+        if (lane == 0) {
+          mbar_expect_tx(&bars.b_full[sg], L::B_TILE);
+          Pass::template load_b<HD>(ph, it, t, stage, &bars.b_full[sg]);
+        }
+        __syncwarp();
+        mbar_arrive(&bars.b_full[sg]);
+        ++st.b_cnt;
       } else {
         if (lane == 0) {
-          mbar_arrive_expect_tx(&bars.b_full[st], L::B_TILE);
-          Pass::template load_b<HD>(p, it, t, stage, &bars.b_full[st]);
+          mbar_arrive_expect_tx(&bars.b_full[sg], L::B_TILE);
+          Pass::template load_b<HD>(ph, it, t, stage, &bars.b_full[sg]);
         }
+        ++st.b_cnt;
       }
-      ++b_cnt;
-    }
-  }
-  if (!ok && lane == 0) {
-    // Let every TMA load issued by this warp land before the CTA exits.
-    for (uint32_t ab = 0; ab < 2; ++ab) {
-      if (a_cnt > ab) wait_drain(&bars.a_full[ab], (((a_cnt - ab + 1) / 2) - 1) & 1u, ctl);
-    }
-    for (uint32_t st = 0; st < kStages; ++st) {
-      if (b_cnt > st) wait_drain(&bars.b_full[st], (((b_cnt - st + kStages - 1) / kStages) - 1) & 1u, ctl);
     }
   }
 }
 
-template <class Pass, int HD>
-__device__ void mma_role(const AttnParams& p, uint8_t* smem, const Bars& bars, const WaitCtl& ctl,
-                         uint32_t tmem_base) {
-  using L = SmemLayout<HD, Pass::kSlab>;
-  uint32_t a_cnt = 0, b_cnt = 0, acc_cnt = 0;
-  bool ok = true, issued = false;
-  const int32_t total = p.sched.total_items;
+// After an abort: let every TMA load issued by the producer land before the
+// CTA exits.
+__device__ void producer_drain(const Bars& bars, const WaitCtl& ctl, const ProducerState& st) {
+  if (st.ok || (threadIdx.x & 31) != 0) return;
+  for (uint32_t ab = 0; ab < 2; ++ab) {
+    if (st.a_cnt > ab) wait_drain(&bars.a_full[ab], (((st.a_cnt - ab + 1) / 2) - 1) & 1u, ctl);
+  }
+  for (uint32_t sg = 0; sg < kStages; ++sg) {
+    if (st.b_cnt > sg) wait_drain(&bars.b_full[sg], (((st.b_cnt - sg + kStages - 1) / kStages) - 1) & 1u, ctl);
+  }
+}
+
+// One pass of the single-thread MMA issuer.
+template <class Pass, int HD, bool kFused>
+__device__ void mma_phase(const AttnParams& p, const Phase& ph, uint8_t* smem, const Bars& bars, const WaitCtl& ctl,
+                          uint32_t tmem_base, MmaState& st) {
+  using L = SmemLayout<HD, Pass::kSlab || kFused>;
+  const LevelSchedule& sched = *ph.sched;
+  const int32_t total = sched.total_items;
   const uint32_t idesc_full = umma_idesc_bf16(kTileRows, kStreamRows);
   const uint32_t idesc_half = umma_idesc_bf16(kTileRows, kStreamRows / 2);
-  for (int32_t k = 0; ok; ++k) {
+  for (int32_t k = 0; st.ok; ++k) {
     const int32_t n = cta_item(k, blockIdx.x, gridDim.x);
     if (n >= total) break;
-    const typename Pass::Item it = Pass::item(p, n);
+    const typename Pass::Item it = Pass::item(p, sched, n);
     if (it.ntiles == 0) continue;
-    const uint32_t ab = a_cnt & 1u;
-    if (!wait_bounded(&bars.a_full[ab], (a_cnt >> 1) & 1u, ctl, SITE_MMA_A_FULL)) {
-      ok = false;
+    const uint32_t ab = st.a_cnt & 1u;
+    if (!wait_bounded(&bars.a_full[ab], (st.a_cnt >> 1) & 1u, ctl, SITE_MMA_A_FULL)) {
+      st.ok = false;
       break;
     }
     tc_fence_after_sync();
     const uint32_t a_addr = smem_u32(smem + L::OFF_A + ab * L::A_BYTES);
     for (int32_t t = 0; t < it.ntiles; ++t) {
-      const uint32_t st = b_cnt % kStages;
-      const uint32_t acc = acc_cnt & 1u;
-      if (!wait_bounded(&bars.b_full[st], (b_cnt / kStages) & 1u, ctl, SITE_MMA_B_FULL) ||
-          !wait_bounded(&bars.acc_empty[acc], ((acc_cnt >> 1) & 1u) ^ 1u, ctl, SITE_MMA_ACC_EMPTY)) {
-        ok = false;
+      const uint32_t sg = st.b_cnt % kStages;
+      const uint32_t acc = st.acc_cnt & 1u;
+      if (!wait_bounded(&bars.b_full[sg], (st.b_cnt / kStages) & 1u, ctl, SITE_MMA_B_FULL) ||
+          !wait_bounded(&bars.acc_empty[acc], ((st.acc_cnt >> 1) & 1u) ^ 1u, ctl, SITE_MMA_ACC_EMPTY)) {
+        st.ok = false;
         break;
       }
       tc_fence_after_sync();
-      const uint32_t b_addr = smem_u32(smem + L::OFF_B + st * L::B_STAGE);
+      const uint32_t b_addr = smem_u32(smem + L::OFF_B + sg * L::B_STAGE);
       const uint32_t d_tmem = tmem_base + acc * kStreamRows;
       const uint32_t idesc = Pass::half_tile(it, t) ? idesc_half : idesc_full;
 #pragma unroll
@@ -386,18 +503,21 @@ __device__ void mma_role(const AttnParams& p, uint8_t* smem, const Bars& bars, c
         umma_bf16(d_tmem, umma_desc_slab(smem_u32(smem + L::OFF_ASLAB)), umma_desc_slab(b_addr + L::B_TILE),
                   idesc, 1u);
       }
-      issued = true;
-      umma_commit(&bars.b_empty[st]);
+      st.issued = true;
+      umma_commit(&bars.b_empty[sg]);
       umma_commit(&bars.acc_full[acc]);
-      ++b_cnt;
-      ++acc_cnt;
+      ++st.b_cnt;
+      ++st.acc_cnt;
     }
-    if (!ok) break;
+    if (!st.ok) break;
     umma_commit(&bars.a_empty[ab]);
-    ++a_cnt;
+    ++st.a_cnt;
   }
-  if (issued) {
-    // Every MMA issued here must be finished before TMEM is released.
+}
+
+// Every MMA issued must be finished before TMEM is released.
+__device__ void mma_finish(const Bars& bars, const WaitCtl& ctl, const MmaState& st) {
+  if (st.issued) {
     umma_commit(bars.mma_done);
     wait_drain(bars.mma_done, 0, ctl);
   }
@@ -596,10 +716,10 @@ __device__ __forceinline__ float half_tile_max(uint32_t taddr, float c, int lo, 
 
 // ------------------------------------------------------------------ softmax: pass 1
 
-template <int HD>
-__device__ void lse_softmax_role(const AttnParams& p, uint8_t* smem, const Bars& bars, const WaitCtl& ctl,
-                                 uint32_t tmem_base) {
-  using L = SmemLayout<HD, false>;
+template <int HD, bool kFused>
+__device__ void lse_softmax_phase(const AttnParams& p, const Phase& ph, uint8_t* smem, const Bars& bars,
+                                  const WaitCtl& ctl, uint32_t tmem_base, SoftmaxState& st) {
+  using L = SmemLayout<HD, kFused>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sw = warp - 2;                 // softmax warp 0..7
   const int wg = sw >> 2;                  // column half
@@ -611,18 +731,17 @@ __device__ void lse_softmax_role(const AttnParams& p, uint8_t* smem, const Bars&
   const uint64_t c2 = f2_pack(c, c);
   const float kBig = 18446744073709551616.0f;   // 2^64: larger tile sums force an exact rescale
   const float kRebase = 4294967296.0f;          // 2^32: keep the running sum moderate
-  uint32_t acc_cnt = 0, item_cnt = 0;
-  bool ok = true;
-  const int32_t total = p.sched.total_items;
-  for (int32_t k = 0; ok; ++k) {
+  const LevelSchedule& sched = *ph.sched;
+  const int32_t total = sched.total_items;
+  for (int32_t k = 0; st.ok; ++k) {
     const int32_t n = cta_item(k, blockIdx.x, gridDim.x);
     if (n >= total) break;
-    const LsePass::Item it = LsePass::item(p, n);
+    const LsePass::Item it = LsePass::item(p, sched, n);
     float off = -INFINITY, sum = 0.f;      // running offset (log2 units) and sum of exp2(y - off)
     for (int32_t t = 0; t < it.ntiles; ++t) {
-      const uint32_t acc = acc_cnt & 1u;
-      if (!warp_wait(&bars.acc_full[acc], (acc_cnt >> 1) & 1u, ctl, SITE_SOFTMAX_ACC_FULL)) {
-        ok = false;
+      const uint32_t acc = st.acc_cnt & 1u;
+      if (!warp_wait(&bars.acc_full[acc], (st.acc_cnt >> 1) & 1u, ctl, SITE_SOFTMAX_ACC_FULL)) {
+        st.ok = false;
         break;
       }
       tc_fence_after_sync();
@@ -664,35 +783,50 @@ __device__ void lse_softmax_role(const AttnParams& p, uint8_t* smem, const Bars&
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.acc_empty[acc]);
-      ++acc_cnt;
+      ++st.acc_cnt;
     }
-    if (!ok) break;
+    if (!st.ok) break;
     // Combine the two column halves of each row.
     if (wg == 1) {
-      if (!warp_wait(bars.comb_empty, (item_cnt & 1u) ^ 1u, ctl, SITE_SOFTMAX_ACC_FULL)) break;
+      if (!warp_wait(bars.comb_empty, (st.item_cnt & 1u) ^ 1u, ctl, SITE_SOFTMAX_ACC_FULL)) {
+        st.ok = false;
+        break;
+      }
       comb[row] = off;
       comb[128 + row] = sum;
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.comb_full);
     } else {
-      if (!warp_wait(bars.comb_full, item_cnt & 1u, ctl, SITE_SOFTMAX_ACC_FULL)) break;
+      if (!warp_wait(bars.comb_full, st.item_cnt & 1u, ctl, SITE_SOFTMAX_ACC_FULL)) {
+        st.ok = false;
+        break;
+      }
       const float off1 = comb[row], sum1 = comb[128 + row];
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.comb_empty);
       const float m = fmaxf(off, off1);
       const float s = sum * ex2_approx(off - m) + (off1 > -INFINITY ? sum1 * ex2_approx(off1 - m) : 0.f);
       const int32_t i = it.i0 + row;
-      if (i < it.L) p.out[static_cast<int64_t>(it.g) * p.total_tokens + it.s + i] = (m + log2f(s)) * kLn2;
+      if (i < it.L) ph.out[static_cast<int64_t>(it.g) * p.total_tokens + it.s + i] = (m + log2f(s)) * kLn2;
+      if constexpr (kFused) {
+        // Publish this warp's 32 rows: the warp barrier orders every lane's
+        // store before lane 0's gpu-scope release.
+        __syncwarp();
+        if (lane == 0)
+          flag_release_add(ph.flags + static_cast<int64_t>(it.g) * ph.n_flag_tiles + ph.tile_base[it.seq] +
+                               it.i0 / kTileRows,
+                           1);
+      }
     }
-    ++item_cnt;
+    ++st.item_cnt;
   }
 }
 
 // ------------------------------------------------------------------ softmax: pass 2
 
 template <int HD>
-__device__ void target_softmax_role(const AttnParams& p, uint8_t* smem, const Bars& bars, const WaitCtl& ctl,
-                                    uint32_t tmem_base) {
+__device__ void target_softmax_phase(const AttnParams& p, const Phase& ph, uint8_t* smem, const Bars& bars,
+                                     const WaitCtl& ctl, uint32_t tmem_base, SoftmaxState& st) {
   using L = SmemLayout<HD, true>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sw = warp - 2;
@@ -704,20 +838,19 @@ __device__ void target_softmax_role(const AttnParams& p, uint8_t* smem, const Ba
   const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
   const uint64_t zero2 = f2_pack(0.f, 0.f);
   const float xmin = -126.f / p.scale_log2;   // below it exp2(c x) < 2^-126: clamp for the polynomial
-  const int32_t total = p.sched.total_items;
-  uint32_t acc_cnt = 0, item_cnt = 0;
-  bool ok = true;
-  for (int32_t k = 0; ok; ++k) {
+  const LevelSchedule& sched = *ph.sched;
+  const int32_t total = sched.total_items;
+  for (int32_t k = 0; st.ok; ++k) {
     const int32_t n = cta_item(k, blockIdx.x, gridDim.x);
     if (n >= total) break;
-    const TargetPass::Item it = TargetPass::item(p, n);
+    const TargetPass::Item it = TargetPass::item(p, sched, n);
     float run = 0.f, comp = 0.f;           // Kahan-compensated running sum over tiles
     const bool ragged_end = it.i0 + it.nq * kStreamRows > it.L;
-    for (int32_t g = 0; g < (it.nq > 0 ? p.group : 0) && ok; ++g) {
+    for (int32_t g = 0; g < (it.nq > 0 ? p.group : 0) && st.ok; ++g) {
       for (int32_t qt = 0; qt < it.nq; ++qt) {
-        const uint32_t acc = acc_cnt & 1u;
-        if (!warp_wait(&bars.acc_full[acc], (acc_cnt >> 1) & 1u, ctl, SITE_SOFTMAX_ACC_FULL)) {
-          ok = false;
+        const uint32_t acc = st.acc_cnt & 1u;
+        if (!warp_wait(&bars.acc_full[acc], (st.acc_cnt >> 1) & 1u, ctl, SITE_SOFTMAX_ACC_FULL)) {
+          st.ok = false;
           break;
         }
         tc_fence_after_sync();
@@ -733,28 +866,34 @@ __device__ void target_softmax_role(const AttnParams& p, uint8_t* smem, const Ba
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.acc_empty[acc]);
-        ++acc_cnt;
+        ++st.acc_cnt;
         const float yk = ts - comp;
         const float tk = run + yk;
         comp = (tk - run) - yk;
         run = tk;
       }
     }
-    if (!ok) break;
+    if (!st.ok) break;
     if (wg == 1) {
-      if (!warp_wait(bars.comb_empty, (item_cnt & 1u) ^ 1u, ctl, SITE_SOFTMAX_ACC_FULL)) break;
+      if (!warp_wait(bars.comb_empty, (st.item_cnt & 1u) ^ 1u, ctl, SITE_SOFTMAX_ACC_FULL)) {
+        st.ok = false;
+        break;
+      }
       comb[row] = run;
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.comb_full);
     } else {
-      if (!warp_wait(bars.comb_full, item_cnt & 1u, ctl, SITE_SOFTMAX_ACC_FULL)) break;
+      if (!warp_wait(bars.comb_full, st.item_cnt & 1u, ctl, SITE_SOFTMAX_ACC_FULL)) {
+        st.ok = false;
+        break;
+      }
       const float other = comb[row];
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.comb_empty);
       const int32_t j = it.j0 + row;
-      if (j < it.L) p.out[static_cast<int64_t>(it.h) * p.total_tokens + it.s + j] = run + other;
+      if (j < it.L) ph.out[static_cast<int64_t>(it.h) * p.total_tokens + it.s + j] = run + other;
     }
-    ++item_cnt;
+    ++st.item_cnt;
   }
 }
 
@@ -764,16 +903,13 @@ __device__ __forceinline__ uint8_t* aligned_smem(uint8_t* raw) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~static_cast<uintptr_t>(1023));
 }
 
-template <class Pass, int HD>
-__device__ __forceinline__ void attn_kernel_body(const AttnParams& p, uint8_t* smem_raw) {
-  using L = SmemLayout<HD, Pass::kSlab>;
-  uint8_t* smem = aligned_smem(smem_raw);
-  const Bars bars = carve_bars(reinterpret_cast<uint64_t*>(smem + L::OFF_BAR));
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  if constexpr (Pass::kSlab) {
+// Barriers, slab constants and TMEM of one CTA.  kSlab: the pass-2 layout
+// (normaliser slabs; B stages completed by 32 lane arrivals).
+template <int HD, bool kSlab>
+__device__ __forceinline__ void cta_setup(uint8_t* smem, const Bars& bars, uint32_t* tmem_slot,
+                                          volatile int* abort_flag) {
+  using L = SmemLayout<HD, kSlab>;
+  if constexpr (kSlab) {
     // Zero the extra K-columns of A and of every B stage, then put the ones in A.
     for (int s = 0; s < kStages; ++s) {
       uint32_t* z = reinterpret_cast<uint32_t*>(smem + L::OFF_B + s * L::B_STAGE + L::B_TILE);
@@ -797,7 +933,7 @@ __device__ __forceinline__ void attn_kernel_body(const AttnParams& p, uint8_t* s
       mbar_init(&bars.acc_empty[i], kSoftmaxWarps);
     }
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&bars.b_full[i], Pass::kSlab ? 32 : 1);
+      mbar_init(&bars.b_full[i], kSlab ? 32 : 1);
       mbar_init(&bars.b_empty[i], 1);
     }
     mbar_init(bars.comb_full, 4);
@@ -806,38 +942,60 @@ __device__ __forceinline__ void attn_kernel_body(const AttnParams& p, uint8_t* s
     *abort_flag = 0;
     fence_mbarrier_init();
   }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_map(&p.tmap_q);
-    tma_prefetch_map(&p.tmap_k);
-  }
-  if (warp == 1) {
+  if ((threadIdx.x >> 5) == 1) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
     tc_fence_before_sync();
   }
   __syncthreads();
   tc_fence_after_sync();
-  const uint32_t tmem_base = *tmem_slot;
-  const WaitCtl ctl{abort_flag, p.status, p.wait_ns};
+}
 
-  if (warp == 0) {
-    producer_role<Pass, HD>(p, smem, bars, ctl);
-  } else if (warp == 1) {
-    if (lane == 0) mma_role<Pass, HD>(p, smem, bars, ctl, tmem_base);
-  } else {
-    if constexpr (std::is_same<Pass, LsePass>::value)
-      lse_softmax_role<HD>(p, smem, bars, ctl, tmem_base);
-    else
-      target_softmax_role<HD>(p, smem, bars, ctl, tmem_base);
-  }
-
+__device__ __forceinline__ void cta_teardown(uint32_t tmem_base) {
   tc_fence_before_sync();
   __syncthreads();
-  if (warp == 1) {
+  if ((threadIdx.x >> 5) == 1) {
     __syncwarp();
     tc_fence_after_sync();
     tmem_dealloc(tmem_base, 512);
   }
+}
+
+template <class Pass, int HD>
+__device__ __forceinline__ void attn_kernel_body(const AttnParams& p, uint8_t* smem_raw) {
+  using L = SmemLayout<HD, Pass::kSlab>;
+  uint8_t* smem = aligned_smem(smem_raw);
+  const Bars bars = carve_bars(reinterpret_cast<uint64_t*>(smem + L::OFF_BAR));
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&p.tmap_q);
+    tma_prefetch_map(&p.tmap_k);
+  }
+  cta_setup<HD, Pass::kSlab>(smem, bars, tmem_slot, abort_flag);
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitCtl ctl{abort_flag, p.status, p.wait_ns};
+  const Phase ph{&p.sched, &p.tmap_q, &p.tmap_k, p.out, nullptr, nullptr, 0, nullptr};
+
+  if (warp == 0) {
+    ProducerState st;
+    producer_phase<Pass, HD, false>(p, ph, smem, bars, ctl, st);
+    producer_drain(bars, ctl, st);
+  } else if (warp == 1) {
+    if (lane == 0) {
+      MmaState st;
+      mma_phase<Pass, HD, false>(p, ph, smem, bars, ctl, tmem_base, st);
+      mma_finish(bars, ctl, st);
+    }
+  } else {
+    SoftmaxState st;
+    if constexpr (std::is_same<Pass, LsePass>::value)
+      lse_softmax_phase<HD, false>(p, ph, smem, bars, ctl, tmem_base, st);
+    else
+      target_softmax_phase<HD>(p, ph, smem, bars, ctl, tmem_base, st);
+  }
+  cta_teardown(tmem_base);
 }
 
 template <int HD>
@@ -850,6 +1008,71 @@ template <int HD>
 __global__ void __launch_bounds__(kThreads, 1) future_target_kernel(const __grid_constant__ AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   attn_kernel_body<TargetPass, HD>(p, smem_raw);
+}
+
+// Both passes in one cooperative launch (one CTA per SM, all co-resident, so
+// a CTA waiting for another CTA's lse tile always has that CTA running).
+// Each role runs pass 1, then pass 2 with its pipeline counters carried over;
+// a role whose pass 1 gave up skips pass 2.
+template <int HD>
+__global__ void __launch_bounds__(kThreads, 1) fused_targets_kernel(const __grid_constant__ FusedParams fp) {
+  extern __shared__ uint8_t smem_raw[];
+  using L = SmemLayout<HD, true>;
+  const AttnParams& p = fp.attn;
+  uint8_t* smem = aligned_smem(smem_raw);
+  const Bars bars = carve_bars(reinterpret_cast<uint64_t*>(smem + L::OFF_BAR));
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+  volatile int* last_cta = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 8);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&p.tmap_q);
+    tma_prefetch_map(&p.tmap_k);
+    tma_prefetch_map(&fp.tmap_q_stream);
+    tma_prefetch_map(&fp.tmap_k_tile);
+  }
+  cta_setup<HD, true>(smem, bars, tmem_slot, abort_flag);
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitCtl ctl{abort_flag, p.status, p.wait_ns};
+  const Phase ph1{&p.sched, &p.tmap_q, &p.tmap_k, p.out, fp.flags, fp.tile_base_lse, fp.n_flag_tiles, fp.lse_done};
+  const Phase ph2{&fp.sched_target, &fp.tmap_q_stream, &fp.tmap_k_tile, fp.target, fp.flags,
+                  fp.tile_base_target, fp.n_flag_tiles, fp.lse_done};
+
+  if (warp == 0) {
+    ProducerState st;
+    producer_phase<LsePass, HD, true>(p, ph1, smem, bars, ctl, st);
+    if (st.ok) producer_phase<TargetPass, HD, true>(p, ph2, smem, bars, ctl, st);
+    producer_drain(bars, ctl, st);
+  } else if (warp == 1) {
+    if (lane == 0) {
+      MmaState st;
+      mma_phase<LsePass, HD, true>(p, ph1, smem, bars, ctl, tmem_base, st);
+      if (st.ok) mma_phase<TargetPass, HD, true>(p, ph2, smem, bars, ctl, tmem_base, st);
+      mma_finish(bars, ctl, st);
+    }
+  } else {
+    SoftmaxState st;
+    lse_softmax_phase<HD, true>(p, ph1, smem, bars, ctl, tmem_base, st);
+    if (st.ok) {
+      // This warp's pass-1 rows are all written (and published tile by tile).
+      __syncwarp();
+      if (lane == 0) flag_release_add(fp.lse_done, 1);
+      target_softmax_phase<HD>(p, ph2, smem, bars, ctl, tmem_base, st);
+    }
+  }
+  cta_teardown(tmem_base);
+
+  // The last CTA out (every other CTA has finished all its flag traffic)
+  // clears the flags and the counter, leaving the workspace zeroed.
+  if (threadIdx.x == 0) *last_cta = (flag_arrive_count(fp.done) == static_cast<int32_t>(gridDim.x) - 1) ? 1 : 0;
+  __syncthreads();
+  if (*last_cta) {
+    for (int32_t i = threadIdx.x; i < fp.n_flags; i += blockDim.x) fp.flags[i] = 0;
+    if (threadIdx.x == 0) {
+      *fp.done = 0;
+      *fp.lse_done = 0;
+    }
+  }
 }
 
 // ------------------------------------------------------------------ launchers
@@ -870,6 +1093,21 @@ cudaError_t launch_row_lse(const AttnParams& p, int head_dim, int grid, cudaStre
 
 cudaError_t launch_future_target(const AttnParams& p, int head_dim, int grid, cudaStream_t stream) {
   return head_dim == 64 ? launch_attn<64, true>(p, grid, stream) : launch_attn<128, true>(p, grid, stream);
+}
+
+template <int HD>
+static cudaError_t launch_fused_hd(const FusedParams& fp, int grid, cudaStream_t stream) {
+  using L = SmemLayout<HD, true>;
+  cudaError_t e =
+      cudaFuncSetAttribute(fused_targets_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+  if (e != cudaSuccess) return e;
+  void* args[] = {const_cast<FusedParams*>(&fp)};
+  return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(fused_targets_kernel<HD>), dim3(grid),
+                                     dim3(kThreads), args, L::ALLOC, stream);
+}
+
+cudaError_t launch_fused_targets(const FusedParams& fp, int head_dim, int grid, cudaStream_t stream) {
+  return head_dim == 64 ? launch_fused_hd<64>(fp, grid, stream) : launch_fused_hd<128>(fp, grid, stream);
 }
 
 // ------------------------------------------------------------------ bounded-wait self-test

@@ -23,6 +23,7 @@ cudaError_t launch_selftest_wait(int32_t* status, uint64_t limit_ns, cudaStream_
 cudaError_t launch_prefix_thresholds(const ThresholdParams& p, int n_kv_heads, cudaStream_t stream);
 cudaError_t launch_compact_kv(const CompactParams& p, cudaStream_t stream);
 cudaError_t launch_decode_attention(const DecodeParams& p, int batch, cudaStream_t stream);
+cudaError_t launch_fused_targets(const FusedParams& fp, int head_dim, int grid, cudaStream_t stream);
 size_t decode_scratch_bytes();
 cudaError_t decode_scratch_address(float** out);
 }  // namespace kvpop
@@ -159,7 +160,8 @@ kvpop_status check_qk(const void* q, const void* k, float scale) {
 
 // Items (level, sequence, head), heaviest level first.  Sequences with t
 // 128-row tiles take part in levels 0 .. t-1.
-void build_schedule(const int32_t* cu, int batch, int n_heads, LevelSchedule* s) {
+// order (optional) receives the original index of each scheduled sequence.
+void build_schedule(const int32_t* cu, int batch, int n_heads, LevelSchedule* s, std::vector<int>* order = nullptr) {
   std::vector<std::pair<int, int>> seqs;  // (tiles, index)
   for (int b = 0; b < batch; ++b) {
     const int L = cu[b + 1] - cu[b];
@@ -177,6 +179,10 @@ void build_schedule(const int32_t* cu, int batch, int n_heads, LevelSchedule* s)
     s->seq_start[r] = cu[seqs[r].second];
     s->seq_len[r] = cu[seqs[r].second + 1] - cu[seqs[r].second];
   }
+  if (order != nullptr) {
+    order->clear();
+    for (const auto& e : seqs) order->push_back(e.second);
+  }
   int32_t running = 0;
   size_t active = 0;  // sequences with a tile at this level form a prefix of the sorted list
   for (int k = 0; k < s->n_levels; ++k) {
@@ -192,7 +198,8 @@ void build_schedule(const int32_t* cu, int batch, int n_heads, LevelSchedule* s)
 int grid_for(int items, int sm_count) { return std::max(1, std::min(items, sm_count)); }
 
 kvpop_status fill_attn_common(AttnParams* p, const void* q, const void* k, const int32_t* cu,
-                              const kvpop_shape& sh, float scale, bool target_pass) {
+                              const kvpop_shape& sh, float scale, bool target_pass,
+                              std::vector<int>* order = nullptr) {
   memset(p, 0, sizeof(*p));
   const int64_t T = sh.total_tokens;
   kvpop_status st;
@@ -210,9 +217,23 @@ kvpop_status fill_attn_common(AttnParams* p, const void* q, const void* k, const
   p->group = sh.n_q_heads / sh.n_kv_heads;
   p->scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p->inv_scale = static_cast<float>(1.0 / static_cast<double>(scale));
-  build_schedule(cu, sh.batch, target_pass ? sh.n_kv_heads : sh.n_q_heads, &p->sched);
+  build_schedule(cu, sh.batch, target_pass ? sh.n_kv_heads : sh.n_q_heads, &p->sched, order);
   return KVPOP_OK;
 }
+
+// 128-row tiles of every sequence (the lse readiness flags of the single
+// launch are one per query head and tile), -1 for a malformed cu_seqlens.
+int64_t flag_tiles(const int32_t* cu, int batch) {
+  int64_t t = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int64_t L = static_cast<int64_t>(cu[b + 1]) - cu[b];
+    if (L < 0) return -1;
+    t += (L + kTileRows - 1) / kTileRows;
+  }
+  return t;
+}
+
+static_assert(sizeof(FusedParams) <= 32764, "kernel parameter space");
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -499,6 +520,74 @@ kvpop_status kvpop_future_targets(const void* q, const void* k, const int32_t* c
   if ((st = kvpop_future_target(q, k, cu_seqlens, shape, scale, window, lse, target, dev_status, stream)) !=
       KVPOP_OK)
     return st;
+  return kvpop_keep_mask(target, cu_seqlens, shape, window, sinks, budgets, keep, stream);
+}
+
+size_t kvpop_fused_workspace_bytes(const int32_t* cu_seqlens, kvpop_shape shape) {
+  if (cu_seqlens == nullptr || shape.batch < 1 || shape.batch > kMaxSeqs || shape.n_q_heads < 1) return 0;
+  const int64_t tiles = flag_tiles(cu_seqlens, shape.batch);
+  if (tiles < 0) return 0;
+  return align256(static_cast<size_t>(shape.n_q_heads * tiles + 2) * sizeof(int32_t));
+}
+
+kvpop_status kvpop_future_targets_fused(const void* q, const void* k, const int32_t* cu_seqlens, kvpop_shape shape,
+                                        float scale, int32_t window, int32_t sinks, const int32_t* budgets,
+                                        float* lse, float* target, uint8_t* keep, void* workspace,
+                                        size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  kvpop_status st;
+  if ((st = check_qk(q, k, scale)) != KVPOP_OK) return st;
+  if (lse == nullptr || target == nullptr || keep == nullptr || budgets == nullptr)
+    return fail(KVPOP_ERR_INVALID_ARG, "lse, target, keep or budgets is NULL");
+  if (window < 0 || sinks < 0) return fail(KVPOP_ERR_INVALID_ARG, "window and sinks must be >= 0");
+  if ((st = check_shape(cu_seqlens, shape, true)) != KVPOP_OK) return st;
+  for (int b = 0; b < shape.batch; ++b)
+    if (static_cast<int64_t>(budgets[b]) < static_cast<int64_t>(sinks) + window)
+      return fail(KVPOP_ERR_INVALID_ARG, "budget[%d] = %d is below sinks + window", b, budgets[b]);
+  const size_t need = kvpop_fused_workspace_bytes(cu_seqlens, shape);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(KVPOP_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu required", workspace_bytes,
+                need);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 3u) != 0)
+    return fail(KVPOP_ERR_INVALID_ARG, "workspace must be 4-byte aligned");
+  if (static_cast<int64_t>(shape.n_q_heads) * flag_tiles(cu_seqlens, shape.batch) >= (int64_t(1) << 31))
+    return fail(KVPOP_ERR_UNSUPPORTED, "too many (query head, tile) flags for one launch");
+  if (shape.total_tokens == 0) return KVPOP_OK;
+  DeviceInfo dev;
+  if ((st = device_info(&dev)) != KVPOP_OK) return st;
+
+  std::vector<FusedParams> holder(1);   // ~21 KB: keep it off the stack
+  FusedParams& fp = holder[0];
+  memset(&fp, 0, sizeof(fp));
+  std::vector<int> order_lse, order_tgt;
+  if ((st = fill_attn_common(&fp.attn, q, k, cu_seqlens, shape, scale, false, &order_lse)) != KVPOP_OK) return st;
+  {
+    std::vector<AttnParams> tgt(1);
+    if ((st = fill_attn_common(&tgt[0], q, k, cu_seqlens, shape, scale, true, &order_tgt)) != KVPOP_OK) return st;
+    fp.tmap_q_stream = tgt[0].tmap_q;
+    fp.tmap_k_tile = tgt[0].tmap_k;
+    fp.sched_target = tgt[0].sched;
+  }
+  fp.attn.window = std::min<int32_t>(window, kMaxLevels * kTileRows + 1);
+  fp.attn.out = lse;
+  fp.attn.lse_in = lse;
+  fp.attn.status = dev_status;
+  fp.target = target;
+  std::vector<int32_t> base(shape.batch + 1, 0);
+  for (int b = 0; b < shape.batch; ++b)
+    base[b + 1] = base[b] + (cu_seqlens[b + 1] - cu_seqlens[b] + kTileRows - 1) / kTileRows;
+  fp.n_flag_tiles = base[shape.batch];
+  fp.n_flags = shape.n_q_heads * fp.n_flag_tiles;
+  fp.flags = static_cast<int32_t*>(workspace);
+  fp.done = fp.flags + fp.n_flags;
+  fp.lse_done = fp.done + 1;
+  for (size_t r = 0; r < order_lse.size(); ++r) fp.tile_base_lse[r] = base[order_lse[r]];
+  for (size_t r = 0; r < order_tgt.size(); ++r) fp.tile_base_target[r] = base[order_tgt[r]];
+  if (fp.attn.sched.total_items > 0) {
+    const int items = std::max(fp.attn.sched.total_items, fp.sched_target.total_items);
+    cudaError_t e = launch_fused_targets(fp, shape.head_dim, grid_for(items, dev.sm_count),
+                                         static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "fused attention launch");
+  }
   return kvpop_keep_mask(target, cu_seqlens, shape, window, sinks, budgets, keep, stream);
 }
 

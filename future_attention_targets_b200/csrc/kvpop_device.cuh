@@ -80,6 +80,7 @@ enum WaitSite : int32_t {
   SITE_SOFTMAX_ACC_FULL = 6,
   SITE_TEARDOWN = 7,
   SITE_SELFTEST = 8,
+  SITE_LSE_FLAG = 9,
 };
 
 struct WaitCtl {
@@ -97,6 +98,48 @@ __device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const 
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 15u) == 0u) {
+      if (*ctl.abort_flag) return false;
+      if (global_timer_ns() - t0 > ctl.limit_ns) {
+        *ctl.abort_flag = 1;
+        if (ctl.status != nullptr) atomicCAS(ctl.status, 0, 4 | (site << 8));
+        return false;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ cross-CTA flags
+
+// Adds v to a counter in global memory with gpu-scope release semantics: the
+// calling thread's earlier writes (and those ordered before it by a barrier)
+// are visible to any thread that later acquires the new value.
+__device__ __forceinline__ void flag_release_add(int32_t* f, int32_t v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int32_t flag_acquire_load(const int32_t* f) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+  return v;
+}
+
+// Returns the old value of *f and adds 1, acquire + release at gpu scope.
+__device__ __forceinline__ int32_t flag_arrive_count(int32_t* f) {
+  int32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(f) : "memory");
+  return old;
+}
+
+// One thread waits until *f >= want.  Gives up like wait_bounded: when the
+// CTA is aborting, or after ctl.limit_ns (then it raises the abort flag and
+// records a timeout at `site`).
+__device__ __noinline__ bool wait_flag_bounded(const int32_t* f, int32_t want, const WaitCtl& ctl, int32_t site) {
+  if (flag_acquire_load(f) >= want) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    if (flag_acquire_load(f) >= want) return true;
     if ((it & 15u) == 0u) {
       if (*ctl.abort_flag) return false;
       if (global_timer_ns() - t0 > ctl.limit_ns) {
@@ -252,6 +295,7 @@ struct WorkItem {
   int32_t seq_len;
   int32_t level;      // pass 1: query tile index; pass 2: key tiles remaining after this one
   int32_t head;       // pass 1: query head; pass 2: KV head
+  int32_t seq;        // position of the sequence in the schedule's sorted list
 };
 
 // Item n of the longest-first order: levels from the top down, then the
@@ -269,6 +313,7 @@ __device__ __forceinline__ WorkItem decode_item(const LevelSchedule& s, int32_t 
   w.seq_len = s.seq_len[r];
   w.level = s.n_levels - 1 - lo;
   w.head = off - r * s.n_heads;
+  w.seq = r;
   return w;
 }
 

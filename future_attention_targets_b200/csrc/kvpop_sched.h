@@ -46,6 +46,27 @@ struct AttnParams {
   LevelSchedule sched;
 };
 
+// Both attention passes in one launch.  attn holds pass 1 (its tensor maps,
+// schedule and lse output, which is also attn.lse_in); pass 2 has its own
+// maps (A = 128 key rows, B = 256 query rows) and schedule.  flags counts,
+// per (query head, 128-row tile of a sequence), the pass-1 warps that have
+// written that tile's lse; it, done and lse_done are zero on entry and zero
+// again when the launch completes.
+struct FusedParams {
+  AttnParams attn;
+  CUtensorMap tmap_q_stream;   // pass 2 B operand: Q, box {64, 256}
+  CUtensorMap tmap_k_tile;     // pass 2 A operand: K, box {64, 128}
+  LevelSchedule sched_target;
+  float* target;               // [H_kv, T]
+  int32_t* flags;              // [H_q, n_flag_tiles]
+  int32_t* done;               // CTAs that have finished
+  int32_t* lse_done;           // softmax warps that have finished pass 1
+  int32_t n_flag_tiles;        // sum over sequences of ceil(L / 128)
+  int32_t n_flags;             // H_q * n_flag_tiles
+  int32_t tile_base_lse[kMaxSeqs];     // first flag tile of each sequence, in pass-1 schedule order
+  int32_t tile_base_target[kMaxSeqs];  // the same in pass-2 schedule order
+};
+
 struct KeepParams {
   const float* score;     // [H_kv, T]
   uint8_t* keep;          // [H_kv, T]

@@ -18,7 +18,7 @@ namespace kvpop {
 // ------------------------------------------------------------------ compaction
 
 constexpr int kCompactThreads = 256;
-constexpr int kCompactUnroll = 8;      // 16-byte words each thread has in flight
+constexpr int kCompactUnroll = 16;     // 16-byte words each thread has in flight
 
 // Non-zero bytes of a 32-bit word: bit 7 of ((b & 0x7f) + 0x7f) | b is set
 // exactly when the byte b is non-zero, and the sum cannot carry into the next byte.
@@ -105,7 +105,7 @@ __device__ __forceinline__ int block_exclusive_scan_256(int x, int* warp_sums, i
 // by output slots gives every CTA the same number of rows to move wherever
 // the kept positions cluster.
 template <int d>
-__global__ void __launch_bounds__(kCompactThreads) compact_kv_kernel(const __grid_constant__ CompactParams p) {
+__global__ void __launch_bounds__(kCompactThreads, 2) compact_kv_kernel(const __grid_constant__ CompactParams p) {
   constexpr int kWords = d / 8;              // 16-byte words per row
   constexpr int kRowWords = 2 * kWords;      // K row then V row
   __shared__ int warp_sums[kCompactThreads / 32];
@@ -138,23 +138,27 @@ __global__ void __launch_bounds__(kCompactThreads) compact_kv_kernel(const __gri
   const int total_words = n_fill * kRowWords;
   for (int base = tid; base < total_words; base += kCompactThreads * kCompactUnroll) {
     uint4 buf[kCompactUnroll];
-    uint16_t* dst[kCompactUnroll];
 #pragma unroll
     for (int u = 0; u < kCompactUnroll; ++u) {
       const int idx = base + u * kCompactThreads;
-      dst[u] = nullptr;
       if (idx < total_words) {
         const int e = idx / kRowWords, rem = idx - e * kRowWords;
         const bool is_v = rem >= kWords;
         const int w = is_v ? rem - kWords : rem;
         const int64_t src = (static_cast<int64_t>(s0 + list_pos[e]) * p.n_kv_heads + h) * d + w * 8;
         buf[u] = __ldg(reinterpret_cast<const uint4*>((is_v ? p.v : p.k) + src));
-        dst[u] = (is_v ? p.v_cache : p.k_cache) + (row0 + S0 + e) * d + w * 8;
       }
     }
 #pragma unroll
-    for (int u = 0; u < kCompactUnroll; ++u)
-      if (dst[u] != nullptr) *reinterpret_cast<uint4*>(dst[u]) = buf[u];
+    for (int u = 0; u < kCompactUnroll; ++u) {
+      const int idx = base + u * kCompactThreads;
+      if (idx < total_words) {
+        const int e = idx / kRowWords, rem = idx - e * kRowWords;
+        const bool is_v = rem >= kWords;
+        const int w = is_v ? rem - kWords : rem;
+        *reinterpret_cast<uint4*>((is_v ? p.v_cache : p.k_cache) + (row0 + S0 + e) * d + w * 8) = buf[u];
+      }
+    }
   }
   // Slot positions (-1 when unused) and zeros in the unused rows.
   for (int e = tid; e < S1 - S0; e += kCompactThreads) p.pos[row0 + S0 + e] = (e < n_fill) ? list_pos[e] : -1;
@@ -202,12 +206,12 @@ __device__ __forceinline__ void dec_unpack(uint64_t v, float& a, float& b) {
 }
 __device__ __forceinline__ uint64_t dec_fma2(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
   return r;
 }
 __device__ __forceinline__ uint64_t dec_mul2(uint64_t a, uint64_t b) {
   uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  asm("mul.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
 // Two bf16 in one 32-bit word -> the packed pair (low half first).

@@ -227,6 +227,29 @@ KVPOP_API kvpop_status kvpop_future_targets(const void* q, const void* k, const 
                                   const int32_t* budgets, float* lse, float* target,
                                   uint8_t* keep, int32_t* dev_status, void* stream);
 
+/* Device workspace (bytes) of kvpop_future_targets_fused: one int32 readiness
+ * counter per (query head, 128-row tile of each sequence) plus two. */
+KVPOP_API size_t kvpop_fused_workspace_bytes(const int32_t* cu_seqlens, kvpop_shape shape);
+
+/* The same three results as kvpop_future_targets with both attention passes
+ * in ONE cooperative launch (then the keep-mask launch).  Each CTA runs its
+ * share of the row-logsumexp pass and then of the transposed pass; before
+ * the transposed pass reads a query tile's lse it waits (at most 1 s, then a
+ * KVPOP_ERR_TIMEOUT code in *dev_status) for the CTAs that write it, through
+ * counters in `workspace`.  lse, target and keep are bit-identical to those
+ * of kvpop_future_targets.
+ *   workspace  device, >= kvpop_fused_workspace_bytes(cu_seqlens, shape) bytes,
+ *              4-byte aligned, ZERO-FILLED before the first call; a launch
+ *              that completes leaves it zero-filled again (after a timeout
+ *              or a failed launch, zero it again before reuse).  Calls that
+ *              share one workspace must not overlap on the GPU.
+ * Other arguments as for kvpop_future_targets. */
+KVPOP_API kvpop_status kvpop_future_targets_fused(const void* q, const void* k, const int32_t* cu_seqlens,
+                                                  kvpop_shape shape, float scale, int32_t window, int32_t sinks,
+                                                  const int32_t* budgets, float* lse, float* target,
+                                                  uint8_t* keep, void* workspace, size_t workspace_bytes,
+                                                  int32_t* dev_status, void* stream);
+
 /* Device workspace (bytes) that kvpop_future_targets_host needs for `shape`. */
 KVPOP_API size_t kvpop_host_workspace_bytes(kvpop_shape shape);
 

@@ -17,7 +17,7 @@ def lib():
 
 def test_exports_every_header_symbol(lib):
     names = B.header_symbols()
-    assert len(names) == 16, names
+    assert len(names) == 18, names
     for name in names:
         assert hasattr(lib, name), f"{name} declared in kvpop.h but not exported"
     assert set(names) == set(B._SIGS), "binding signatures and header disagree"
@@ -142,6 +142,13 @@ def test_pipeline_rejects(lib):
                                          None) == B.INVALID_ARG
     assert lib.kvpop_future_targets_host(FAKE, FAKE, cu, sh, 0.1, 16, 4, bud, FAKE, FAKE, FAKE + 16, need, None,
                                          None) == B.INVALID_ARG
+    F = lib.kvpop_future_targets_fused
+    fneed = lib.kvpop_fused_workspace_bytes(cu, sh)
+    assert F(FAKE, FAKE, cu, sh, 0.1, 16, 4, bud, FAKE, FAKE, FAKE, None, fneed, None, None) == B.INVALID_ARG
+    assert F(FAKE, FAKE, cu, sh, 0.1, 16, 4, bud, FAKE, FAKE, FAKE, FAKE, fneed - 1, None, None) == B.INVALID_ARG
+    assert F(FAKE, FAKE, cu, sh, 0.1, 16, 4, bud, FAKE, FAKE, FAKE, FAKE + 2, fneed, None, None) == B.INVALID_ARG
+    assert F(FAKE, FAKE, cu, sh, 0.1, 16, 4, _cu(10), FAKE, FAKE, FAKE, FAKE, fneed, None, None) == B.INVALID_ARG
+    assert F(FAKE, FAKE, cu, sh, 0.1, 16, 4, bud, None, FAKE, FAKE, FAKE, fneed, None, None) == B.INVALID_ARG
     assert lib.kvpop_check_device_status(None, None) == B.INVALID_ARG
     assert lib.kvpop_selftest_bounded_wait(FAKE, 0, None) == B.INVALID_ARG
     assert lib.kvpop_selftest_bounded_wait(None, 1000, None) == B.INVALID_ARG
@@ -154,6 +161,16 @@ def test_workspace_bytes(lib):
     want = r(T * 32 * 128 * 2) + r(T * 8 * 128 * 2) + r(T * 32 * 4) + r(T * 8 * 4) + r(T * 8)
     assert lib.kvpop_host_workspace_bytes(sh) == want
     assert lib.kvpop_host_workspace_bytes(B.Shape(1, 0, 32, 8, 128)) == 0
+
+
+def test_fused_workspace_bytes(lib):
+    # one int32 per (query head, 128-row tile of each sequence), plus two completion counters
+    r = lambda x: (x + 255) // 256 * 256
+    assert lib.kvpop_fused_workspace_bytes(_cu(0, 16384), B.Shape(1, 16384, 32, 8, 128)) == r((32 * 128 + 2) * 4)
+    assert lib.kvpop_fused_workspace_bytes(_cu(0, 1, 129, 129, 300), B.Shape(4, 300, 4, 2, 64)) == \
+        r((4 * (1 + 1 + 0 + 2) + 2) * 4)
+    assert lib.kvpop_fused_workspace_bytes(None, B.Shape(1, 10, 4, 2, 64)) == 0
+    assert lib.kvpop_fused_workspace_bytes(_cu(0, 10), B.Shape(1, 10, 0, 2, 64)) == 0
 
 
 def test_empty_input_is_a_no_op(lib):

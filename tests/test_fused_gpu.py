@@ -1,0 +1,82 @@
+"""Single-launch variant (kvpop_future_targets_fused) through the C ABI.
+
+Every work item runs the same arithmetic in the same order as in the
+two-launch path, so lse, target and keep must be bit-identical to
+future_targets; the small cases are also checked against the oracle
+directly.  The flag workspace must come back zero-filled after each call so
+that it can be reused.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from future_attention_targets_b200 import (check_status, fused_workspace, future_targets, future_targets_fused)
+from future_attention_targets_b200.workloads import make_inputs, random_qk
+
+pytestmark = pytest.mark.gpu
+TARGET_TOL = 2e-3
+
+
+def dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def rel_err(gpu, ref):
+    gpu, ref = np.asarray(gpu, np.float64), np.asarray(ref, np.float64)
+    return float(np.max(np.abs(gpu - ref) / np.maximum(np.abs(ref), 1e-3))) if gpu.size else 0.0
+
+
+def run_both(q_bits, k_bits, cu, W, S, budgets, scale, calls=2):
+    q, k = dev(q_bits), dev(k_bits)
+    hq, hkv, d = q.shape[1], k.shape[1], q.shape[2]
+    st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ref = future_targets(q, k, cu, W, S, budgets, scale=scale, status=st2)
+    ws = fused_workspace(cu, hq, hkv, d)
+    st1 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    outs = [future_targets_fused(q, k, cu, W, S, budgets, scale=scale, workspace=ws, status=st1)
+            for _ in range(calls)]
+    torch.cuda.synchronize()
+    check_status(st1)
+    check_status(st2)
+    assert int(torch.count_nonzero(ws)) == 0, "flag workspace not cleared by the launch"
+    for out in outs:
+        for a, b in zip(out, ref):
+            assert torch.equal(a, b)
+    return outs[-1]
+
+
+@pytest.mark.parametrize("name", ["tiny", "qwen3_4b_4k", "varlen_8x"])
+def test_fused_matches_two_launch_path(name):
+    d = make_inputs(name)
+    run_both(d["q_bits"], d["k_bits"], d["cu_seqlens"], d["window"], d["sinks"], d["budgets"], d["scale"])
+
+
+@pytest.mark.parametrize("seqlens,hq,hkv,d,W", [
+    ((300,), 4, 2, 64, 16),                  # head_dim 64
+    ((1, 0, 129, 257, 700), 8, 2, 128, 5),   # empty and one-token sequences, ragged tiles
+    ((400, 90), 2, 1, 128, 1000),            # window beyond every sequence: targets all zero
+    ((2048,), 16, 1, 64, 0),                 # no window, group of 16
+])
+def test_fused_edge_shapes_against_oracle(seqlens, hq, hkv, d, W):
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    T = int(cu[-1])
+    q_bits, k_bits = random_qk(T, hq, hkv, d, seed=T + hq)
+    scale = 1.0 / math.sqrt(d)
+    S = 2
+    budgets = [max(S + W, L // 2) for L in seqlens]
+    lse, tgt, keep = run_both(q_bits, k_bits, cu, W, S, budgets, scale)
+    ref_t = oracle.future_target(q_bits, k_bits, cu, W, scale)
+    ref_lse = oracle.row_lse(q_bits, k_bits, cu, scale)
+    assert rel_err(tgt.cpu().numpy(), ref_t) <= TARGET_TOL
+    assert np.max(np.abs(lse.cpu().numpy() - ref_lse)) <= 1e-4
+    assert np.array_equal(keep.cpu().numpy(), oracle.keep_mask(tgt.cpu().numpy(), cu, W, S, budgets))
+
+
+def test_fused_full_size_16k():
+    d = make_inputs("qwen3_8b_16k")
+    lse, tgt, keep = run_both(d["q_bits"], d["k_bits"], d["cu_seqlens"], d["window"], d["sinks"], d["budgets"],
+                              d["scale"], calls=3)
+    assert int(keep.sum()) == 8 * 4032
