@@ -397,7 +397,8 @@ def run_ours(args):
             "ms": ms, "steps_per_s": steps_total / (ms * 1e-3),
             "bound": "latency", "hbm_gbs": moved / (ms * 1e-3) / 1e9,
             "frac_of_hbm": moved / (ms * 1e-3) / 1e9 / float(peaks_x["hbm_gbs"]),
-            "launch": f"{len(cu) - 1} x {w.n_kv_heads} CTAs of 1024 threads, one per (sequence, KV head)"}
+            "launch": (f"{len(cu) - 1} x {w.n_kv_heads} x {-(-(int(max(np.diff(cu))) - S - W) // 1024)} CTAs of 1024 "
+                       "threads, one per (sequence, KV head, block of 1024 steps)")}
 
         # Static cache: compact this step's keep set, then one decode step over it.
         from future_attention_targets_b200 import compact_kv, decode_attention

@@ -20,7 +20,7 @@ cudaError_t launch_row_lse(const AttnParams& p, int head_dim, int grid, cudaStre
 cudaError_t launch_future_target(const AttnParams& p, int head_dim, int grid, cudaStream_t stream);
 cudaError_t launch_keep_mask(const KeepParams& p, int n_kv_heads, cudaStream_t stream);
 cudaError_t launch_selftest_wait(int32_t* status, uint64_t limit_ns, cudaStream_t stream);
-cudaError_t launch_prefix_thresholds(const ThresholdParams& p, int n_kv_heads, cudaStream_t stream);
+cudaError_t launch_prefix_thresholds(const ThresholdParams& p, int n_kv_heads, int max_len, cudaStream_t stream);
 cudaError_t launch_compact_kv(const CompactParams& p, cudaStream_t stream);
 cudaError_t launch_decode_attention(const DecodeParams& p, int batch, cudaStream_t stream);
 cudaError_t launch_fused_targets(const FusedParams& fp, int head_dim, int grid, cudaStream_t stream);
@@ -346,9 +346,6 @@ kvpop_status kvpop_prefix_topk_thresholds(const float* score, const int32_t* cu_
     if (k < 0)
       return fail(KVPOP_ERR_INVALID_ARG, "budget[%d] = %d is below sinks + window = %lld", b, budgets[b],
                   static_cast<long long>(sinks) + window);
-    if (k > kMaxScored)
-      return fail(KVPOP_ERR_UNSUPPORTED, "budget[%d] leaves %lld scored slots (limit %d)", b,
-                  static_cast<long long>(k), kMaxScored);
   }
   if (shape.total_tokens == 0) return KVPOP_OK;
   DeviceInfo dev;
@@ -362,12 +359,14 @@ kvpop_status kvpop_prefix_topk_thresholds(const float* score, const int32_t* cu_
   p.window = window;
   p.sinks = sinks;
   p.n_seqs = shape.batch;
+  int max_len = 0;
   for (int b = 0; b < shape.batch; ++b) {
     p.seq_start[b] = cu_seqlens[b];
     p.seq_len[b] = cu_seqlens[b + 1] - cu_seqlens[b];
     p.budget[b] = budgets[b];
+    max_len = std::max(max_len, p.seq_len[b]);
   }
-  cudaError_t e = launch_prefix_thresholds(p, shape.n_kv_heads, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_prefix_thresholds(p, shape.n_kv_heads, max_len, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "prefix thresholds launch");
 }
 

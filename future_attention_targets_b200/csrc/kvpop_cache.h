@@ -8,8 +8,6 @@
 
 namespace kvpop {
 
-constexpr int kMaxScored = 8192;   // largest scored-slot count k for the prefix thresholds
-
 struct ThresholdParams {
   const float* score;     // [H_kv, T]
   float* thr_score;       // [H_kv, T]

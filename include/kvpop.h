@@ -132,8 +132,7 @@ KVPOP_API kvpop_status kvpop_keep_mask(const float* score, const int32_t* cu_seq
  * the scored slots overflow, and at the last step it selects the same tokens
  * as kvpop_keep_mask.
  *   score      device fp32 [n_kv_heads, T]
- *   budgets    HOST int32 [batch], each >= sinks + window, and
- *              budget - sinks - window <= 8192 (else KVPOP_ERR_UNSUPPORTED)
+ *   budgets    HOST int32 [batch], each >= sinks + window
  *   thr_score  device fp32 [n_kv_heads, T]: the threshold token's score
  *              (-0 reported as +0); -inf while fewer than k tokens compete
  *              (nothing evicted yet); +inf when k = 0 (nothing kept)

@@ -102,7 +102,6 @@ def test_thresholds_reject(lib):
     assert T(FAKE, cu, sh, 16, 4, bud, FAKE, None, None) == B.INVALID_ARG
     assert T(FAKE, cu, sh, 16, 4, None, FAKE, FAKE, None) == B.INVALID_ARG
     assert T(FAKE, cu, sh, 16, 4, _cu(19), FAKE, FAKE, None) == B.INVALID_ARG        # below sinks + window
-    assert T(FAKE, cu, sh, 16, 4, _cu(20 + 8193), FAKE, FAKE, None) == B.UNSUPPORTED  # too many scored slots
     assert T(FAKE, _cu(0, 0), B.Shape(1, 0, 4, 2, 128), 16, 4, bud, FAKE, FAKE, None) == B.OK
 
 

@@ -29,6 +29,9 @@ CASES = [
     ((2500,), 2, 8, 2, [2000], "ties"),           # k larger than a block
     ((9000,), 1, 4, 4, [8192], "uniform"),        # the largest k
     ((1500, 1, 2100), 2, 64, 0, [300, 5, 1], "special"),
+    ((20000,), 1, 16, 4, [10000], "uniform"),     # k beyond 8192: the band is taken from a large K
+    ((6000, 3000), 2, 8, 4, [1500, 2900], "coarse"),   # four distinct scores: ties across the band edges
+    ((5000,), 1, 8, 4, [1024], "coarse"),         # band of exactly kBlock + 1 with k near a block
 ]
 
 
@@ -37,6 +40,8 @@ def make_scores(kind, H, T, seed):
     s = rng.random((H, T)).astype(np.float32)
     if kind == "ties":
         s = np.round(s * 16) / 16
+    if kind == "coarse":
+        s = np.floor(s * 4) / 4
     if kind == "special":
         s[:, ::11] = 0.5
         s[0, 5::97] = np.nan
