@@ -17,12 +17,14 @@
 // queries, so each thread owns one key and sums over all its queries and all
 // G heads without any cross-thread reduction.
 //
-// Warp roles (320 threads, one CTA per SM):
+// Warp roles (576 threads, one CTA per SM):
 //   warp 0      TMA producer: A tile once per item, B tiles into a 2-stage
 //               ring (pass 2: the warp also writes the normaliser slab)
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
-//   warps 2..9  softmax: two groups of four warps split the 256 accumulator
-//               columns (each warp reads its TMEM lane quadrant, warp % 4)
+//   warps 2..17 softmax: four groups of four warps split the 256 accumulator
+//               columns, 64 each (each warp reads its TMEM lane quadrant,
+//               warp % 4); four warps per scheduler hide the exponential
+//               chains' latency
 // Two TMEM accumulators of 256 fp32 columns (all 512 columns) let the MMA of
 // tile t+1 run while the softmax warps read tile t.
 //
@@ -44,7 +46,11 @@ namespace kvpop {
 
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kStages = 2;
-constexpr int kSoftmaxWarps = 8;
+constexpr int kColGroups = 4;                          // softmax warp groups per CTA
+constexpr int kGroupCols = kStreamRows / kColGroups;   // accumulator columns per group
+constexpr int kSoftmaxWarps = 4 * kColGroups;          // one warp per TMEM lane quadrant per group
+static_assert(kThreads == 32 * (2 + kSoftmaxWarps), "producer warp + MMA warp + softmax warps");
+static_assert(kGroupCols == 64, "group_exp_sum walks two 32-column chunks");
 // Extra K=16 slab (no swizzle, K-major): 8-row groups of two 8x16-byte core
 // matrices; element (r, e) sits at (r/8)*256 + (e/8)*128 + (r%8)*16 + (e%8)*2.
 constexpr int kSlabLBO = 128;   // between the two core matrices along K
@@ -63,8 +69,8 @@ struct SmemLayout {
   static constexpr int OFF_A = 0;                                // 2 buffers
   static constexpr int OFF_B = OFF_A + 2 * A_BYTES;              // kStages stages
   static constexpr int OFF_ASLAB = OFF_B + kStages * B_STAGE;
-  static constexpr int OFF_COMB = OFF_ASLAB + A_SLAB;            // float [2][128]
-  static constexpr int OFF_BAR = OFF_COMB + 2 * 128 * 4;
+  static constexpr int OFF_COMB = OFF_ASLAB + A_SLAB;            // float [kColGroups - 1][2][128]
+  static constexpr int OFF_BAR = OFF_COMB + (kColGroups - 1) * 2 * 128 * 4;
   // a_full[2] a_empty[2] b_full[S] b_empty[S] acc_full[2] acc_empty[2] comb_full comb_empty mma_done
   static constexpr int N_BARS = 4 + 2 * kStages + 4 + 3;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
@@ -614,10 +620,10 @@ __device__ __forceinline__ uint64_t exp2_mufu_pair(uint64_t y) {
 // evaluated by the polynomial, spread evenly over the chunk (measured on
 // B200 for each pass at the Qwen3-8B 16k shape).
 #ifndef KVPOP_POLY16_LSE
-#define KVPOP_POLY16_LSE 4
+#define KVPOP_POLY16_LSE 3
 #endif
 #ifndef KVPOP_POLY16_TARGET
-#define KVPOP_POLY16_TARGET 4
+#define KVPOP_POLY16_TARGET 3
 #endif
 
 template <int kPoly>
@@ -668,12 +674,12 @@ __device__ __forceinline__ float acc_total(uint64_t (&acc)[4]) {
   return a + b;
 }
 
-// Sum of exp2(x * c - off) over the 128 columns of this thread's TMEM lane
-// starting at taddr: four chunks of 32, the load of chunk c+1 in flight
-// while chunk c is summed.  kMasked: column m counts iff lo <= m < hi.
+// Sum of exp2(x * c - off) over the kGroupCols = 64 columns of this thread's
+// TMEM lane starting at taddr: two chunks of 32, the second load in flight
+// while the first chunk is summed.  kMasked: column m counts iff lo <= m < hi.
 template <bool kMasked, int kPoly, bool kBiasFree = false>
-__device__ __forceinline__ float half_tile_exp_sum(uint32_t taddr, uint64_t c2, uint64_t nb, int lo, int hi,
-                                                   float xmin = 0.f) {
+__device__ __forceinline__ float group_exp_sum(uint32_t taddr, uint64_t c2, uint64_t nb, int lo, int hi,
+                                               float xmin = 0.f) {
   uint32_t ra[32], rb[32];
   uint64_t acc[4] = {0, 0, 0, 0};
   auto run = [&](const uint32_t (&r)[32], int ch) {
@@ -687,21 +693,15 @@ __device__ __forceinline__ float half_tile_exp_sum(uint32_t taddr, uint64_t c2, 
   tmem_load<32>(taddr + 32, rb);
   run(ra, 0);
   tmem_load_wait<32>(rb);
-  tmem_load<32>(taddr + 64, ra);
   run(rb, 1);
-  tmem_load_wait<32>(ra);
-  tmem_load<32>(taddr + 96, rb);
-  run(ra, 2);
-  tmem_load_wait<32>(rb);
-  run(rb, 3);
   return acc_total(acc);
 }
 
-// Max of x * c over columns lo <= m < hi of the 128 (pass-1 rescale path).
-__device__ __forceinline__ float half_tile_max(uint32_t taddr, float c, int lo, int hi) {
+// Max of x * c over columns lo <= m < hi of the group's 64 (pass-1 rescale path).
+__device__ __forceinline__ float group_max(uint32_t taddr, float c, int lo, int hi) {
   float m = -INFINITY;
 #pragma unroll 1
-  for (int ch = 0; ch < 4; ++ch) {
+  for (int ch = 0; ch < kGroupCols / 32; ++ch) {
     uint32_t r[32];
     tmem_load<32>(taddr + 32 * ch, r);
     tmem_load_wait<32>(r);
@@ -721,11 +721,12 @@ __device__ void lse_softmax_phase(const AttnParams& p, const Phase& ph, uint8_t*
                                   const WaitCtl& ctl, uint32_t tmem_base, SoftmaxState& st) {
   using L = SmemLayout<HD, kFused>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int sw = warp - 2;                 // softmax warp 0..7
-  const int wg = sw >> 2;                  // column half
+  const int sw = warp - 2;                 // softmax warp 0 .. kSoftmaxWarps-1
+  const int wg = sw >> 2;                  // column group
+  const int c0 = wg * kGroupCols;          // its first accumulator column
   const int quad = warp & 3;               // TMEM lane quadrant this warp may access
   const int row = quad * 32 + lane;        // query row within the tile
-  const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + wg * 128;
+  const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + c0;
   float* comb = reinterpret_cast<float*>(smem + L::OFF_COMB);
   const float c = p.scale_log2;
   const uint64_t c2 = f2_pack(c, c);
@@ -745,32 +746,37 @@ __device__ void lse_softmax_phase(const AttnParams& p, const Phase& ph, uint8_t*
         break;
       }
       tc_fence_after_sync();
+      // The last key tile holds the diagonal 128-key block, at column 0 when
+      // the query tile starts on a 256-key boundary (then only columns 0..127
+      // were computed) and at column 128 otherwise; key column m of that
+      // block is unmasked iff m <= query row.
       const bool last = (t == it.ntiles - 1);
       const bool half = LsePass::half_tile(it, t);
-      const bool skip = half && wg == 1;                  // columns 128..255 not computed
-      const bool masked = last && (half ? wg == 0 : wg == 1);
-      const int hi = masked ? row + 1 : 128;              // on the diagonal: key column m <= query row
+      const bool skip = half && c0 >= kStreamRows / 2;
+      const int dcol = half ? 0 : kStreamRows / 2;
+      const bool masked = last && !skip && c0 >= dcol;
+      const int hi = masked ? min(kGroupCols, max(0, row - (c0 - dcol) + 1)) : kGroupCols;
       if (!skip) {
         const uint32_t taddr = lane_addr + acc * kStreamRows;
         float ts = 0.f;
         bool rescale = (off == -INFINITY);                 // first tile of the row: no offset yet
         if (!rescale) {
           const uint64_t nb = f2_pack(-off, -off);
-          ts = masked ? half_tile_exp_sum<true, 0>(taddr, c2, nb, 0, hi)
-                      : half_tile_exp_sum<false, KVPOP_POLY16_LSE>(taddr, c2, nb, 0, 128);
+          ts = masked ? group_exp_sum<true, 0>(taddr, c2, nb, 0, hi)
+                      : group_exp_sum<false, KVPOP_POLY16_LSE>(taddr, c2, nb, 0, kGroupCols);
           rescale = !(ts < kBig);
         }
         // Warp-uniform: the rescale path issues warp-collective TMEM loads.
         if (__any_sync(0xffffffffu, rescale)) {
-          const float tm = half_tile_max(taddr, c, 0, hi);
+          const float tm = group_max(taddr, c, 0, hi);
           const float noff = fmaxf(off, tm);
           if (noff > -INFINITY) {
             sum = (off > -INFINITY) ? sum * ex2_approx(off - noff) : 0.f;
             off = noff;
           }
           const uint64_t nb = f2_pack(-off, -off);
-          ts = masked ? half_tile_exp_sum<true, 0>(taddr, c2, nb, 0, hi)
-                      : half_tile_exp_sum<false, KVPOP_POLY16_LSE>(taddr, c2, nb, 0, 128);
+          ts = masked ? group_exp_sum<true, 0>(taddr, c2, nb, 0, hi)
+                      : group_exp_sum<false, KVPOP_POLY16_LSE>(taddr, c2, nb, 0, kGroupCols);
           if (!(off > -INFINITY)) ts = 0.f;
         }
         sum += ts;
@@ -786,14 +792,15 @@ __device__ void lse_softmax_phase(const AttnParams& p, const Phase& ph, uint8_t*
       ++st.acc_cnt;
     }
     if (!st.ok) break;
-    // Combine the two column halves of each row.
-    if (wg == 1) {
+    // Combine the column groups of each row: groups 1.. hand (offset, sum)
+    // to group 0 through shared memory.
+    if (wg != 0) {
       if (!warp_wait(bars.comb_empty, (st.item_cnt & 1u) ^ 1u, ctl, SITE_SOFTMAX_ACC_FULL)) {
         st.ok = false;
         break;
       }
-      comb[row] = off;
-      comb[128 + row] = sum;
+      comb[(2 * (wg - 1)) * 128 + row] = off;
+      comb[(2 * (wg - 1) + 1) * 128 + row] = sum;
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.comb_full);
     } else {
@@ -801,11 +808,22 @@ __device__ void lse_softmax_phase(const AttnParams& p, const Phase& ph, uint8_t*
         st.ok = false;
         break;
       }
-      const float off1 = comb[row], sum1 = comb[128 + row];
+      float offs[kColGroups], sums[kColGroups];
+      offs[0] = off;
+      sums[0] = sum;
+#pragma unroll
+      for (int g = 1; g < kColGroups; ++g) {
+        offs[g] = comb[(2 * (g - 1)) * 128 + row];
+        sums[g] = comb[(2 * (g - 1) + 1) * 128 + row];
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.comb_empty);
-      const float m = fmaxf(off, off1);
-      const float s = sum * ex2_approx(off - m) + (off1 > -INFINITY ? sum1 * ex2_approx(off1 - m) : 0.f);
+      float m = offs[0];
+#pragma unroll
+      for (int g = 1; g < kColGroups; ++g) m = fmaxf(m, offs[g]);
+      float s = 0.f;
+#pragma unroll
+      for (int g = 0; g < kColGroups; ++g) s += (offs[g] > -INFINITY) ? sums[g] * ex2_approx(offs[g] - m) : 0.f;
       const int32_t i = it.i0 + row;
       if (i < it.L) ph.out[static_cast<int64_t>(it.g) * p.total_tokens + it.s + i] = (m + log2f(s)) * kLn2;
       if constexpr (kFused) {
@@ -830,10 +848,11 @@ __device__ void target_softmax_phase(const AttnParams& p, const Phase& ph, uint8
   using L = SmemLayout<HD, true>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sw = warp - 2;
-  const int wg = sw >> 2;
+  const int wg = sw >> 2;                  // column group
+  const int c0 = wg * kGroupCols;          // its first accumulator column
   const int quad = warp & 3;
   const int row = quad * 32 + lane;        // key row within the tile
-  const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + wg * 128;
+  const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + c0;
   float* comb = reinterpret_cast<float*>(smem + L::OFF_COMB);
   const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
   const uint64_t zero2 = f2_pack(0.f, 0.f);
@@ -855,14 +874,18 @@ __device__ void target_softmax_phase(const AttnParams& p, const Phase& ph, uint8
         }
         tc_fence_after_sync();
         const uint32_t taddr = lane_addr + acc * kStreamRows;
-        // First query tile: column m of the first half is valid iff m >= row.
-        // Last query tile: columns past the sequence hold -1e30 (exp2 -> 0 on MUFU).
-        const bool diag = (qt == 0) && (wg == 0);
+        // First query tile: query column m is valid iff m >= row, which can
+        // mask columns of the groups below column 128 (per-lane bound lo).
+        // Last query tile: columns past the sequence hold -1e30 (exp2 -> 0 on
+        // MUFU).  The path is chosen per warp: its TMEM loads are
+        // warp-collective.
+        const bool diag = (qt == 0) && (c0 < kTileRows);
         const bool ragged = (qt == it.nq - 1) && ragged_end;
+        const int lo = diag ? max(0, row - c0) : 0;
         const float ts = (diag || ragged)
-                             ? half_tile_exp_sum<true, 0>(taddr, c2, zero2, diag ? row : 0, 128)
-                             : half_tile_exp_sum<false, KVPOP_POLY16_TARGET, true>(taddr, c2, zero2, 0, 128,
-                                                                                      xmin);
+                             ? group_exp_sum<true, 0>(taddr, c2, zero2, lo, kGroupCols)
+                             : group_exp_sum<false, KVPOP_POLY16_TARGET, true>(taddr, c2, zero2, 0, kGroupCols,
+                                                                                  xmin);
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.acc_empty[acc]);
@@ -874,12 +897,12 @@ __device__ void target_softmax_phase(const AttnParams& p, const Phase& ph, uint8
       }
     }
     if (!st.ok) break;
-    if (wg == 1) {
+    if (wg != 0) {
       if (!warp_wait(bars.comb_empty, (st.item_cnt & 1u) ^ 1u, ctl, SITE_SOFTMAX_ACC_FULL)) {
         st.ok = false;
         break;
       }
-      comb[row] = run;
+      comb[(wg - 1) * 128 + row] = run;
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.comb_full);
     } else {
@@ -887,11 +910,13 @@ __device__ void target_softmax_phase(const AttnParams& p, const Phase& ph, uint8
         st.ok = false;
         break;
       }
-      const float other = comb[row];
+      float total = run;
+#pragma unroll
+      for (int g = 1; g < kColGroups; ++g) total += comb[(g - 1) * 128 + row];
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.comb_empty);
       const int32_t j = it.j0 + row;
-      if (j < it.L) ph.out[static_cast<int64_t>(it.h) * p.total_tokens + it.s + j] = run + other;
+      if (j < it.L) ph.out[static_cast<int64_t>(it.h) * p.total_tokens + it.s + j] = total;
     }
     ++st.item_cnt;
   }
@@ -936,7 +961,7 @@ __device__ __forceinline__ void cta_setup(uint8_t* smem, const Bars& bars, uint3
       mbar_init(&bars.b_full[i], kSlab ? 32 : 1);
       mbar_init(&bars.b_empty[i], 1);
     }
-    mbar_init(bars.comb_full, 4);
+    mbar_init(bars.comb_full, 4 * (kColGroups - 1));
     mbar_init(bars.comb_empty, 4);
     mbar_init(bars.mma_done, 1);
     *abort_flag = 0;

@@ -10,7 +10,7 @@ constexpr int kMaxSeqs = 512;        // sequences per call
 constexpr int kTileRows = 128;       // rows of the resident (A) tile = MMA M
 constexpr int kMaxLevels = 1024;     // longest sequence = kMaxLevels * kTileRows tokens
 constexpr int kStreamRows = 256;     // rows of a streamed (B) tile = MMA N
-constexpr int kThreads = 320;        // producer warp + MMA warp + 8 softmax warps
+constexpr int kThreads = 576;        // producer warp + MMA warp + 16 softmax warps
 constexpr uint64_t kDefaultWaitNs = 1000000000ull;  // 1 s per on-chip wait
 
 // Work items ordered longest first.  An item is (level, sequence, head); all
