@@ -54,6 +54,9 @@ _SIGS = {
     "kvpop_decode_attention_noalloc": (ctypes.c_int, [_P, _P, _P, _P, CacheShape, ctypes.c_float, _P, _P, _P]),
     "kvpop_future_targets": (ctypes.c_int, [_P, _P, _I32P, Shape, ctypes.c_float, ctypes.c_int32, ctypes.c_int32,
                                             _I32P, _P, _P, _P, _P, _P]),
+    "kvpop_target_split_workspace_bytes": (ctypes.c_size_t, [Shape]),
+    "kvpop_future_target_split": (ctypes.c_int, [_P, _P, _I32P, Shape, ctypes.c_float, ctypes.c_int32, _P, _P, _P,
+                                                 ctypes.c_size_t, _P, _P]),
     "kvpop_fused_workspace_bytes": (ctypes.c_size_t, [_I32P, Shape]),
     "kvpop_future_targets_fused": (ctypes.c_int, [_P, _P, _I32P, Shape, ctypes.c_float, ctypes.c_int32,
                                                   ctypes.c_int32, _I32P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
@@ -176,6 +179,31 @@ def future_target(q, k, cu_seqlens, window: int, lse, scale: float | None = None
     _check(lib().kvpop_future_target(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, int(window),
                                      lse.contiguous().data_ptr(), out.data_ptr(), _ptr(status), _stream_ptr(stream)))
     return out
+
+
+def future_target_split(q, k, cu_seqlens, window: int, lse, scale: float | None = None, out=None, workspace=None,
+                        status=None, stream=None):
+    """future_target with one item per (key tile, query head); bit-identical result, for few KV heads per call."""
+    import torch
+    _check_qk(q, k)
+    cu, cu_c = _cu_host(cu_seqlens)
+    sh = _shape(q, k, cu)
+    scale = 1.0 / math.sqrt(sh.head_dim) if scale is None else float(scale)
+    if lse.dtype != torch.float32 or not lse.is_cuda or tuple(lse.shape) != (sh.n_q_heads, sh.total_tokens):
+        raise ValueError("lse must be a fp32 CUDA tensor [H_q, T]")
+    if out is None:
+        out = torch.empty((sh.n_kv_heads, sh.total_tokens), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(int(lib().kvpop_target_split_workspace_bytes(sh)), 16), dtype=torch.uint8,
+                                device=q.device)
+    _check(lib().kvpop_future_target_split(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, int(window),
+                                           lse.contiguous().data_ptr(), out.data_ptr(), workspace.data_ptr(),
+                                           workspace.numel(), _ptr(status), _stream_ptr(stream)))
+    return out
+
+
+def target_split_workspace_bytes(total_tokens: int, n_q_heads: int, n_kv_heads: int, head_dim: int) -> int:
+    return int(lib().kvpop_target_split_workspace_bytes(Shape(1, total_tokens, n_q_heads, n_kv_heads, head_dim)))
 
 
 def keep_mask(score, cu_seqlens, window: int, sinks: int, budgets, out=None, stream=None):

@@ -38,6 +38,8 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include <algorithm>
+
 #include <type_traits>
 
 #include "kvpop_device.cuh"
@@ -183,23 +185,28 @@ struct LsePass {
   }
 };
 
-// Pass 2: item = (sequence, key tile, KV head); level = key tiles after this one.
+// Pass 2: item = (sequence, key tile, KV head) with all G query heads of
+// the group, or, when p.g_split = G, (sequence, key tile, KV head, one query
+// head) so that few KV heads still give enough items; level = key tiles
+// after this one.
 struct TargetPass {
   static constexpr bool kSlab = true;
   struct Item {
-    int32_t s, L, h, j0, i0, nq, ntiles, seq;
+    int32_t s, L, h, g0, ng, j0, i0, nq, ntiles, seq;
   };
   static __device__ __forceinline__ Item item(const AttnParams& p, const LevelSchedule& sched, int32_t n) {
     const WorkItem w = decode_item(sched, n);
     Item it;
     it.s = w.seq_start;
     it.L = w.seq_len;
-    it.h = w.head;
+    it.h = w.head / p.g_split;
+    it.ng = p.group / p.g_split;                 // query heads of this item
+    it.g0 = (w.head % p.g_split) * it.ng;        // the first of them, within the group
     const int32_t nkt = (w.seq_len + kTileRows - 1) / kTileRows;
     it.j0 = (nkt - 1 - w.level) * kTileRows;
     it.i0 = it.j0 + p.window;
     it.nq = it.i0 < it.L ? (it.L - it.i0 + kStreamRows - 1) / kStreamRows : 0;
-    it.ntiles = it.nq * p.group;
+    it.ntiles = it.nq * it.ng;
     it.seq = w.seq;
     return it;
   }
@@ -246,7 +253,7 @@ struct TileCursor {
   __device__ __forceinline__ void advance(const AttnParams& p, const LevelSchedule& sched) {
     if (++qt == it.nq) {
       qt = 0;
-      if (++g == p.group) next_item(p, sched);
+      if (++g == it.ng) next_item(p, sched);
     }
   }
 };
@@ -293,7 +300,7 @@ __device__ __forceinline__ bool norm_ready(const AttnParams& p, const Phase& ph,
     return true;
   } else {
     if (all_lse) return true;
-    const int32_t qh = cur.it.h * p.group + cur.g;
+    const int32_t qh = cur.it.h * p.group + cur.it.g0 + cur.g;
     const int32_t a = cur.it.i0 + cur.qt * kStreamRows;
     const int32_t b = min(a + kStreamRows, cur.it.L);
     const int32_t t0 = a / kTileRows, nt = (b - 1) / kTileRows - t0 + 1;
@@ -334,7 +341,7 @@ __device__ __forceinline__ bool norm_ready(const AttnParams& p, const Phase& ph,
 template <bool kFused>
 __device__ __forceinline__ void load_norm_rows(const AttnParams& p, const TileCursor& cur, int lane,
                                                float (&v)[8]) {
-  const int32_t qh = cur.it.h * p.group + cur.g;
+  const int32_t qh = cur.it.h * p.group + cur.it.g0 + cur.g;
   const float* src = p.lse_in + static_cast<int64_t>(qh) * p.total_tokens + cur.it.s;
 #pragma unroll
   for (int m = 0; m < 8; ++m) {
@@ -414,7 +421,7 @@ __device__ void producer_phase(const AttnParams& p, const Phase& ph, uint8_t* sm
         const int32_t g = t / it.nq, qt = t - g * it.nq;
         if (lane == 0) {
           mbar_expect_tx(&bars.b_full[sg], L::B_TILE);
-          Pass::template load_b<HD>(ph, it, it.h * p.group + g, qt, stage, &bars.b_full[sg]);
+          Pass::template load_b<HD>(ph, it, it.h * p.group + it.g0 + g, qt, stage, &bars.b_full[sg]);
         }
         float cur[8];
 #pragma unroll
@@ -863,9 +870,13 @@ __device__ void target_softmax_phase(const AttnParams& p, const Phase& ph, uint8
     const int32_t n = cta_item(k, blockIdx.x, gridDim.x);
     if (n >= total) break;
     const TargetPass::Item it = TargetPass::item(p, sched, n);
-    float run = 0.f, comp = 0.f;           // Kahan-compensated running sum over tiles
+    // Each query head's tiles are summed on their own (Kahan-compensated),
+    // then the heads are added in order: the same sums, in the same order,
+    // whether an item covers all G heads or one of them.
+    float heads = 0.f;
     const bool ragged_end = it.i0 + it.nq * kStreamRows > it.L;
-    for (int32_t g = 0; g < (it.nq > 0 ? p.group : 0) && st.ok; ++g) {
+    for (int32_t g = 0; g < (it.nq > 0 ? it.ng : 0) && st.ok; ++g) {
+      float run = 0.f, comp = 0.f;
       for (int32_t qt = 0; qt < it.nq; ++qt) {
         const uint32_t acc = st.acc_cnt & 1u;
         if (!warp_wait(&bars.acc_full[acc], (st.acc_cnt >> 1) & 1u, ctl, SITE_SOFTMAX_ACC_FULL)) {
@@ -895,14 +906,22 @@ __device__ void target_softmax_phase(const AttnParams& p, const Phase& ph, uint8
         comp = (tk - run) - yk;
         run = tk;
       }
+      heads += run;
     }
     if (!st.ok) break;
-    if (wg != 0) {
+    if (p.g_split > 1) {
+      // One query head per item: every column group writes its own partial
+      // [g, column group, h, T]; a merge kernel adds them in the order below.
+      const int32_t j = it.j0 + row;
+      if (j < it.L)
+        ph.out[(static_cast<int64_t>(it.g0 * kColGroups + wg) * p.n_kv_heads + it.h) * p.total_tokens + it.s + j] =
+            heads;
+    } else if (wg != 0) {
       if (!warp_wait(bars.comb_empty, (st.item_cnt & 1u) ^ 1u, ctl, SITE_SOFTMAX_ACC_FULL)) {
         st.ok = false;
         break;
       }
-      comb[(wg - 1) * 128 + row] = run;
+      comb[(wg - 1) * 128 + row] = heads;
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.comb_full);
     } else {
@@ -910,13 +929,13 @@ __device__ void target_softmax_phase(const AttnParams& p, const Phase& ph, uint8
         st.ok = false;
         break;
       }
-      float total = run;
+      float sum = heads;
 #pragma unroll
-      for (int g = 1; g < kColGroups; ++g) total += comb[(g - 1) * 128 + row];
+      for (int g = 1; g < kColGroups; ++g) sum += comb[(g - 1) * 128 + row];
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.comb_empty);
       const int32_t j = it.j0 + row;
-      if (j < it.L) ph.out[static_cast<int64_t>(it.h) * p.total_tokens + it.s + j] = total;
+      if (j < it.L) ph.out[static_cast<int64_t>(it.h) * p.total_tokens + it.s + j] = sum;
     }
     ++st.item_cnt;
   }
@@ -1134,6 +1153,36 @@ static cudaError_t launch_fused_hd(const FusedParams& fp, int grid, cudaStream_t
 cudaError_t launch_fused_targets(const FusedParams& fp, int head_dim, int grid, cudaStream_t stream) {
   return head_dim == 64 ? launch_fused_hd<64>(fp, grid, stream) : launch_fused_hd<128>(fp, grid, stream);
 }
+
+// Sum of the split pass's partials [G][kColGroups][H_kv][T] into the target
+// [H_kv][T], in the order the unsplit pass adds them: per column group the
+// query heads in order, then the column groups in order.
+__global__ void __launch_bounds__(256) merge_partials_kernel(const float* __restrict__ part, float* __restrict__ target,
+                                                             int32_t group, int32_t n_kv_heads, int32_t total_tokens) {
+  const int64_t n = static_cast<int64_t>(n_kv_heads) * total_tokens;
+  const int64_t plane = n;   // one (g, column group) slice
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float sum = 0.f;
+#pragma unroll
+    for (int c = 0; c < kColGroups; ++c) {
+      float heads = 0.f;
+      for (int32_t g = 0; g < group; ++g) heads += part[(static_cast<int64_t>(g) * kColGroups + c) * plane + i];
+      sum = (c == 0) ? heads : sum + heads;
+    }
+    target[i] = sum;
+  }
+}
+
+cudaError_t launch_merge_partials(const float* part, float* target, int group, int n_kv_heads, int total_tokens,
+                                  int sm_count, cudaStream_t stream) {
+  const int64_t n = static_cast<int64_t>(n_kv_heads) * total_tokens;
+  const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, static_cast<int64_t>(sm_count) * 8));
+  merge_partials_kernel<<<std::max(blocks, 1), 256, 0, stream>>>(part, target, group, n_kv_heads, total_tokens);
+  return cudaGetLastError();
+}
+
+int target_split_groups() { return kColGroups; }
 
 // ------------------------------------------------------------------ bounded-wait self-test
 

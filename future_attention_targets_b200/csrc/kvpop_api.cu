@@ -24,6 +24,9 @@ cudaError_t launch_prefix_thresholds(const ThresholdParams& p, int n_kv_heads, i
 cudaError_t launch_compact_kv(const CompactParams& p, cudaStream_t stream);
 cudaError_t launch_decode_attention(const DecodeParams& p, int batch, cudaStream_t stream);
 cudaError_t launch_fused_targets(const FusedParams& fp, int head_dim, int grid, cudaStream_t stream);
+cudaError_t launch_merge_partials(const float* part, float* target, int group, int n_kv_heads, int total_tokens,
+                                  int sm_count, cudaStream_t stream);
+int target_split_groups();
 size_t decode_scratch_bytes();
 cudaError_t decode_scratch_address(float** out);
 }  // namespace kvpop
@@ -217,6 +220,7 @@ kvpop_status fill_attn_common(AttnParams* p, const void* q, const void* k, const
   p->group = sh.n_q_heads / sh.n_kv_heads;
   p->scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p->inv_scale = static_cast<float>(1.0 / static_cast<double>(scale));
+  p->g_split = 1;
   build_schedule(cu, sh.batch, target_pass ? sh.n_kv_heads : sh.n_q_heads, &p->sched, order);
   return KVPOP_OK;
 }
@@ -236,6 +240,54 @@ int64_t flag_tiles(const int32_t* cu, int batch) {
 static_assert(sizeof(FusedParams) <= 32764, "kernel parameter space");
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// KV-head groups of the host-buffer pipeline (copy of group c+1 overlaps the
+// compute of group c).
+constexpr int kHostGroups = 8;
+
+// Two internal streams per device for the host-buffer pipeline's copies in
+// and out, created on first use and kept for the life of the process.
+struct HostStreams {
+  cudaStream_t in = nullptr;
+  cudaStream_t out = nullptr;
+};
+
+kvpop_status host_streams(HostStreams* out) {
+  static std::mutex mu;
+  static std::vector<HostStreams> cache;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lock(mu);
+  if (static_cast<int>(cache.size()) <= dev) cache.resize(dev + 1);
+  HostStreams& h = cache[dev];
+  if (h.in == nullptr) {
+    HostStreams n;
+    if ((e = cudaStreamCreateWithFlags(&n.in, cudaStreamNonBlocking)) == cudaSuccess &&
+        (e = cudaStreamCreateWithFlags(&n.out, cudaStreamNonBlocking)) == cudaSuccess) {
+      h = n;
+    } else {
+      if (n.in != nullptr) cudaStreamDestroy(n.in);
+      return cuda_fail(e, "cudaStreamCreate");
+    }
+  }
+  *out = h;
+  return KVPOP_OK;
+}
+
+// Events of one call, destroyed when the call returns (an event still pending
+// on the GPU is released once it completes).
+struct EventSet {
+  std::vector<cudaEvent_t> ev;
+  cudaError_t make(cudaEvent_t* out) {
+    cudaError_t e = cudaEventCreateWithFlags(out, cudaEventDisableTiming);
+    if (e == cudaSuccess) ev.push_back(*out);
+    return e;
+  }
+  ~EventSet() {
+    for (cudaEvent_t x : ev) cudaEventDestroy(x);
+  }
+};
 
 }  // namespace
 
@@ -298,6 +350,50 @@ kvpop_status kvpop_future_target(const void* q, const void* k, const int32_t* cu
   cudaError_t e = launch_future_target(p, shape.head_dim, grid_for(p.sched.total_items, dev.sm_count),
                                        static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "future_target launch");
+}
+
+size_t kvpop_target_split_workspace_bytes(kvpop_shape shape) {
+  if (shape.total_tokens <= 0 || shape.n_kv_heads <= 0 || shape.n_q_heads <= 0 ||
+      shape.n_q_heads % shape.n_kv_heads != 0)
+    return 0;
+  return static_cast<size_t>(shape.n_q_heads) * target_split_groups() * static_cast<size_t>(shape.total_tokens) *
+         sizeof(float);
+}
+
+kvpop_status kvpop_future_target_split(const void* q, const void* k, const int32_t* cu_seqlens, kvpop_shape shape,
+                                       float scale, int32_t window, const float* lse, float* target, float* partials,
+                                       size_t partials_bytes, int32_t* dev_status, void* stream) {
+  kvpop_status st;
+  if ((st = check_qk(q, k, scale)) != KVPOP_OK) return st;
+  if (lse == nullptr || target == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "lse or target is NULL");
+  if (window < 0) return fail(KVPOP_ERR_INVALID_ARG, "window must be >= 0 (got %d)", window);
+  if ((st = check_shape(cu_seqlens, shape, true)) != KVPOP_OK) return st;
+  const int G = shape.n_q_heads / shape.n_kv_heads;
+  if (G == 1)   // one query head per KV head: the split is the plain pass
+    return kvpop_future_target(q, k, cu_seqlens, shape, scale, window, lse, target, dev_status, stream);
+  const size_t need = kvpop_target_split_workspace_bytes(shape);
+  if (partials == nullptr || partials_bytes < need)
+    return fail(KVPOP_ERR_INVALID_ARG, "partials workspace of %zu bytes is smaller than the %zu required",
+                partials_bytes, need);
+  if ((reinterpret_cast<uintptr_t>(partials) & 15u) != 0)
+    return fail(KVPOP_ERR_INVALID_ARG, "partials must be 16-byte aligned");
+  if (shape.total_tokens == 0) return KVPOP_OK;
+  DeviceInfo dev;
+  if ((st = device_info(&dev)) != KVPOP_OK) return st;
+  AttnParams p;
+  if ((st = fill_attn_common(&p, q, k, cu_seqlens, shape, scale, true)) != KVPOP_OK) return st;
+  build_schedule(cu_seqlens, shape.batch, shape.n_kv_heads * G, &p.sched);
+  p.g_split = G;
+  p.window = std::min<int32_t>(window, kMaxLevels * kTileRows + 1);
+  p.lse_in = lse;
+  p.out = partials;
+  p.status = dev_status;
+  if (p.sched.total_items == 0) return KVPOP_OK;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_future_target(p, shape.head_dim, grid_for(p.sched.total_items, dev.sm_count), s);
+  if (e != cudaSuccess) return cuda_fail(e, "future_target launch");
+  e = launch_merge_partials(partials, target, G, shape.n_kv_heads, shape.total_tokens, dev.sm_count, s);
+  return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "merge of the split partials");
 }
 
 kvpop_status kvpop_keep_mask(const float* score, const int32_t* cu_seqlens, kvpop_shape shape, int32_t window,
@@ -590,11 +686,22 @@ kvpop_status kvpop_future_targets_fused(const void* q, const void* k, const int3
   return kvpop_keep_mask(target, cu_seqlens, shape, window, sinks, budgets, keep, stream);
 }
 
+// Largest KV-head group of the host-buffer pipeline.
+static int host_group_max(int n_kv_heads) {
+  const int n_groups = std::min(n_kv_heads, kHostGroups);
+  return (n_kv_heads + n_groups - 1) / n_groups;
+}
+
 size_t kvpop_host_workspace_bytes(kvpop_shape shape) {
-  if (shape.total_tokens <= 0 || shape.n_q_heads <= 0 || shape.n_kv_heads <= 0 || shape.head_dim <= 0) return 0;
+  if (shape.total_tokens <= 0 || shape.n_q_heads <= 0 || shape.n_kv_heads <= 0 || shape.head_dim <= 0 ||
+      shape.n_q_heads % shape.n_kv_heads != 0)
+    return 0;
   const size_t T = static_cast<size_t>(shape.total_tokens);
+  const size_t G = static_cast<size_t>(shape.n_q_heads / shape.n_kv_heads);
+  const size_t partials = G * host_group_max(shape.n_kv_heads) * target_split_groups() * T * 4;
   return align256(T * shape.n_q_heads * shape.head_dim * 2) + align256(T * shape.n_kv_heads * shape.head_dim * 2) +
-         align256(T * shape.n_q_heads * 4) + align256(T * shape.n_kv_heads * 4) + align256(T * shape.n_kv_heads);
+         align256(T * shape.n_q_heads * 4) + align256(T * shape.n_kv_heads * 4) + align256(T * shape.n_kv_heads) +
+         align256(partials);
 }
 
 kvpop_status kvpop_future_targets_host(const void* q_host, const void* k_host, const int32_t* cu_seqlens,
@@ -604,7 +711,13 @@ kvpop_status kvpop_future_targets_host(const void* q_host, const void* k_host, c
   kvpop_status st;
   if (q_host == nullptr || k_host == nullptr || target_host == nullptr || keep_host == nullptr)
     return fail(KVPOP_ERR_INVALID_ARG, "a host buffer is NULL");
+  if (!isfinite(scale) || !(scale > 0.f)) return fail(KVPOP_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (budgets == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "budgets is NULL");
+  if (window < 0 || sinks < 0) return fail(KVPOP_ERR_INVALID_ARG, "window and sinks must be >= 0");
   if ((st = check_shape(cu_seqlens, shape, true)) != KVPOP_OK) return st;
+  for (int b = 0; b < shape.batch; ++b)
+    if (static_cast<int64_t>(budgets[b]) < static_cast<int64_t>(sinks) + window)
+      return fail(KVPOP_ERR_INVALID_ARG, "budget[%d] = %d is below sinks + window", b, budgets[b]);
   if (shape.total_tokens == 0) return KVPOP_OK;
   const size_t need = kvpop_host_workspace_bytes(shape);
   if (workspace == nullptr || workspace_bytes < need)
@@ -613,25 +726,88 @@ kvpop_status kvpop_future_targets_host(const void* q_host, const void* k_host, c
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(KVPOP_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   const size_t T = static_cast<size_t>(shape.total_tokens);
-  const size_t qb = T * shape.n_q_heads * shape.head_dim * 2, kb = T * shape.n_kv_heads * shape.head_dim * 2;
-  const size_t lb = T * shape.n_q_heads * 4, tb = T * shape.n_kv_heads * 4, mb = T * shape.n_kv_heads;
+  const int G = shape.n_q_heads / shape.n_kv_heads, d = shape.head_dim;
+  const size_t qb = T * shape.n_q_heads * d * 2, kb = T * shape.n_kv_heads * d * 2;
+  const size_t lb = T * shape.n_q_heads * 4, tb = T * shape.n_kv_heads * 4;
   uint8_t* w = static_cast<uint8_t*>(workspace);
-  void* q = w;
-  void* k = w + align256(qb);
+  uint8_t* q_all = w;
+  uint8_t* k_all = w + align256(qb);
   float* lse = reinterpret_cast<float*>(w + align256(qb) + align256(kb));
   float* target = reinterpret_cast<float*>(w + align256(qb) + align256(kb) + align256(lb));
   uint8_t* keep = w + align256(qb) + align256(kb) + align256(lb) + align256(tb);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* partials = reinterpret_cast<float*>(w + align256(qb) + align256(kb) + align256(lb) + align256(tb) +
+                                             align256(T * shape.n_kv_heads));
+  const size_t partials_bytes = need - (align256(qb) + align256(kb) + align256(lb) + align256(tb) +
+                                        align256(T * shape.n_kv_heads));
+  HostStreams hs;
+  if ((st = host_streams(&hs)) != KVPOP_OK) return st;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  // KV-head groups: group c's Q and K land as a compact problem of their own
+  // (strided 2-D copies), so its two passes and keep mask can run while the
+  // next group is still being copied in.  Groups of (nearly) equal size; the
+  // split transposed pass keeps even one-head groups balanced, and smaller
+  // groups leave less compute after the last copy.
+  const int n_groups = std::min(shape.n_kv_heads, kHostGroups);
+  int sizes[kHostGroups] = {};
+  for (int c = 0; c < n_groups; ++c) sizes[c] = shape.n_kv_heads / n_groups + (c < shape.n_kv_heads % n_groups ? 1 : 0);
+  EventSet ev;
   cudaError_t e;
-  if ((e = cudaMemcpyAsync(q, q_host, qb, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy q");
-  if ((e = cudaMemcpyAsync(k, k_host, kb, cudaMemcpyHostToDevice, s)) != cudaSuccess) return cuda_fail(e, "copy k");
-  if ((st = kvpop_future_targets(q, k, cu_seqlens, shape, scale, window, sinks, budgets, lse, target, keep,
-                                 dev_status, stream)) != KVPOP_OK)
-    return st;
-  if ((e = cudaMemcpyAsync(target_host, target, tb, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
-    return cuda_fail(e, "copy target");
-  if ((e = cudaMemcpyAsync(keep_host, keep, mb, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
-    return cuda_fail(e, "copy keep");
+  cudaEvent_t start;
+  if ((e = ev.make(&start)) != cudaSuccess) return cuda_fail(e, "cudaEventCreate");
+  // The copies must not overwrite the workspace while earlier work on `stream` may still read it.
+  if ((e = cudaEventRecord(start, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  if ((e = cudaStreamWaitEvent(hs.in, start, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+  size_t q_off = 0, k_off = 0;
+  int h0 = 0;
+  for (int c = 0; c < n_groups; ++c) {
+    const int hn = sizes[c];
+    const size_t q_row = static_cast<size_t>(hn) * G * d * 2, k_row = static_cast<size_t>(hn) * d * 2;
+    uint8_t* qc = q_all + q_off;
+    uint8_t* kc = k_all + k_off;
+    const uint8_t* qh = static_cast<const uint8_t*>(q_host) + static_cast<size_t>(h0) * G * d * 2;
+    const uint8_t* kh = static_cast<const uint8_t*>(k_host) + static_cast<size_t>(h0) * d * 2;
+    cudaEvent_t copied, computed;
+    if ((e = ev.make(&copied)) != cudaSuccess || (e = ev.make(&computed)) != cudaSuccess)
+      return cuda_fail(e, "cudaEventCreate");
+    if ((e = cudaMemcpy2DAsync(qc, q_row, qh, static_cast<size_t>(shape.n_q_heads) * d * 2, q_row, T,
+                               cudaMemcpyHostToDevice, hs.in)) != cudaSuccess)
+      return cuda_fail(e, "copy q");
+    if ((e = cudaMemcpy2DAsync(kc, k_row, kh, static_cast<size_t>(shape.n_kv_heads) * d * 2, k_row, T,
+                               cudaMemcpyHostToDevice, hs.in)) != cudaSuccess)
+      return cuda_fail(e, "copy k");
+    if ((e = cudaEventRecord(copied, hs.in)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    if ((e = cudaStreamWaitEvent(s, copied, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+    // A group holds few KV heads, so its transposed pass takes one item per
+    // (key tile, query head): same result, G times as many items.
+    kvpop_shape sc = shape;
+    sc.n_q_heads = hn * G;
+    sc.n_kv_heads = hn;
+    float* lse_c = lse + static_cast<size_t>(h0) * G * T;
+    float* target_c = target + static_cast<size_t>(h0) * T;
+    if ((st = kvpop_row_lse(qc, kc, cu_seqlens, sc, scale, lse_c, dev_status, stream)) != KVPOP_OK ||
+        (st = kvpop_future_target_split(qc, kc, cu_seqlens, sc, scale, window, lse_c, target_c, partials,
+                                        partials_bytes, dev_status, stream)) != KVPOP_OK ||
+        (st = kvpop_keep_mask(target_c, cu_seqlens, sc, window, sinks, budgets, keep + static_cast<size_t>(h0) * T,
+                              stream)) != KVPOP_OK)
+      return st;
+    if ((e = cudaEventRecord(computed, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    if ((e = cudaStreamWaitEvent(hs.out, computed, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+    if ((e = cudaMemcpyAsync(target_host + static_cast<size_t>(h0) * T, target + static_cast<size_t>(h0) * T,
+                             static_cast<size_t>(hn) * T * 4, cudaMemcpyDeviceToHost, hs.out)) != cudaSuccess)
+      return cuda_fail(e, "copy target");
+    if ((e = cudaMemcpyAsync(keep_host + static_cast<size_t>(h0) * T, keep + static_cast<size_t>(h0) * T,
+                             static_cast<size_t>(hn) * T, cudaMemcpyDeviceToHost, hs.out)) != cudaSuccess)
+      return cuda_fail(e, "copy keep");
+    q_off += q_row * T;
+    k_off += k_row * T;
+    h0 += hn;
+  }
+  // `stream` completes only after the last copy back.
+  cudaEvent_t done;
+  if ((e = ev.make(&done)) != cudaSuccess) return cuda_fail(e, "cudaEventCreate");
+  if ((e = cudaEventRecord(done, hs.out)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+  if ((e = cudaStreamWaitEvent(s, done, 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
   return KVPOP_OK;
 }
 

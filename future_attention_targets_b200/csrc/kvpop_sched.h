@@ -43,6 +43,7 @@ struct AttnParams {
   int32_t window;
   float scale_log2;       // softmax scale * log2(e)
   float inv_scale;        // 1 / softmax scale (pass 2 normaliser slab)
+  int32_t g_split;        // pass 2: 1 = an item covers the G query heads; G = one query head per item
   LevelSchedule sched;
 };
 

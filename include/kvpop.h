@@ -107,6 +107,24 @@ KVPOP_API kvpop_status kvpop_future_target(const void* q, const void* k, const i
                                  const float* lse, float* target,
                                  int32_t* dev_status, void* stream);
 
+/* Device workspace (bytes) of kvpop_future_target_split:
+ * n_q_heads * 4 * T floats (per query head and softmax column group). */
+KVPOP_API size_t kvpop_target_split_workspace_bytes(kvpop_shape shape);
+
+/* kvpop_future_target with one work item per (key tile, query head) instead
+ * of per (key tile, KV head): for few KV heads per call (a group of heads, a
+ * tensor-parallel shard) the G-fold larger item count keeps every SM busy.
+ * Each item writes per-head partial sums to `partials`; a second kernel adds
+ * them in the order the one-item-per-KV-head pass uses, so `target` is
+ * bit-identical to kvpop_future_target's.  With G = 1 it is that call.
+ *   partials   device, >= kvpop_target_split_workspace_bytes(shape) bytes,
+ *              16-byte aligned; contents on entry are ignored
+ * Other arguments as for kvpop_future_target. */
+KVPOP_API kvpop_status kvpop_future_target_split(const void* q, const void* k, const int32_t* cu_seqlens,
+                                                 kvpop_shape shape, float scale, int32_t window, const float* lse,
+                                                 float* target, float* partials, size_t partials_bytes,
+                                                 int32_t* dev_status, void* stream);
+
 /* Sink + top-k + recent-window keep set (model card, introduction; French
  * article, second paragraph).  Per sequence b and KV head h: keep p < sinks,
  * keep p >= L - window, and among p in [sinks, L - window) keep the
@@ -255,8 +273,15 @@ KVPOP_API size_t kvpop_host_workspace_bytes(kvpop_shape shape);
 /* The whole hot path on HOST buffers: copies q and k (host, preferably pinned)
  * into `workspace` (device, at least kvpop_host_workspace_bytes(shape) bytes,
  * 256-byte aligned), runs the three passes and copies target and keep back to
- * host memory, all enqueued on `stream`.  The results are valid once the
- * stream has been synchronised. */
+ * host memory.  The KV heads are processed in up to eight groups of nearly
+ * equal size (every head's result depends only on its own K head and query
+ * heads): each group's passes run on `stream` as soon as its copy in has
+ * landed, while the next group is copied in.  The copies in and back run on
+ * two internal streams that the library creates once per device.  The
+ * copies in wait for the work already queued on `stream` (which may still
+ * read the workspace), and `stream` waits for the last copy back, so the
+ * results are valid once `stream` has been synchronised.
+ * Results are identical to kvpop_future_targets on device copies of q and k. */
 KVPOP_API kvpop_status kvpop_future_targets_host(const void* q_host, const void* k_host,
                                        const int32_t* cu_seqlens, kvpop_shape shape,
                                        float scale, int32_t window, int32_t sinks,

@@ -17,7 +17,7 @@ def lib():
 
 def test_exports_every_header_symbol(lib):
     names = B.header_symbols()
-    assert len(names) == 18, names
+    assert len(names) == 20, names
     for name in names:
         assert hasattr(lib, name), f"{name} declared in kvpop.h but not exported"
     assert set(names) == set(B._SIGS), "binding signatures and header disagree"
@@ -157,9 +157,25 @@ def test_workspace_bytes(lib):
     sh = B.Shape(1, 16384, 32, 8, 128)
     r = lambda x: (x + 255) // 256 * 256
     T = 16384
-    want = r(T * 32 * 128 * 2) + r(T * 8 * 128 * 2) + r(T * 32 * 4) + r(T * 8 * 4) + r(T * 8)
+    # q, k, lse, target, keep, and the split partials of the largest KV-head group
+    # (eight groups of one head: G = 4 query heads x 4 column groups x T floats)
+    want = (r(T * 32 * 128 * 2) + r(T * 8 * 128 * 2) + r(T * 32 * 4) + r(T * 8 * 4) + r(T * 8) +
+            r(4 * 1 * 4 * T * 4))
     assert lib.kvpop_host_workspace_bytes(sh) == want
     assert lib.kvpop_host_workspace_bytes(B.Shape(1, 0, 32, 8, 128)) == 0
+
+
+def test_split_target_rejects_and_sizes(lib):
+    cu, sh = _cu(0, 100), _shape()                       # 4 query heads over 2 KV heads
+    need = lib.kvpop_target_split_workspace_bytes(sh)
+    assert need == 4 * 4 * 100 * 4                      # query heads x column groups x T floats
+    S = lib.kvpop_future_target_split
+    assert S(FAKE, FAKE, cu, sh, 0.1, 16, FAKE, FAKE, None, need, None, None) == B.INVALID_ARG       # no workspace
+    assert S(FAKE, FAKE, cu, sh, 0.1, 16, FAKE, FAKE, FAKE, need - 4, None, None) == B.INVALID_ARG   # too small
+    assert S(FAKE, FAKE, cu, sh, 0.1, 16, FAKE, FAKE, FAKE + 4, need, None, None) == B.INVALID_ARG   # misaligned
+    assert S(FAKE, FAKE, cu, sh, 0.1, -1, FAKE, FAKE, FAKE, need, None, None) == B.INVALID_ARG       # window
+    assert S(FAKE, FAKE, cu, sh, 0.1, 16, None, FAKE, FAKE, need, None, None) == B.INVALID_ARG       # lse
+    assert lib.kvpop_target_split_workspace_bytes(B.Shape(1, 100, 6, 4, 128)) == 0                  # 6 % 4 != 0
 
 
 def test_fused_workspace_bytes(lib):

@@ -251,6 +251,30 @@ def test_host_pipeline_matches_device():
     np.testing.assert_array_equal(k_h.numpy(), keep)
 
 
+@pytest.mark.parametrize("seqlens,hq,hkv,d", [((700, 1, 300), 12, 6, 128),   # six groups of one KV head
+                                               ((900,), 16, 8, 64),             # eight groups of one
+                                               ((600,), 20, 10, 64),            # groups of 2, 2, 1, ... 1
+                                               ((513,), 3, 3, 64),              # three groups of one
+                                               ((200,), 4, 1, 128)])            # one group
+def test_host_pipeline_groups_match_device(seqlens, hq, hkv, d):
+    """The host-buffer pipeline splits the KV heads into groups copied and computed in turn; every
+    group must reproduce the device pipeline exactly, also when the call is repeated on one workspace."""
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    T = int(cu[-1])
+    q_bits, k_bits = random_qk(T, hq, hkv, d, seed=T + hkv)
+    scale, W, S = 1.0 / math.sqrt(d), 32, 4
+    budgets = [max(S + W, L // 3) for L in seqlens]
+    _, tgt, keep = run_gpu(q_bits, k_bits, cu, W, S, budgets, scale)
+    pipe = B.HostPipeline(cu, hq, hkv, d, W, S, budgets, scale)
+    qh = torch.from_numpy(q_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    kh = torch.from_numpy(k_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    for _ in range(2):
+        t_h, k_h = pipe(qh, kh)
+        np.testing.assert_array_equal(t_h.numpy(), tgt)
+        np.testing.assert_array_equal(k_h.numpy(), keep)
+    check_status(pipe.status)
+
+
 def test_bounded_wait_times_out_and_context_survives():
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     selftest_bounded_wait(status, 50_000_000)          # 50 ms on a barrier nothing completes
