@@ -52,7 +52,7 @@ constexpr int kColGroups = 4;                          // softmax warp groups pe
 constexpr int kGroupCols = kStreamRows / kColGroups;   // accumulator columns per group
 constexpr int kSoftmaxWarps = 4 * kColGroups;          // one warp per TMEM lane quadrant per group
 static_assert(kThreads == 32 * (2 + kSoftmaxWarps), "producer warp + MMA warp + softmax warps");
-static_assert(kGroupCols == 64, "group_exp_sum walks two 32-column chunks");
+static_assert(kGroupCols == 64, "group_exp_sum walks four 16-column chunks");
 // Extra K=16 slab (no swizzle, K-major): 8-row groups of two 8x16-byte core
 // matrices; element (r, e) sits at (r/8)*256 + (e/8)*128 + (r%8)*16 + (e%8)*2.
 constexpr int kSlabLBO = 128;   // between the two core matrices along K
@@ -638,18 +638,19 @@ __device__ __forceinline__ constexpr bool poly_pair(int q) {
   return ((q * kPoly) & 15) < kPoly;
 }
 
-// acc += exp2(x * c + nb) over one 32-column chunk (nb: one negated offset
-// for the whole chunk); kPoly of the 16 pairs go through the polynomial, the
-// rest through MUFU.  kBiasFree: nb is zero (pass 2), the scale is folded
-// into the polynomial's range reduction and x >= xmin keeps c x >= -126.
-template <int kPoly, bool kBiasFree>
-__device__ __forceinline__ void chunk_exp_sum(const uint32_t (&r)[32], uint64_t c2, uint64_t nb, float xmin,
+// acc += exp2(x * c + nb) over one 16-column chunk (nb: one negated offset
+// for the whole chunk); of every 16 pairs kPoly go through the polynomial
+// (pairs kQ0 .. kQ0+7 of that pattern are this chunk's), the rest through
+// MUFU.  kBiasFree: nb is zero (pass 2), the scale is folded into the
+// polynomial's range reduction and x >= xmin keeps c x >= -126.
+template <int kPoly, bool kBiasFree, int kQ0>
+__device__ __forceinline__ void chunk_exp_sum(const uint32_t (&r)[16], uint64_t c2, uint64_t nb, float xmin,
                                               uint64_t (&acc)[4]) {
 #pragma unroll
-  for (int q = 0; q < 16; ++q) {
+  for (int q = 0; q < 8; ++q) {
     const uint64_t x = f2_pack(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
     uint64_t e;
-    if (poly_pair<kPoly>(q)) {
+    if (poly_pair<kPoly>(kQ0 + q)) {
       e = kBiasFree ? exp2_poly_pair_scaled(x, c2, xmin) : exp2_poly_pair(f2_fma(x, c2, nb));
     } else {
       e = exp2_mufu_pair(f2_fma(x, c2, nb));
@@ -660,10 +661,10 @@ __device__ __forceinline__ void chunk_exp_sum(const uint32_t (&r)[32], uint64_t 
 
 // Same with only columns lo <= e < hi of the chunk counted (MUFU only, so
 // huge negative arguments give exact zeros).
-__device__ __forceinline__ void chunk_exp_sum_masked(const uint32_t (&r)[32], uint64_t c2, uint64_t nb, int lo,
+__device__ __forceinline__ void chunk_exp_sum_masked(const uint32_t (&r)[16], uint64_t c2, uint64_t nb, int lo,
                                                      int hi, uint64_t (&acc)[4]) {
 #pragma unroll
-  for (int q = 0; q < 16; ++q) {
+  for (int q = 0; q < 8; ++q) {
     const uint64_t x = f2_pack(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
     float y0, y1;
     f2_unpack(f2_fma(x, c2, nb), y0, y1);
@@ -682,25 +683,31 @@ __device__ __forceinline__ float acc_total(uint64_t (&acc)[4]) {
 }
 
 // Sum of exp2(x * c - off) over the kGroupCols = 64 columns of this thread's
-// TMEM lane starting at taddr: two chunks of 32, the second load in flight
-// while the first chunk is summed.  kMasked: column m counts iff lo <= m < hi.
+// TMEM lane starting at taddr: four chunks of 16, each load in flight while
+// the chunk before it is summed (small chunks shorten the load every warp of
+// the CTA waits for at the start of a tile).  kMasked: column m counts iff
+// lo <= m < hi.
 template <bool kMasked, int kPoly, bool kBiasFree = false>
 __device__ __forceinline__ float group_exp_sum(uint32_t taddr, uint64_t c2, uint64_t nb, int lo, int hi,
                                                float xmin = 0.f) {
-  uint32_t ra[32], rb[32];
+  uint32_t ra[16], rb[16];
   uint64_t acc[4] = {0, 0, 0, 0};
-  auto run = [&](const uint32_t (&r)[32], int ch) {
-    if constexpr (kMasked)
-      chunk_exp_sum_masked(r, c2, nb, lo - 32 * ch, hi - 32 * ch, acc);
-    else
-      chunk_exp_sum<kPoly, kBiasFree>(r, c2, nb, xmin, acc);
-  };
-  tmem_load<32>(taddr, ra);
-  tmem_load_wait<32>(ra);
-  tmem_load<32>(taddr + 32, rb);
-  run(ra, 0);
-  tmem_load_wait<32>(rb);
-  run(rb, 1);
+  tmem_load<16>(taddr, ra);
+  tmem_load_wait<16>(ra);
+  tmem_load<16>(taddr + 16, rb);
+  if constexpr (kMasked) chunk_exp_sum_masked(ra, c2, nb, lo, hi, acc);
+  else chunk_exp_sum<kPoly, kBiasFree, 0>(ra, c2, nb, xmin, acc);
+  tmem_load_wait<16>(rb);
+  tmem_load<16>(taddr + 32, ra);
+  if constexpr (kMasked) chunk_exp_sum_masked(rb, c2, nb, lo - 16, hi - 16, acc);
+  else chunk_exp_sum<kPoly, kBiasFree, 8>(rb, c2, nb, xmin, acc);
+  tmem_load_wait<16>(ra);
+  tmem_load<16>(taddr + 48, rb);
+  if constexpr (kMasked) chunk_exp_sum_masked(ra, c2, nb, lo - 32, hi - 32, acc);
+  else chunk_exp_sum<kPoly, kBiasFree, 0>(ra, c2, nb, xmin, acc);
+  tmem_load_wait<16>(rb);
+  if constexpr (kMasked) chunk_exp_sum_masked(rb, c2, nb, lo - 48, hi - 48, acc);
+  else chunk_exp_sum<kPoly, kBiasFree, 8>(rb, c2, nb, xmin, acc);
   return acc_total(acc);
 }
 
