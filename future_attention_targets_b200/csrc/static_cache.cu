@@ -195,247 +195,228 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// Packed fp32 pairs (the f32x2 forms issue two lanes of work per instruction).
-__device__ __forceinline__ uint64_t dec_pack(float a, float b) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1,%2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
+// Warp-level bf16 MMA (m16n8k16, fp32 accumulate) and the shared-memory
+// matrix loads that feed it.  A decode step is a G x d by d x n product and
+// its P.V follow-up; with the G query heads padded to the MMA's 16 rows one
+// instruction does the multiply-adds that would otherwise take hundreds of
+// scalar ones, which keeps this memory-bound kernel off the issue limit.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const uint16_t* row) {
+  const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(row));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
 }
-__device__ __forceinline__ void dec_unpack(uint64_t v, float& a, float& b) {
-  asm("mov.b64 {%0,%1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const uint16_t* row) {
+  const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(row));
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
 }
-__device__ __forceinline__ uint64_t dec_fma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-__device__ __forceinline__ uint64_t dec_mul2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("mul.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
 }
-// Two bf16 in one 32-bit word -> the packed pair (low half first).
-__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
-  return dec_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-}
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
-// D consecutive bf16 (D = 2, 4 or 8; 4, 8 or 16 aligned bytes) as D / 2 packed pairs.
-template <int D>
-__device__ __forceinline__ void load_pairs(const uint16_t* p, uint64_t (&x)[D / 2]) {
-  if constexpr (D == 8) {
-    const uint4 w = *reinterpret_cast<const uint4*>(p);
-    x[0] = bf16x2_to_f32x2(w.x); x[1] = bf16x2_to_f32x2(w.y);
-    x[2] = bf16x2_to_f32x2(w.z); x[3] = bf16x2_to_f32x2(w.w);
-  } else if constexpr (D == 4) {
-    const uint2 w = *reinterpret_cast<const uint2*>(p);
-    x[0] = bf16x2_to_f32x2(w.x); x[1] = bf16x2_to_f32x2(w.y);
-  } else {
-    x[0] = bf16x2_to_f32x2(*reinterpret_cast<const uint32_t*>(p));
-  }
-}
-
-// Sums v[i] over the N lanes of a lane group for all N indices at once and
-// leaves the sum of index `sub` (the lane's index in its group) in that
-// lane: at each butterfly level a lane keeps the half of its entries whose
-// index bit matches its own lane bit and ships the other half to its partner
-// (N - 1 shuffles for N sums).
-template <int N>
-__device__ __forceinline__ float transpose_reduce(float (&v)[N], int sub) {
-#pragma unroll
-  for (int w = N / 2; w >= 1; w >>= 1) {
-    const bool upper = (sub & w) != 0;
-#pragma unroll
-    for (int i = 0; i < w; ++i) {
-      const float send = upper ? v[i] : v[i + w];
-      const float keep = upper ? v[i + w] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
-    }
-  }
-  return v[0];
+// Shared-memory address of 16-byte chunk `c` of cache row `r` (rows of HD
+// bf16): the chunks of a row are permuted by r mod 8, so the eight row
+// addresses of an ldmatrix hit eight different bank groups.
+template <int HD>
+__device__ __forceinline__ uint16_t* swz(uint16_t* base, int r, int c) {
+  return base + r * HD + ((c ^ (r & 7)) << 3);
 }
 
 // One CTA: KV head h of sequence b, cache slots [split * kDecSplit, ...), all
-// G query heads of the group.  Each warp stages its 32 rows of K and V in
-// shared memory with one burst of cp.async (two commit groups, so the first
-// rows can be used while the rest arrive), then walks them in batches of
-// R = 32 / G rows.  A row is owned by a group of LPR lanes (16 when G <= 4,
-// else 32), each holding D = d / LPR head dims, so a warp step covers
-// 32 / LPR rows.  The q.k partial sums of a batch (LPR per lane) become one
-// score per lane with one transpose-reduce (lane index i * G + g of its group
-// = batch row i of the group, head g); the online softmax runs on those
-// lanes, then the P.V update with packed f32x2 FMAs.
-template <int LPR, int D, int G>
+// G <= 16 query heads of the group.  Each warp stages its 32 rows of K and V
+// in shared memory with one burst of cp.async (rows past the filled slots
+// are zeroed so 0 x garbage cannot make a NaN), then:
+//   S = Q K^T   16 (heads, padded) x 32 keys, fp32, by MMA (q unscaled bf16,
+//               the scale applied to S in fp32)
+//   softmax     per head over its 32 keys (rows of S live on four lanes)
+//   O = P V     16 x d, P split into bf16 high and low parts (two MMAs) so the
+//               product keeps ~16 bits of P
+// and the four warps' (max, sum, O) are merged in shared memory into this
+// split's partial.
+template <int HD>
 __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_constant__ DecodeParams p) {
-  constexpr int d = LPR * D;
-  constexpr int RS = 32 / LPR;          // rows per warp step
-  constexpr int R = 32 / G;             // rows per batch
-  constexpr int NI = R / RS;            // rows of one lane group per batch
-  constexpr int P = D / 2;              // packed pairs per lane
-  constexpr int kWords = d / 8;
-  static_assert(NI * G == LPR, "one score per lane after the transpose-reduce");
-  extern __shared__ __align__(16) uint16_t dec_smem[];     // K rows [kDecSplit][d], then V rows
-  __shared__ float sm_m[kDecThreads / 32][G];
-  __shared__ float sm_l[kDecThreads / 32][G];
+  constexpr int kChunks = HD / 8;      // 16-byte chunks per row
+  constexpr int KS = HD / 16;          // k-steps of S = Q K^T
+  constexpr int NT = HD / 8;           // 8-column tiles of O
+  extern __shared__ __align__(16) uint16_t dec_smem[];     // K rows [kDecSplit][HD], then V rows (swizzled)
+  __shared__ float sm_m[kDecThreads / 32][16];
+  __shared__ float sm_l[kDecThreads / 32][16];
 
   const int bh = blockIdx.x, split = blockIdx.y;
   const int b = bh / p.n_kv_heads, h = bh - b * p.n_kv_heads;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int grp = lane / LPR, sub = lane % LPR;
+  const int gid = lane >> 2, tid4 = lane & 3;
+  const int G = p.n_q_heads / p.n_kv_heads;
   const int n = min(p.count[b * p.n_kv_heads + h], p.capacity);
   const int w_lo = split * kDecSplit + warp * kDecRowsPerWarp;
   const int rows = max(0, min(kDecRowsPerWarp, n - w_lo));
-  uint16_t* sk = dec_smem + warp * kDecRowsPerWarp * d;
-  uint16_t* sv = dec_smem + kDecSplit * d + warp * kDecRowsPerWarp * d;
+  uint16_t* sk = dec_smem + warp * kDecRowsPerWarp * HD;
+  uint16_t* sv = dec_smem + kDecSplit * HD + warp * kDecRowsPerWarp * HD;
   {
-    const int64_t g0 = ((static_cast<int64_t>(b) * p.n_kv_heads + h) * p.capacity + w_lo) * d;
-    const int half_words = min(rows, kDecRowsPerWarp / 2) * kWords;
-    for (int idx = lane; idx < half_words; idx += 32) {
-      cp_async16(sk + idx * 8, p.k_cache + g0 + idx * 8);
-      cp_async16(sv + idx * 8, p.v_cache + g0 + idx * 8);
+    const int64_t g0 = ((static_cast<int64_t>(b) * p.n_kv_heads + h) * p.capacity + w_lo) * HD;
+    for (int idx = lane; idx < rows * kChunks; idx += 32) {
+      const int r = idx / kChunks, c = idx - r * kChunks;
+      cp_async16(swz<HD>(sk, r, c), p.k_cache + g0 + idx * 8);
+      cp_async16(swz<HD>(sv, r, c), p.v_cache + g0 + idx * 8);
     }
     cp_async_commit();
-    for (int idx = half_words + lane; idx < rows * kWords; idx += 32) {
-      cp_async16(sk + idx * 8, p.k_cache + g0 + idx * 8);
-      cp_async16(sv + idx * 8, p.v_cache + g0 + idx * 8);
+    for (int idx = rows * kChunks + lane; idx < kDecRowsPerWarp * kChunks; idx += 32) {
+      const int r = idx / kChunks, c = idx - r * kChunks;
+      *reinterpret_cast<uint4*>(swz<HD>(sv, r, c)) = make_uint4(0, 0, 0, 0);
     }
-    cp_async_commit();
   }
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  uint64_t q2[G][P];
+  // q as the A operand: rows = query heads (>= G read as 0), cols = head dims.
+  uint32_t qa[KS][4];
+  {
+    const uint16_t* qb = p.q + (static_cast<int64_t>(b) * p.n_q_heads + h * G) * HD;
 #pragma unroll
-  for (int g = 0; g < G; ++g) {
-    load_pairs<D>(p.q + (static_cast<int64_t>(b) * p.n_q_heads + h * G + g) * d + sub * D, q2[g]);
-    const uint64_t s2 = dec_pack(p.scale_log2, p.scale_log2);   // scores in log2 units
-#pragma unroll
-    for (int j = 0; j < P; ++j) q2[g][j] = dec_mul2(q2[g][j], s2);
-  }
-  float m = -INFINITY, l = 0.f;      // running max and sum of head sub % G (equal on all its lanes)
-  uint64_t o2[G][P];
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int j = 0; j < P; ++j) o2[g][j] = 0ull;
-
-  bool all_here = false;
-  for (int r0 = 0; r0 < rows; r0 += R) {
-    if (!all_here) {
-      if (r0 + R <= kDecRowsPerWarp / 2) {
-        cp_async_wait<1>();
-      } else {
-        cp_async_wait<0>();
-        all_here = true;
-      }
-      __syncwarp();
-    }
-    float part[LPR];
-#pragma unroll
-    for (int i = 0; i < NI; ++i) {
-      uint64_t k2[P];
-      load_pairs<D>(sk + (r0 + i * RS + grp) * d + sub * D, k2);
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        uint64_t acc = dec_mul2(q2[g][0], k2[0]);
-#pragma unroll
-        for (int j = 1; j < P; ++j) acc = dec_fma2(q2[g][j], k2[j], acc);
-        float a, c;
-        dec_unpack(acc, a, c);
-        part[i * G + g] = a + c;
-      }
-    }
-    float x = transpose_reduce<LPR>(part, sub);
-    if (r0 + (sub / G) * RS + grp >= rows) x = -INFINITY;   // past the filled slots (never read below)
-    float bm = x;
-#pragma unroll
-    for (int off = G; off < 32; off <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
-    const float mn = fmaxf(m, bm);
-    const bool none = (mn == -INFINITY);
-    const float corr = none ? 1.f : exp2f(m - mn);
-    const float pr = none ? 0.f : exp2f(x - mn);
-    float bs = pr;
-#pragma unroll
-    for (int off = G; off < 32; off <<= 1) bs += __shfl_xor_sync(0xffffffffu, bs, off);
-    l = l * corr + bs;
-    m = mn;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float c = __shfl_sync(0xffffffffu, corr, g);
-      const uint64_t c2 = dec_pack(c, c);
-#pragma unroll
-      for (int j = 0; j < P; ++j) o2[g][j] = dec_mul2(o2[g][j], c2);
-    }
-#pragma unroll
-    for (int i = 0; i < NI; ++i) {
-      const int row = r0 + i * RS + grp;
-      uint64_t v2[P];
-      if (row < rows) {
-        load_pairs<D>(sv + row * d + sub * D, v2);
-      } else {
-#pragma unroll
-        for (int j = 0; j < P; ++j) v2[j] = 0ull;
-      }
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float pg = __shfl_sync(0xffffffffu, pr, grp * LPR + i * G + g);
-        const uint64_t p2 = dec_pack(pg, pg);
-#pragma unroll
-        for (int j = 0; j < P; ++j) o2[g][j] = dec_fma2(p2, v2[j], o2[g][j]);
-      }
+    for (int kk = 0; kk < KS; ++kk) {
+      const int d0 = 16 * kk + 2 * tid4;
+      qa[kk][0] = (gid < G) ? *reinterpret_cast<const uint32_t*>(qb + gid * HD + d0) : 0u;
+      qa[kk][1] = (gid + 8 < G) ? *reinterpret_cast<const uint32_t*>(qb + (gid + 8) * HD + d0) : 0u;
+      qa[kk][2] = (gid < G) ? *reinterpret_cast<const uint32_t*>(qb + gid * HD + d0 + 8) : 0u;
+      qa[kk][3] = (gid + 8 < G) ? *reinterpret_cast<const uint32_t*>(qb + (gid + 8) * HD + d0 + 8) : 0u;
     }
   }
-  cp_async_wait<0>();                // nothing left in flight when the staging area is reused
+  cp_async_wait<0>();
+  __syncwarp();
 
-  // The lane groups hold the same dims for different rows: add them up.
+  // S = Q K^T over the warp's 32 keys: four 8-key tiles.
+  float s[4][4];
 #pragma unroll
-  for (int g = 0; g < G; ++g)
+  for (int j = 0; j < 4; ++j)
 #pragma unroll
-    for (int j = 0; j < P; ++j)
+    for (int e = 0; e < 4; ++e) s[j][e] = 0.f;
+  const int mi = lane >> 3, ri = lane & 7;    // this lane's ldmatrix row address: matrix mi, row ri
 #pragma unroll
-      for (int off = LPR; off < 32; off <<= 1) {
-        const uint64_t y = __shfl_xor_sync(0xffffffffu, static_cast<unsigned long long>(o2[g][j]), off);
-        float a, c, ya, yc;
-        dec_unpack(o2[g][j], a, c);
-        dec_unpack(y, ya, yc);
-        o2[g][j] = dec_pack(a + ya, c + yc);
-      }
+  for (int kk = 0; kk < KS; ++kk) {
+#pragma unroll
+    for (int np = 0; np < 2; ++np) {
+      uint32_t kb[4];
+      ldsm_x4(kb, swz<HD>(sk, 16 * np + (mi >> 1) * 8 + ri, 2 * kk + (mi & 1)));
+      mma_bf16(s[2 * np], qa[kk], kb[0], kb[1]);
+      mma_bf16(s[2 * np + 1], qa[kk], kb[2], kb[3]);
+    }
+  }
+  // Scale to log2 units, mask keys past the filled slots, softmax per head row
+  // (rows gid and gid + 8 of S; a row's 32 keys are spread over four lanes).
+  float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int key = 8 * j + 2 * tid4 + (e & 1);
+      s[j][e] = (key < rows) ? s[j][e] * p.scale_log2 : -INFINITY;
+      if (e < 2) mx0 = fmaxf(mx0, s[j][e]); else mx1 = fmaxf(mx1, s[j][e]);
+    }
+#pragma unroll
+  for (int off = 1; off <= 2; off <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+  }
+  float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float m = (e < 2) ? mx0 : mx1;
+      const float pe = (m == -INFINITY) ? 0.f : exp2f(s[j][e] - m);
+      s[j][e] = pe;
+      if (e < 2) l0 += pe; else l1 += pe;
+    }
+#pragma unroll
+  for (int off = 1; off <= 2; off <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+  }
+
+  // O = P V: two k-steps of 16 keys, P as the A operand straight from S's
+  // registers (high and low bf16 parts), V through transposing matrix loads.
+  float o[NT][4];
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[t][e] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < 2; ++kk) {
+    uint32_t ph[4], pl[4];
+    const float* t0 = s[2 * kk];
+    const float* t1 = s[2 * kk + 1];
+    const float src[4][2] = {{t0[0], t0[1]}, {t0[2], t0[3]}, {t1[0], t1[1]}, {t1[2], t1[3]}};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      ph[i] = pack_bf16x2(src[i][0], src[i][1]);
+      pl[i] = pack_bf16x2(src[i][0] - bf16_lo(ph[i]), src[i][1] - bf16_hi(ph[i]));
+    }
+#pragma unroll
+    for (int jp = 0; jp < NT / 2; ++jp) {
+      uint32_t vb[4];
+      ldsm_x4_trans(vb, swz<HD>(sv, 16 * kk + (mi & 1) * 8 + ri, 2 * jp + (mi >> 1)));
+      mma_bf16(o[2 * jp], ph, vb[0], vb[1]);
+      mma_bf16(o[2 * jp], pl, vb[0], vb[1]);
+      mma_bf16(o[2 * jp + 1], ph, vb[2], vb[3]);
+      mma_bf16(o[2 * jp + 1], pl, vb[2], vb[3]);
+    }
+  }
 
   // Merge the four warps (the K/V staging area is reused for their outputs),
   // then write this split's partial.
-  if (lane < G) {
-    sm_m[warp][lane] = m;
-    sm_l[warp][lane] = l;
+  if (tid4 == 0) {
+    if (gid < G) {
+      sm_m[warp][gid] = mx0;
+      sm_l[warp][gid] = l0;
+    }
+    if (gid + 8 < G) {
+      sm_m[warp][gid + 8] = mx1;
+      sm_l[warp][gid + 8] = l1;
+    }
   }
   __syncthreads();
-  float* so = reinterpret_cast<float*>(dec_smem);          // [4][G][d]
-  if (grp == 0) {
+  float* so = reinterpret_cast<float*>(dec_smem);          // [4][G][HD]
 #pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-      for (int j = 0; j < P; ++j) {
-        float a, c;
-        dec_unpack(o2[g][j], a, c);
-        so[(warp * G + g) * d + sub * D + 2 * j] = a;
-        so[(warp * G + g) * d + sub * D + 2 * j + 1] = c;
-      }
+  for (int t = 0; t < NT; ++t) {
+    const int d0 = 8 * t + 2 * tid4;
+    if (gid < G) {
+      so[(warp * G + gid) * HD + d0] = o[t][0];
+      so[(warp * G + gid) * HD + d0 + 1] = o[t][1];
+    }
+    if (gid + 8 < G) {
+      so[(warp * G + gid + 8) * HD + d0] = o[t][2];
+      so[(warp * G + gid + 8) * HD + d0 + 1] = o[t][3];
+    }
   }
   __syncthreads();
-  for (int idx = threadIdx.x; idx < G * d; idx += kDecThreads) {
-    const int g = idx / d, e = idx - g * d;
+  for (int idx = threadIdx.x; idx < G * HD; idx += kDecThreads) {
+    const int g = idx / HD, e = idx - g * HD;
     float mm = -INFINITY;
     for (int w = 0; w < kDecThreads / 32; ++w) mm = fmaxf(mm, sm_m[w][g]);
     float ll = 0.f, oo = 0.f;
     if (mm > -INFINITY) {
       for (int w = 0; w < kDecThreads / 32; ++w) {
-        const float c = exp2f(sm_m[w][g] - mm);
+        const float c = (sm_m[w][g] > -INFINITY) ? exp2f(sm_m[w][g] - mm) : 0.f;
         ll += sm_l[w][g] * c;
-        oo += so[(w * G + g) * d + e] * c;
+        oo += so[(w * G + g) * HD + e] * c;
       }
     }
-    float* dst = p.partial + ((static_cast<int64_t>(b) * p.n_q_heads + h * G + g) * p.n_split + split) * (d + 2);
+    float* dst = p.partial + ((static_cast<int64_t>(b) * p.n_q_heads + h * G + g) * p.n_split + split) * (HD + 2);
     dst[e] = oo;
     if (e == 0) {
-      dst[d] = mm;
-      dst[d + 1] = ll;
+      dst[HD] = mm;
+      dst[HD + 1] = ll;
     }
   }
 }
@@ -461,55 +442,58 @@ __device__ __forceinline__ float block_reduce_128(float x, float* red, bool is_m
 
 __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_constant__ DecodeParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  constexpr int kMaxSplitsInSmem = 1024;      // split weights kept in shared memory (more splits: recomputed)
   __shared__ float red[4];
+  __shared__ float wsplit[kMaxSplitsInSmem];
   const int bg = blockIdx.x, tid = threadIdx.x;
   const int d = p.head_dim, ns = p.n_split, stride = d + 2;
   const float* part = p.partial + static_cast<int64_t>(bg) * ns * stride;
+  // Split maxima, their maximum, then each split's weight exp2(m_s - m) and the total sum.
   float mm = -INFINITY;
   for (int s = tid; s < ns; s += 128) mm = fmaxf(mm, part[s * stride + d]);
   mm = block_reduce_128(mm, red, true);
   float ll = 0.f;
-  if (mm > -INFINITY)
-    for (int s = tid; s < ns; s += 128) ll += part[s * stride + d + 1] * exp2f(part[s * stride + d] - mm);
-  ll = block_reduce_128(ll, red, false);
+  for (int s = tid; s < ns; s += 128) {
+    const float m_s = part[s * stride + d];
+    const float w = (mm > -INFINITY && m_s > -INFINITY) ? exp2f(m_s - mm) : 0.f;
+    if (s < kMaxSplitsInSmem) wsplit[s] = w;
+    ll += part[s * stride + d + 1] * w;
+  }
+  ll = block_reduce_128(ll, red, false);   // its barriers also publish wsplit
+  // Output: 16 independent loads in flight per thread before their sums.
   for (int e = tid; e < d; e += 128) {
     float oo = 0.f;
-    if (mm > -INFINITY) {
-#pragma unroll 8
-      for (int s = 0; s < ns; ++s) oo += part[s * stride + e] * exp2f(part[s * stride + d] - mm);
+    int s = 0;
+    for (; s + 16 <= ns && s + 16 <= kMaxSplitsInSmem; s += 16) {
+      float v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) v[u] = part[(s + u) * stride + e];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) oo = fmaf(v[u], wsplit[s + u], oo);
+    }
+    for (; s < ns; ++s) {
+      const float m_s = part[s * stride + d];
+      const float w = (s < kMaxSplitsInSmem) ? wsplit[s]
+                                             : ((mm > -INFINITY && m_s > -INFINITY) ? exp2f(m_s - mm) : 0.f);
+      oo = fmaf(part[s * stride + e], w, oo);
     }
     p.out[static_cast<int64_t>(bg) * d + e] = (ll > 0.f) ? oo / ll : 0.f;
   }
   if (tid == 0 && p.lse != nullptr) p.lse[bg] = (ll > 0.f) ? (mm + log2f(ll)) * 0.6931471805599453f : -INFINITY;
 }
 
-template <int LPR, int D, int G>
-static cudaError_t launch_split_g(const DecodeParams& p, dim3 grid, cudaStream_t stream) {
-  const int smem = 2 * kDecSplit * LPR * D * static_cast<int>(sizeof(uint16_t));
-  cudaError_t e =
-      cudaFuncSetAttribute(decode_split_kernel<LPR, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+template <int HD>
+static cudaError_t launch_split(const DecodeParams& p, dim3 grid, cudaStream_t stream) {
+  const int smem = 2 * kDecSplit * HD * static_cast<int>(sizeof(uint16_t));
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  decode_split_kernel<LPR, D, G><<<grid, kDecThreads, smem, stream>>>(p);
+  decode_split_kernel<HD><<<grid, kDecThreads, smem, stream>>>(p);
   return cudaGetLastError();
-}
-
-// Lane groups of 16 for G <= 4 (16-byte slices of a row per lane), of 32
-// for larger groups (whose per-lane registers grow with G).
-template <int d>
-static cudaError_t launch_split(const DecodeParams& p, dim3 grid, int G, cudaStream_t stream) {
-  switch (G) {
-    case 1: return launch_split_g<16, d / 16, 1>(p, grid, stream);
-    case 2: return launch_split_g<16, d / 16, 2>(p, grid, stream);
-    case 4: return launch_split_g<16, d / 16, 4>(p, grid, stream);
-    case 8: return launch_split_g<32, d / 32, 8>(p, grid, stream);
-    default: return launch_split_g<32, d / 32, 16>(p, grid, stream);
-  }
 }
 
 cudaError_t launch_decode_attention(const DecodeParams& p, int batch, cudaStream_t stream) {
   dim3 grid(batch * p.n_kv_heads, p.n_split);
-  const int G = p.n_q_heads / p.n_kv_heads;
-  cudaError_t e = (p.head_dim == 128) ? launch_split<128>(p, grid, G, stream) : launch_split<64>(p, grid, G, stream);
+  cudaError_t e = (p.head_dim == 128) ? launch_split<128>(p, grid, stream) : launch_split<64>(p, grid, stream);
   if (e != cudaSuccess) return e;
   // The merge overlaps its launch with the split kernel's tail.
   cudaLaunchConfig_t cfg = {};
