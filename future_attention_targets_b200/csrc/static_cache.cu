@@ -17,8 +17,8 @@ namespace kvpop {
 
 // ------------------------------------------------------------------ compaction
 
-constexpr int kCompactThreads = 256;
-constexpr int kCompactUnroll = 16;     // 16-byte words each thread has in flight
+constexpr int kCompactThreads = 512;    // short per-thread mask runs: 32 positions at 16k
+constexpr int kCompactUnroll = 8;       // 16-byte words each thread has in flight (128 rows = one round)
 
 // Non-zero bytes of a 32-bit word: bit 7 of ((b & 0x7f) + 0x7f) | b is set
 // exactly when the byte b is non-zero, and the sum cannot carry into the next byte.
@@ -76,8 +76,8 @@ __device__ __forceinline__ int count_kept(const uint8_t* mask, int lo, int hi) {
   return n;
 }
 
-// Exclusive prefix sum over the block's 256 threads; *total gets the sum.
-__device__ __forceinline__ int block_exclusive_scan_256(int x, int* warp_sums, int* total) {
+// Exclusive prefix sum over the block's threads; *total gets the sum.
+__device__ __forceinline__ int block_exclusive_scan(int x, int* warp_sums, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int incl = x;
 #pragma unroll
@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_kv_kernel(const __
   const int c0 = min(L, tid * chunk), c1 = min(L, c0 + chunk);
   const int mine = count_kept(mask, c0, c1);
   int total = 0;
-  const int first = block_exclusive_scan_256(mine, warp_sums, &total);
+  const int first = block_exclusive_scan(mine, warp_sums, &total);
   if (first < S1 && first + mine > S0) {
     int slot = first;
     for_each_kept(mask, c0, c1, [&](int i) {
