@@ -274,8 +274,8 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
 
-    from future_attention_targets_b200 import (HostPipeline, check_status, future_target, keep_mask, lib,
-                                               row_lse)
+    from future_attention_targets_b200 import (HostPipeline, check_status, future_target, future_targets, keep_mask,
+                                               lib, row_lse)
     from future_attention_targets_b200.build import build
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -436,6 +436,35 @@ def run_ours(args):
             "frac_of_hbm": moved / (ms * 1e-3) / 1e9 / float(peaks_x["hbm_gbs"]),
             "launch": (f"{len(cu) - 1} x {w.n_kv_heads} x {-(-(int(max(np.diff(cu))) - S - W) // 1024)} CTAs of 1024 "
                        "threads, one per (sequence, KV head, block of 1024 steps)")}
+
+        # The hot path on the other two large workloads (the same kernels, other shapes).
+        for other in ("long_64k", "varlen_8x"):
+            do = make_inputs(other, seed=rank_seed(rank))
+            wo = do["workload"]
+            qo = torch.from_numpy(do["q_bits"].view(np.int16)).view(torch.bfloat16).to(dev)
+            ko = torch.from_numpy(do["k_bits"].view(np.int16)).view(torch.bfloat16).to(dev)
+            To = qo.shape[0]
+            lo_ = torch.empty((wo.n_q_heads, To), dtype=torch.float32, device=dev)
+            to_ = torch.empty((wo.n_kv_heads, To), dtype=torch.float32, device=dev)
+            ko_ = torch.empty((wo.n_kv_heads, To), dtype=torch.uint8, device=dev)
+            run_o = lambda: future_targets(qo, ko, do["cu_seqlens"], do["window"], do["sinks"], do["budgets"],
+                                           do["scale"], lse=lo_, target=to_, keep=ko_, status=status, stream=stream)
+            for _ in range(2):
+                run_o()
+            o0, o1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            n_o = 3
+            o0.record(stream)
+            for _ in range(n_o):
+                run_o()
+            o1.record(stream)
+            torch.cuda.synchronize(dev)
+            check_status(status, stream)
+            ms_o = o0.elapsed_time(o1) / n_o
+            flo = algorithmic_flops([int(x) for x in np.diff(do["cu_seqlens"])], wo.n_q_heads, wo.head_dim, wo.window)
+            extras[f"step_{other}"] = {"ms": ms_o, "value": flo["total"] / (ms_o * 1e-3) / 1e12, "unit": UNIT,
+                                       "pct_of_bf16_peak": 100.0 * flo["total"] / (ms_o * 1e-3) / 1e12 / peak,
+                                       "tokens": int(To), "sequences": int(len(do["cu_seqlens"]) - 1)}
+            del qo, ko, lo_, to_, ko_
 
         # Static cache: compact this step's keep set, then one decode step over it.
         from future_attention_targets_b200 import compact_kv, decode_attention
