@@ -275,7 +275,7 @@ def run_ours(args):
     import torch.distributed as dist
 
     from future_attention_targets_b200 import (HostPipeline, check_status, future_target, future_targets, keep_mask,
-                                               lib, row_lse)
+                                               lib, row_lse, target_workspace_bytes)
     from future_attention_targets_b200.build import build
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -303,6 +303,9 @@ def run_ours(args):
     keep = torch.empty((w.n_kv_heads, T), dtype=torch.uint8, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    # The transposed pass's normaliser rows (16 bytes per query head and token).
+    tws = torch.empty(target_workspace_bytes(T, w.n_q_heads, w.n_kv_heads, w.head_dim), dtype=torch.uint8,
+                      device=dev)
 
     def step(evs=None):
         if evs is not None:
@@ -310,7 +313,8 @@ def run_ours(args):
         row_lse(q, k, cu, scale, out=lse, status=status, stream=stream)
         if evs is not None:
             evs[1].record(stream)
-        future_target(q, k, cu, W, lse, scale, out=tgt, status=status, stream=stream)
+        # two launches: lse -> normaliser rows, then the transposed pass
+        future_target(q, k, cu, W, lse, scale, out=tgt, workspace=tws, status=status, stream=stream)
         if evs is not None:
             evs[2].record(stream)
         keep_mask(tgt, cu, W, S, budgets, out=keep, stream=stream)
@@ -447,8 +451,11 @@ def run_ours(args):
             lo_ = torch.empty((wo.n_q_heads, To), dtype=torch.float32, device=dev)
             to_ = torch.empty((wo.n_kv_heads, To), dtype=torch.float32, device=dev)
             ko_ = torch.empty((wo.n_kv_heads, To), dtype=torch.uint8, device=dev)
+            wso = torch.empty(target_workspace_bytes(To, wo.n_q_heads, wo.n_kv_heads, wo.head_dim), dtype=torch.uint8,
+                              device=dev)
             run_o = lambda: future_targets(qo, ko, do["cu_seqlens"], do["window"], do["sinks"], do["budgets"],
-                                           do["scale"], lse=lo_, target=to_, keep=ko_, status=status, stream=stream)
+                                           do["scale"], lse=lo_, target=to_, keep=ko_, workspace=wso, status=status,
+                                           stream=stream)
             for _ in range(2):
                 run_o()
             o0, o1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -548,7 +555,7 @@ def run_ours(args):
                          "algorithmic_flops_per_launch": dom_flops},
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": 4 * args.steps,
             "next_rows": extras,
             "clocks": clocks.summary(),
         }

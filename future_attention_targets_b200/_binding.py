@@ -43,7 +43,9 @@ _P = ctypes.c_void_p
 _I32P = ctypes.POINTER(ctypes.c_int32)
 _SIGS = {
     "kvpop_row_lse": (ctypes.c_int, [_P, _P, _I32P, Shape, ctypes.c_float, _P, _P, _P]),
-    "kvpop_future_target": (ctypes.c_int, [_P, _P, _I32P, Shape, ctypes.c_float, ctypes.c_int32, _P, _P, _P, _P]),
+    "kvpop_target_workspace_bytes": (ctypes.c_size_t, [Shape]),
+    "kvpop_future_target": (ctypes.c_int, [_P, _P, _I32P, Shape, ctypes.c_float, ctypes.c_int32, _P, _P, _P,
+                                           ctypes.c_size_t, _P, _P]),
     "kvpop_keep_mask": (ctypes.c_int, [_P, _I32P, Shape, ctypes.c_int32, ctypes.c_int32, _I32P, _P, _P]),
     "kvpop_prefix_topk_thresholds": (ctypes.c_int, [_P, _I32P, Shape, ctypes.c_int32, ctypes.c_int32, _I32P, _P,
                                                     _P, _P]),
@@ -53,7 +55,7 @@ _SIGS = {
                                               _P]),
     "kvpop_decode_attention_noalloc": (ctypes.c_int, [_P, _P, _P, _P, CacheShape, ctypes.c_float, _P, _P, _P]),
     "kvpop_future_targets": (ctypes.c_int, [_P, _P, _I32P, Shape, ctypes.c_float, ctypes.c_int32, ctypes.c_int32,
-                                            _I32P, _P, _P, _P, _P, _P]),
+                                            _I32P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
     "kvpop_target_split_workspace_bytes": (ctypes.c_size_t, [Shape]),
     "kvpop_future_target_split": (ctypes.c_int, [_P, _P, _I32P, Shape, ctypes.c_float, ctypes.c_int32, _P, _P, _P,
                                                  ctypes.c_size_t, _P, _P]),
@@ -164,8 +166,16 @@ def row_lse(q, k, cu_seqlens, scale: float | None = None, out=None, status=None,
     return out
 
 
-def future_target(q, k, cu_seqlens, window: int, lse, scale: float | None = None, out=None, status=None,
-                  stream=None):
+def _workspace(nbytes: int, device, workspace):
+    """The caller's workspace if given, else a fresh uint8 CUDA tensor of nbytes (at least 256)."""
+    import torch
+    if workspace is not None:
+        return workspace
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def future_target(q, k, cu_seqlens, window: int, lse, scale: float | None = None, out=None, workspace=None,
+                  status=None, stream=None):
     """target [H_kv, T] fp32: mass each key receives from queries i >= j + W, summed over its GQA group."""
     import torch
     _check_qk(q, k)
@@ -176,8 +186,10 @@ def future_target(q, k, cu_seqlens, window: int, lse, scale: float | None = None
         raise ValueError("lse must be a fp32 CUDA tensor [H_q, T]")
     if out is None:
         out = torch.empty((sh.n_kv_heads, sh.total_tokens), dtype=torch.float32, device=q.device)
+    workspace = _workspace(lib().kvpop_target_workspace_bytes(sh), q.device, workspace)
     _check(lib().kvpop_future_target(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, int(window),
-                                     lse.contiguous().data_ptr(), out.data_ptr(), _ptr(status), _stream_ptr(stream)))
+                                     lse.contiguous().data_ptr(), out.data_ptr(), workspace.data_ptr(),
+                                     workspace.numel(), _ptr(status), _stream_ptr(stream)))
     return out
 
 
@@ -193,13 +205,16 @@ def future_target_split(q, k, cu_seqlens, window: int, lse, scale: float | None 
         raise ValueError("lse must be a fp32 CUDA tensor [H_q, T]")
     if out is None:
         out = torch.empty((sh.n_kv_heads, sh.total_tokens), dtype=torch.float32, device=q.device)
-    if workspace is None:
-        workspace = torch.empty(max(int(lib().kvpop_target_split_workspace_bytes(sh)), 16), dtype=torch.uint8,
-                                device=q.device)
+    workspace = _workspace(lib().kvpop_target_split_workspace_bytes(sh), q.device, workspace)
     _check(lib().kvpop_future_target_split(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, int(window),
                                            lse.contiguous().data_ptr(), out.data_ptr(), workspace.data_ptr(),
                                            workspace.numel(), _ptr(status), _stream_ptr(stream)))
     return out
+
+
+def target_workspace_bytes(total_tokens: int, n_q_heads: int, n_kv_heads: int, head_dim: int) -> int:
+    """Device workspace of future_target and future_targets (the transposed pass's normaliser rows)."""
+    return int(lib().kvpop_target_workspace_bytes(Shape(1, total_tokens, n_q_heads, n_kv_heads, head_dim)))
 
 
 def target_split_workspace_bytes(total_tokens: int, n_q_heads: int, n_kv_heads: int, head_dim: int) -> int:
@@ -295,7 +310,7 @@ def decode_attention(q, k_cache, v_cache, count, scale: float | None = None, out
 
 
 def future_targets(q, k, cu_seqlens, window: int, sinks: int, budgets, scale: float | None = None,
-                   lse=None, target=None, keep=None, status=None, stream=None):
+                   lse=None, target=None, keep=None, workspace=None, status=None, stream=None):
     """The whole hot path on device tensors: returns (lse, target, keep)."""
     import torch
     _check_qk(q, k)
@@ -310,14 +325,16 @@ def future_targets(q, k, cu_seqlens, window: int, sinks: int, budgets, scale: fl
     if keep is None:
         keep = torch.empty((sh.n_kv_heads, sh.total_tokens), dtype=torch.uint8, device=dev)
     bud = _i32_host(budgets)
+    workspace = _workspace(lib().kvpop_target_workspace_bytes(sh), dev, workspace)
     _check(lib().kvpop_future_targets(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, int(window), int(sinks), bud,
-                                      lse.data_ptr(), target.data_ptr(), keep.data_ptr(), _ptr(status),
-                                      _stream_ptr(stream)))
+                                      lse.data_ptr(), target.data_ptr(), keep.data_ptr(), workspace.data_ptr(),
+                                      workspace.numel(), _ptr(status), _stream_ptr(stream)))
     return lse, target, keep
 
 
 def fused_workspace(cu_seqlens, n_q_heads: int, n_kv_heads: int, head_dim: int, device=None):
-    """Zero-filled flag workspace for future_targets_fused (reusable: each completed call leaves it zeroed)."""
+    """Zero-filled workspace for future_targets_fused: the flag counters (each completed call leaves them
+    zeroed, so the workspace is reusable), then the normaliser rows (scratch)."""
     import torch
     cu, cu_c = _cu_host(cu_seqlens)
     sh = Shape(len(cu) - 1, int(cu[-1]), n_q_heads, n_kv_heads, head_dim)

@@ -53,11 +53,15 @@ constexpr int kGroupCols = kStreamRows / kColGroups;   // accumulator columns pe
 constexpr int kSoftmaxWarps = 4 * kColGroups;          // one warp per TMEM lane quadrant per group
 static_assert(kThreads == 32 * (2 + kSoftmaxWarps), "producer warp + MMA warp + softmax warps");
 static_assert(kGroupCols == 64, "group_exp_sum walks four 16-column chunks");
-// Extra K=16 slab (no swizzle, K-major): 8-row groups of two 8x16-byte core
-// matrices; element (r, e) sits at (r/8)*256 + (e/8)*128 + (r%8)*16 + (e%8)*2.
-constexpr int kSlabLBO = 128;   // between the two core matrices along K
-constexpr int kSlabSBO = 256;   // between 8-row groups
-constexpr float kPastEnd = 1e30f;  // normaliser of query columns past the sequence: exp2 -> 0
+// Extra K=16 slabs (no swizzle, K-major) that subtract lse_i / s from every
+// pass-2 score.  A (ones, 128 rows): 8-row groups of two 8x16-byte core
+// matrices, element (r, e) at (r/8)*256 + (e/8)*128 + (r%8)*16 + (e%8)*2.
+// B (normaliser rows, 256 rows): row r's 16 bytes (e = 0..7) at r * 16, so
+// that one bulk copy of consecutive rows fills it; the e = 8..15 half is a
+// zero block kSlabRowBytes further on.
+constexpr int kSlabLBO = 128;   // A: between the two core matrices along K
+constexpr int kSlabSBO = 256;   // A: between 8-row groups
+constexpr int kSlabRowBytes = kStreamRows * 16;   // B: rows of one tile; also its LBO
 
 template <int HD, bool kSlab>
 struct SmemLayout {
@@ -116,6 +120,12 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Orders this thread's generic-proxy view of global memory with its later
+// (or, on the writing side, earlier) async-proxy bulk copies.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // Descriptor of a K=16 slab in the no-swizzle K-major layout above.
 __device__ __forceinline__ uint64_t umma_desc_slab(uint32_t saddr) {
   uint64_t d = 0;
@@ -126,7 +136,36 @@ __device__ __forceinline__ uint64_t umma_desc_slab(uint32_t saddr) {
   return d;
 }
 
+// Descriptor of the B normaliser slab (LBO kSlabRowBytes, SBO one 8-row group).
+__device__ __forceinline__ uint64_t umma_desc_slab_rows(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(kSlabRowBytes >> 4) << 16;
+  d |= static_cast<uint64_t>(128 >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  return d;
+}
+
 __device__ __forceinline__ uint32_t slab_row_offset(int r) { return (r >> 3) * kSlabSBO + (r & 7) * 16; }
+
+// Normaliser row of one query row: (-hi, -mid, -lo, 0, 0, 0, 0, 0) in bf16
+// with hi + mid + lo = lse * inv_scale (each part the bf16 rounding of what
+// the parts before it leave), so that (1, 1, 1) . row = -lse / s to within
+// fp32 rounding of the three-term sum.
+__device__ __forceinline__ uint4 norm_row(float lse, float inv_scale) {
+  const float x = lse * inv_scale;
+  const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+  const float r1 = x - __bfloat162float(hi);
+  const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+  uint4 v;
+  v.x = static_cast<uint32_t>(__bfloat16_as_ushort(__hneg(hi))) |
+        (static_cast<uint32_t>(__bfloat16_as_ushort(__hneg(mid))) << 16);
+  v.y = static_cast<uint32_t>(__bfloat16_as_ushort(__hneg(lo)));
+  v.z = 0u;
+  v.w = 0u;
+  return v;
+}
 
 // ------------------------------------------------------------------ policies
 
@@ -226,37 +265,6 @@ struct TargetPass {
   static __device__ __forceinline__ bool half_tile(const Item&, int32_t) { return false; }
 };
 
-// Walks this CTA's pass-2 tiles in issue order (items without tiles skipped).
-struct TileCursor {
-  int32_t k;
-  TargetPass::Item it;
-  int32_t g, qt;
-  bool have;
-  __device__ __forceinline__ void next_item(const AttnParams& p, const LevelSchedule& sched) {
-    have = false;
-    for (;;) {
-      const int32_t n = cta_item(k++, blockIdx.x, gridDim.x);
-      if (n >= sched.total_items) return;
-      it = TargetPass::item(p, sched, n);
-      if (it.ntiles > 0) {
-        g = 0;
-        qt = 0;
-        have = true;
-        return;
-      }
-    }
-  }
-  __device__ __forceinline__ void start(const AttnParams& p, const LevelSchedule& sched) {
-    k = 0;
-    next_item(p, sched);
-  }
-  __device__ __forceinline__ void advance(const AttnParams& p, const LevelSchedule& sched) {
-    if (++qt == it.nq) {
-      qt = 0;
-      if (++g == it.ng) next_item(p, sched);
-    }
-  }
-};
 
 // Pipeline counters of each role, carried from one phase to the next.
 struct ProducerState {
@@ -288,38 +296,43 @@ __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity, const
   return wait_bounded(bar, parity, c2, SITE_TEARDOWN);
 }
 
-// Single launch: waits until every 128-row lse tile under the cursor's 256
-// query rows has been published.  Lanes 0..2 poll the (at most three) tile
-// flags and lane 31 the count of softmax warps that finished pass 1, all in
-// one round trip; once every CTA's pass 1 is done (*all_lse) no flag is read
-// again.  Bounded like every other wait; warp-uniform result.
+// Single launch: waits until every 128-row lse tile under query rows
+// [a, a + 256) of query head qh (a = i0 + qt * 256) has been published.
+// Lanes 0..2 poll the (at most three) tile flags and lane 31 the count of
+// softmax warps that finished pass 1, all in one round trip; once every CTA's
+// pass 1 is done (*all_lse) no flag is read again.  Bounded like every other
+// wait; warp-uniform result.  The warp barrier on success passes every
+// lane's acquire on to the whole warp.
 template <bool kFused>
-__device__ __forceinline__ bool norm_ready(const AttnParams& p, const Phase& ph, const TileCursor& cur, int lane,
-                                           const WaitCtl& ctl, bool& all_lse) {
+__device__ __forceinline__ bool norm_ready(const AttnParams& p, const Phase& ph, const TargetPass::Item& it,
+                                           int32_t qh, int32_t qt, int lane, const WaitCtl& ctl, bool& all_lse) {
   if constexpr (!kFused) {
     return true;
   } else {
     if (all_lse) return true;
-    const int32_t qh = cur.it.h * p.group + cur.it.g0 + cur.g;
-    const int32_t a = cur.it.i0 + cur.qt * kStreamRows;
-    const int32_t b = min(a + kStreamRows, cur.it.L);
+    const int32_t a = it.i0 + qt * kStreamRows;
+    const int32_t b = min(a + kStreamRows, it.L);
     const int32_t t0 = a / kTileRows, nt = (b - 1) / kTileRows - t0 + 1;
-    const int32_t* f = ph.flags + static_cast<int64_t>(qh) * ph.n_flag_tiles + ph.tile_base[cur.it.seq] + t0;
+    const int32_t* f = ph.flags + static_cast<int64_t>(qh) * ph.n_flag_tiles + ph.tile_base[it.seq] + t0;
     const int32_t all_warps = kSoftmaxWarps * static_cast<int32_t>(gridDim.x);
     uint64_t t_start = 0;
-    for (uint32_t it = 0;; ++it) {
+    for (uint32_t k = 0;; ++k) {
       bool mine = true;
       if (lane < nt) mine = flag_acquire_load(f + lane) >= kLseFlagWriters;
       const bool done_all = (lane == 31) && flag_acquire_load(ph.lse_done) >= all_warps;
       if (__any_sync(0xffffffffu, done_all)) {
         all_lse = true;
+        __syncwarp();
         return true;
       }
-      if (__all_sync(0xffffffffu, mine)) return true;
+      if (__all_sync(0xffffffffu, mine)) {
+        __syncwarp();
+        return true;
+      }
       int give_up = 0;
-      if (lane == 0 && (it & 15u) == 0u) {
+      if (lane == 0 && (k & 15u) == 0u) {
         const uint64_t now = global_timer_ns();
-        if (it == 0) t_start = now;
+        if (k == 0) t_start = now;
         if (*ctl.abort_flag) {
           give_up = 1;
         } else if (now - t_start > ctl.limit_ns) {
@@ -334,44 +347,12 @@ __device__ __forceinline__ bool norm_ready(const AttnParams& p, const Phase& ph,
   }
 }
 
-// Normaliser rows of one pass-2 B tile, this lane's 8 rows (lane + 32 m):
-// lse_i / s, or kPastEnd past the sequence end.  In the single launch the
-// lse rows were written by other CTAs during this launch, so they are read
-// through L2 (ld.global.cg), never from a possibly stale L1 line.
-template <bool kFused>
-__device__ __forceinline__ void load_norm_rows(const AttnParams& p, const TileCursor& cur, int lane,
-                                               float (&v)[8]) {
-  const int32_t qh = cur.it.h * p.group + cur.it.g0 + cur.g;
-  const float* src = p.lse_in + static_cast<int64_t>(qh) * p.total_tokens + cur.it.s;
-#pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    const int32_t i = cur.it.i0 + cur.qt * kStreamRows + lane + 32 * m;
-    const float x = (i < cur.it.L) ? (kFused ? __ldcg(src + i) : __ldg(src + i)) : 0.f;
-    v[m] = (i < cur.it.L) ? x * p.inv_scale : kPastEnd;
-  }
-}
-
-// Writes (-hi, -mid, -lo, 0) with hi + mid + lo = v (three bf16 parts) into
-// the slab rows of this lane.
-__device__ __forceinline__ void store_norm_rows(uint8_t* slab, int lane, const float (&v)[8]) {
-#pragma unroll
-  for (int m = 0; m < 8; ++m) {
-    const float x = v[m];
-    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-    const float r1 = x - __bfloat162float(hi);
-    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
-    const uint32_t w0 = static_cast<uint32_t>(__bfloat16_as_ushort(__hneg(hi))) |
-                        (static_cast<uint32_t>(__bfloat16_as_ushort(__hneg(mid))) << 16);
-    const uint32_t w1 = static_cast<uint32_t>(__bfloat16_as_ushort(__hneg(lo)));
-    const uint32_t addr = smem_u32(slab + slab_row_offset(lane + 32 * m));
-    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(w0), "r"(w1) : "memory");
-  }
-}
-
-// One pass of the TMA producer warp.  kFused: the single launch, whose B
-// stages complete with 32 lane arrivals in both passes (pass 2 needs them
-// for the slab rows) and whose pass-2 normalisers wait for their lse flags.
+// One pass of the TMA producer warp.  Pass 2 also copies, per B stage, the
+// 256 normaliser rows of its query tile (p.nrm_rows, 16 bytes per row, one
+// bulk copy that stops at row T; columns past the sequence end are masked by
+// the softmax).  kFused: the single launch, whose normaliser rows are written
+// by pass 1 during the launch; the query tile is requested first, the rows
+// only once their lse flags are set.
 template <class Pass, int HD, bool kFused>
 __device__ void producer_phase(const AttnParams& p, const Phase& ph, uint8_t* smem, const Bars& bars,
                                const WaitCtl& ctl, ProducerState& st) {
@@ -379,20 +360,7 @@ __device__ void producer_phase(const AttnParams& p, const Phase& ph, uint8_t* sm
   const int lane = threadIdx.x & 31;
   const LevelSchedule& sched = *ph.sched;
   const int32_t total = sched.total_items;
-  // Pass 2: normaliser values of the next tile, loaded one tile ahead.
-  TileCursor nxt;
-  float norm[8];
   bool all_lse = false;
-  if constexpr (Pass::kSlab) {
-    nxt.start(p, sched);
-    if (nxt.have) {
-      if (!norm_ready<kFused>(p, ph, nxt, lane, ctl, all_lse)) {
-        st.ok = false;
-        return;
-      }
-      load_norm_rows<kFused>(p, nxt, lane, norm);
-    }
-  }
   for (int32_t k = 0; st.ok; ++k) {
     const int32_t n = cta_item(k, blockIdx.x, gridDim.x);
     if (n >= total) break;
@@ -416,38 +384,28 @@ __device__ void producer_phase(const AttnParams& p, const Phase& ph, uint8_t* sm
       }
       uint8_t* stage = smem + L::OFF_B + sg * L::B_STAGE;
       if constexpr (Pass::kSlab) {
-        // Tile bytes are expected before the loads are issued; the 32 lane
-        // arrivals below (after their slab rows are written) complete the phase.
         const int32_t g = t / it.nq, qt = t - g * it.nq;
+        const int32_t qh = it.h * p.group + it.g0 + g;
+        const int32_t row0 = it.s + it.i0 + qt * kStreamRows;   // < T: qt < nq
+        const uint32_t rows_bytes = static_cast<uint32_t>(min(kStreamRows, p.total_tokens - row0)) * 16u;
         if (lane == 0) {
-          mbar_expect_tx(&bars.b_full[sg], L::B_TILE);
-          Pass::template load_b<HD>(ph, it, it.h * p.group + it.g0 + g, qt, stage, &bars.b_full[sg]);
+          mbar_arrive_expect_tx(&bars.b_full[sg], L::B_TILE + rows_bytes);
+          Pass::template load_b<HD>(ph, it, qh, qt, stage, &bars.b_full[sg]);
         }
-        float cur[8];
-#pragma unroll
-        for (int m = 0; m < 8; ++m) cur[m] = norm[m];
-        nxt.advance(p, sched);
-        bool ready = true;
-        if (nxt.have) {
-          ready = norm_ready<kFused>(p, ph, nxt, lane, ctl, all_lse);
-          if (ready) load_norm_rows<kFused>(p, nxt, lane, norm);
+        // After a failed wait the rows are still copied (in bounds, unused)
+        // so that the stage completes and the drain below ends.
+        const bool ready = norm_ready<kFused>(p, ph, it, qh, qt, lane, ctl, all_lse);
+        if (lane == 0) {
+          if constexpr (kFused) fence_proxy_async_global();
+          bulk_load_1d(stage + L::B_TILE,
+                       static_cast<const uint8_t*>(p.nrm_rows) + (static_cast<int64_t>(qh) * p.total_tokens + row0) * 16,
+                       rows_bytes, &bars.b_full[sg]);
         }
-        store_norm_rows(stage + L::B_TILE, lane, cur);
-        fence_proxy_async_smem();
-        mbar_arrive(&bars.b_full[sg]);
         ++st.b_cnt;
         if (!ready) {
           st.ok = false;
           break;
         }
-      } else if constexpr (kFused) {
-        if (lane == 0) {
-          mbar_expect_tx(&bars.b_full[sg], L::B_TILE);
-          Pass::template load_b<HD>(ph, it, t, stage, &bars.b_full[sg]);
-        }
-        __syncwarp();
-        mbar_arrive(&bars.b_full[sg]);
-        ++st.b_cnt;
       } else {
         if (lane == 0) {
           mbar_arrive_expect_tx(&bars.b_full[sg], L::B_TILE);
@@ -513,7 +471,7 @@ __device__ void mma_phase(const AttnParams& p, const Phase& ph, uint8_t* smem, c
       }
       if constexpr (Pass::kSlab) {
         // acc += (1, 1, 1) . (-hi, -mid, -lo): subtract lse_i / s from every column.
-        umma_bf16(d_tmem, umma_desc_slab(smem_u32(smem + L::OFF_ASLAB)), umma_desc_slab(b_addr + L::B_TILE),
+        umma_bf16(d_tmem, umma_desc_slab(smem_u32(smem + L::OFF_ASLAB)), umma_desc_slab_rows(b_addr + L::B_TILE),
                   idesc, 1u);
       }
       st.issued = true;
@@ -839,10 +797,17 @@ __device__ void lse_softmax_phase(const AttnParams& p, const Phase& ph, uint8_t*
 #pragma unroll
       for (int g = 0; g < kColGroups; ++g) s += (offs[g] > -INFINITY) ? sums[g] * ex2_approx(offs[g] - m) : 0.f;
       const int32_t i = it.i0 + row;
-      if (i < it.L) ph.out[static_cast<int64_t>(it.g) * p.total_tokens + it.s + i] = (m + log2f(s)) * kLn2;
+      if (i < it.L) {
+        const float lse = (m + log2f(s)) * kLn2;
+        const int64_t at = static_cast<int64_t>(it.g) * p.total_tokens + it.s + i;
+        ph.out[at] = lse;
+        if (p.nrm_rows != nullptr) static_cast<uint4*>(p.nrm_rows)[at] = norm_row(lse, p.inv_scale);
+      }
       if constexpr (kFused) {
-        // Publish this warp's 32 rows: the warp barrier orders every lane's
-        // store before lane 0's gpu-scope release.
+        // Publish this warp's 32 rows: the proxy fence and the warp barrier
+        // order every lane's stores (read by other CTAs' bulk copies) before
+        // lane 0's gpu-scope release.
+        fence_proxy_async_global();
         __syncwarp();
         if (lane == 0)
           flag_release_add(ph.flags + static_cast<int64_t>(it.g) * ph.n_flag_tiles + ph.tile_base[it.seq] +
@@ -894,14 +859,15 @@ __device__ void target_softmax_phase(const AttnParams& p, const Phase& ph, uint8
         const uint32_t taddr = lane_addr + acc * kStreamRows;
         // First query tile: query column m is valid iff m >= row, which can
         // mask columns of the groups below column 128 (per-lane bound lo).
-        // Last query tile: columns past the sequence hold -1e30 (exp2 -> 0 on
-        // MUFU).  The path is chosen per warp: its TMEM loads are
-        // warp-collective.
+        // Last query tile: columns past the sequence end (their normaliser
+        // rows belong to another sequence, or are stale) are cut by hi.  The
+        // path is chosen per warp: its TMEM loads are warp-collective.
         const bool diag = (qt == 0) && (c0 < kTileRows);
         const bool ragged = (qt == it.nq - 1) && ragged_end;
         const int lo = diag ? max(0, row - c0) : 0;
+        const int hi = ragged ? min(kGroupCols, it.L - it.i0 - qt * kStreamRows - c0) : kGroupCols;
         const float ts = (diag || ragged)
-                             ? group_exp_sum<true, 0>(taddr, c2, zero2, lo, kGroupCols)
+                             ? group_exp_sum<true, 0>(taddr, c2, zero2, lo, hi)
                              : group_exp_sum<false, KVPOP_POLY16_TARGET, true>(taddr, c2, zero2, 0, kGroupCols,
                                                                                   xmin);
         tc_fence_before_sync();
@@ -984,7 +950,7 @@ __device__ __forceinline__ void cta_setup(uint8_t* smem, const Bars& bars, uint3
       mbar_init(&bars.acc_empty[i], kSoftmaxWarps);
     }
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&bars.b_full[i], kSlab ? 32 : 1);
+      mbar_init(&bars.b_full[i], 1);
       mbar_init(&bars.b_empty[i], 1);
     }
     mbar_init(bars.comb_full, 4 * (kColGroups - 1));
@@ -1190,6 +1156,22 @@ cudaError_t launch_merge_partials(const float* part, float* target, int group, i
 }
 
 int target_split_groups() { return kColGroups; }
+
+// Normaliser rows [H_q, T] of pass 2 from a given lse [H_q, T] (the
+// standalone pass; the pipelines have pass 1 write them next to lse).
+__global__ void __launch_bounds__(256) norm_rows_kernel(const float* __restrict__ lse, uint4* __restrict__ rows,
+                                                        int64_t n, float inv_scale) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    rows[i] = norm_row(__ldg(lse + i), inv_scale);
+}
+
+cudaError_t launch_norm_rows(const float* lse, void* rows, int64_t n, float inv_scale, int sm_count,
+                             cudaStream_t stream) {
+  const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, static_cast<int64_t>(sm_count) * 8));
+  norm_rows_kernel<<<std::max(blocks, 1), 256, 0, stream>>>(lse, static_cast<uint4*>(rows), n, inv_scale);
+  return cudaGetLastError();
+}
 
 // ------------------------------------------------------------------ bounded-wait self-test
 

@@ -27,6 +27,8 @@ cudaError_t launch_fused_targets(const FusedParams& fp, int head_dim, int grid, 
 cudaError_t launch_merge_partials(const float* part, float* target, int group, int n_kv_heads, int total_tokens,
                                   int sm_count, cudaStream_t stream);
 int target_split_groups();
+cudaError_t launch_norm_rows(const float* lse, void* rows, int64_t n, float inv_scale, int sm_count,
+                             cudaStream_t stream);
 size_t decode_scratch_bytes();
 cudaError_t decode_scratch_address(float** out);
 }  // namespace kvpop
@@ -308,6 +310,63 @@ const char* kvpop_status_string(kvpop_status s) {
   return "unknown status";
 }
 
+// Bytes of the normaliser rows that the transposed pass streams beside its
+// query tiles: 16 per (query head, token).
+static size_t norm_rows_bytes(const kvpop_shape& shape) {
+  return static_cast<size_t>(shape.n_q_heads) * static_cast<size_t>(shape.total_tokens) * 16;
+}
+
+// Pass 1 on validated device arguments; rows (nullable) also receives the
+// normaliser rows of pass 2.
+static kvpop_status run_row_lse(const void* q, const void* k, const int32_t* cu_seqlens, const kvpop_shape& shape,
+                                float scale, float* lse, void* rows, int32_t* dev_status, cudaStream_t stream,
+                                const DeviceInfo& dev) {
+  AttnParams p;
+  kvpop_status st;
+  if ((st = fill_attn_common(&p, q, k, cu_seqlens, shape, scale, false)) != KVPOP_OK) return st;
+  p.out = lse;
+  p.nrm_rows = rows;
+  p.status = dev_status;
+  if (p.sched.total_items == 0) return KVPOP_OK;
+  cudaError_t e = launch_row_lse(p, shape.head_dim, grid_for(p.sched.total_items, dev.sm_count), stream);
+  return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "row_lse launch");
+}
+
+// Pass 2 on validated device arguments, from normaliser rows.  partials
+// non-null: one item per (key tile, query head), then the ordered merge.
+static kvpop_status run_target(const void* q, const void* k, const int32_t* cu_seqlens, const kvpop_shape& shape,
+                               float scale, int32_t window, const void* rows, float* target, float* partials,
+                               int32_t* dev_status, cudaStream_t stream, const DeviceInfo& dev) {
+  AttnParams p;
+  kvpop_status st;
+  if ((st = fill_attn_common(&p, q, k, cu_seqlens, shape, scale, true)) != KVPOP_OK) return st;
+  const int G = shape.n_q_heads / shape.n_kv_heads;
+  if (partials != nullptr) {
+    build_schedule(cu_seqlens, shape.batch, shape.n_kv_heads * G, &p.sched);
+    p.g_split = G;
+  }
+  // A window longer than any sequence leaves every target at zero; clamp it
+  // so the tile arithmetic stays in range.
+  p.window = std::min<int32_t>(window, kMaxLevels * kTileRows + 1);
+  p.nrm_rows = const_cast<void*>(rows);
+  p.out = partials != nullptr ? partials : target;
+  p.status = dev_status;
+  if (p.sched.total_items == 0) return KVPOP_OK;
+  cudaError_t e = launch_future_target(p, shape.head_dim, grid_for(p.sched.total_items, dev.sm_count), stream);
+  if (e != cudaSuccess) return cuda_fail(e, "future_target launch");
+  if (partials == nullptr) return KVPOP_OK;
+  e = launch_merge_partials(partials, target, G, shape.n_kv_heads, shape.total_tokens, dev.sm_count, stream);
+  return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "merge of the split partials");
+}
+
+static kvpop_status check_workspace(const void* ws, size_t bytes, size_t need, size_t align) {
+  if (ws == nullptr || bytes < need)
+    return fail(KVPOP_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu required", bytes, need);
+  if ((reinterpret_cast<uintptr_t>(ws) & (align - 1)) != 0)
+    return fail(KVPOP_ERR_INVALID_ARG, "workspace must be %zu-byte aligned", align);
+  return KVPOP_OK;
+}
+
 kvpop_status kvpop_row_lse(const void* q, const void* k, const int32_t* cu_seqlens, kvpop_shape shape, float scale,
                            float* lse, int32_t* dev_status, void* stream) {
   kvpop_status st;
@@ -317,83 +376,68 @@ kvpop_status kvpop_row_lse(const void* q, const void* k, const int32_t* cu_seqle
   if (shape.total_tokens == 0) return KVPOP_OK;
   DeviceInfo dev;
   if ((st = device_info(&dev)) != KVPOP_OK) return st;
-  AttnParams p;
-  if ((st = fill_attn_common(&p, q, k, cu_seqlens, shape, scale, false)) != KVPOP_OK) return st;
-  p.out = lse;
-  p.status = dev_status;
-  if (p.sched.total_items == 0) return KVPOP_OK;
-  cudaError_t e = launch_row_lse(p, shape.head_dim, grid_for(p.sched.total_items, dev.sm_count),
-                                 static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "row_lse launch");
+  return run_row_lse(q, k, cu_seqlens, shape, scale, lse, nullptr, dev_status, static_cast<cudaStream_t>(stream),
+                     dev);
+}
+
+size_t kvpop_target_workspace_bytes(kvpop_shape shape) {
+  if (shape.total_tokens <= 0 || shape.n_q_heads <= 0) return 0;
+  return align256(norm_rows_bytes(shape));
 }
 
 kvpop_status kvpop_future_target(const void* q, const void* k, const int32_t* cu_seqlens, kvpop_shape shape,
-                                 float scale, int32_t window, const float* lse, float* target,
-                                 int32_t* dev_status, void* stream) {
+                                 float scale, int32_t window, const float* lse, float* target, void* workspace,
+                                 size_t workspace_bytes, int32_t* dev_status, void* stream) {
   kvpop_status st;
   if ((st = check_qk(q, k, scale)) != KVPOP_OK) return st;
   if (lse == nullptr || target == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "lse or target is NULL");
   if (window < 0) return fail(KVPOP_ERR_INVALID_ARG, "window must be >= 0 (got %d)", window);
   if ((st = check_shape(cu_seqlens, shape, true)) != KVPOP_OK) return st;
   if (shape.total_tokens == 0) return KVPOP_OK;
+  if ((st = check_workspace(workspace, workspace_bytes, kvpop_target_workspace_bytes(shape), 16)) != KVPOP_OK)
+    return st;
   DeviceInfo dev;
   if ((st = device_info(&dev)) != KVPOP_OK) return st;
-  AttnParams p;
-  if ((st = fill_attn_common(&p, q, k, cu_seqlens, shape, scale, true)) != KVPOP_OK) return st;
-  // A window longer than any sequence leaves every target at zero; clamp it
-  // so the tile arithmetic stays in range.
-  p.window = std::min<int32_t>(window, kMaxLevels * kTileRows + 1);
-  p.lse_in = lse;
-  p.out = target;
-  p.status = dev_status;
-  if (p.sched.total_items == 0) return KVPOP_OK;
-  cudaError_t e = launch_future_target(p, shape.head_dim, grid_for(p.sched.total_items, dev.sm_count),
-                                       static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "future_target launch");
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const float inv_scale = static_cast<float>(1.0 / static_cast<double>(scale));
+  cudaError_t e = launch_norm_rows(lse, workspace, static_cast<int64_t>(shape.n_q_heads) * shape.total_tokens,
+                                   inv_scale, dev.sm_count, s);
+  if (e != cudaSuccess) return cuda_fail(e, "normaliser rows launch");
+  return run_target(q, k, cu_seqlens, shape, scale, window, workspace, target, nullptr, dev_status, s, dev);
 }
 
 size_t kvpop_target_split_workspace_bytes(kvpop_shape shape) {
   if (shape.total_tokens <= 0 || shape.n_kv_heads <= 0 || shape.n_q_heads <= 0 ||
       shape.n_q_heads % shape.n_kv_heads != 0)
     return 0;
-  return static_cast<size_t>(shape.n_q_heads) * target_split_groups() * static_cast<size_t>(shape.total_tokens) *
-         sizeof(float);
+  return kvpop_target_workspace_bytes(shape) + static_cast<size_t>(shape.n_q_heads) * target_split_groups() *
+                                                   static_cast<size_t>(shape.total_tokens) * sizeof(float);
 }
 
 kvpop_status kvpop_future_target_split(const void* q, const void* k, const int32_t* cu_seqlens, kvpop_shape shape,
-                                       float scale, int32_t window, const float* lse, float* target, float* partials,
-                                       size_t partials_bytes, int32_t* dev_status, void* stream) {
+                                       float scale, int32_t window, const float* lse, float* target, void* workspace,
+                                       size_t workspace_bytes, int32_t* dev_status, void* stream) {
   kvpop_status st;
   if ((st = check_qk(q, k, scale)) != KVPOP_OK) return st;
   if (lse == nullptr || target == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "lse or target is NULL");
   if (window < 0) return fail(KVPOP_ERR_INVALID_ARG, "window must be >= 0 (got %d)", window);
   if ((st = check_shape(cu_seqlens, shape, true)) != KVPOP_OK) return st;
+  if (shape.total_tokens == 0) return KVPOP_OK;
+  if ((st = check_workspace(workspace, workspace_bytes, kvpop_target_split_workspace_bytes(shape), 16)) != KVPOP_OK)
+    return st;
   const int G = shape.n_q_heads / shape.n_kv_heads;
   if (G == 1)   // one query head per KV head: the split is the plain pass
-    return kvpop_future_target(q, k, cu_seqlens, shape, scale, window, lse, target, dev_status, stream);
-  const size_t need = kvpop_target_split_workspace_bytes(shape);
-  if (partials == nullptr || partials_bytes < need)
-    return fail(KVPOP_ERR_INVALID_ARG, "partials workspace of %zu bytes is smaller than the %zu required",
-                partials_bytes, need);
-  if ((reinterpret_cast<uintptr_t>(partials) & 15u) != 0)
-    return fail(KVPOP_ERR_INVALID_ARG, "partials must be 16-byte aligned");
-  if (shape.total_tokens == 0) return KVPOP_OK;
+    return kvpop_future_target(q, k, cu_seqlens, shape, scale, window, lse, target, workspace, workspace_bytes,
+                               dev_status, stream);
   DeviceInfo dev;
   if ((st = device_info(&dev)) != KVPOP_OK) return st;
-  AttnParams p;
-  if ((st = fill_attn_common(&p, q, k, cu_seqlens, shape, scale, true)) != KVPOP_OK) return st;
-  build_schedule(cu_seqlens, shape.batch, shape.n_kv_heads * G, &p.sched);
-  p.g_split = G;
-  p.window = std::min<int32_t>(window, kMaxLevels * kTileRows + 1);
-  p.lse_in = lse;
-  p.out = partials;
-  p.status = dev_status;
-  if (p.sched.total_items == 0) return KVPOP_OK;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_future_target(p, shape.head_dim, grid_for(p.sched.total_items, dev.sm_count), s);
-  if (e != cudaSuccess) return cuda_fail(e, "future_target launch");
-  e = launch_merge_partials(partials, target, G, shape.n_kv_heads, shape.total_tokens, dev.sm_count, s);
-  return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "merge of the split partials");
+  const float inv_scale = static_cast<float>(1.0 / static_cast<double>(scale));
+  cudaError_t e = launch_norm_rows(lse, workspace, static_cast<int64_t>(shape.n_q_heads) * shape.total_tokens,
+                                   inv_scale, dev.sm_count, s);
+  if (e != cudaSuccess) return cuda_fail(e, "normaliser rows launch");
+  float* partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kvpop_target_workspace_bytes(shape));
+  return run_target(q, k, cu_seqlens, shape, scale, window, workspace, target, partials, dev_status, s, dev);
 }
 
 kvpop_status kvpop_keep_mask(const float* score, const int32_t* cu_seqlens, kvpop_shape shape, int32_t window,
@@ -600,7 +644,8 @@ kvpop_status kvpop_decode_attention_noalloc(const void* q, const void* k_cache, 
 
 kvpop_status kvpop_future_targets(const void* q, const void* k, const int32_t* cu_seqlens, kvpop_shape shape,
                                   float scale, int32_t window, int32_t sinks, const int32_t* budgets, float* lse,
-                                  float* target, uint8_t* keep, int32_t* dev_status, void* stream) {
+                                  float* target, uint8_t* keep, void* workspace, size_t workspace_bytes,
+                                  int32_t* dev_status, void* stream) {
   kvpop_status st;
   // Validate everything before the first launch.
   if ((st = check_qk(q, k, scale)) != KVPOP_OK) return st;
@@ -611,9 +656,16 @@ kvpop_status kvpop_future_targets(const void* q, const void* k, const int32_t* c
   for (int b = 0; b < shape.batch; ++b)
     if (static_cast<int64_t>(budgets[b]) < static_cast<int64_t>(sinks) + window)
       return fail(KVPOP_ERR_INVALID_ARG, "budget[%d] = %d is below sinks + window", b, budgets[b]);
-  if ((st = kvpop_row_lse(q, k, cu_seqlens, shape, scale, lse, dev_status, stream)) != KVPOP_OK) return st;
-  if ((st = kvpop_future_target(q, k, cu_seqlens, shape, scale, window, lse, target, dev_status, stream)) !=
-      KVPOP_OK)
+  if (shape.total_tokens == 0) return KVPOP_OK;
+  if ((st = check_workspace(workspace, workspace_bytes, kvpop_target_workspace_bytes(shape), 16)) != KVPOP_OK)
+    return st;
+  DeviceInfo dev;
+  if ((st = device_info(&dev)) != KVPOP_OK) return st;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // Pass 1 writes the normaliser rows next to lse; pass 2 streams them.
+  if ((st = run_row_lse(q, k, cu_seqlens, shape, scale, lse, workspace, dev_status, s, dev)) != KVPOP_OK ||
+      (st = run_target(q, k, cu_seqlens, shape, scale, window, workspace, target, nullptr, dev_status, s, dev)) !=
+          KVPOP_OK)
     return st;
   return kvpop_keep_mask(target, cu_seqlens, shape, window, sinks, budgets, keep, stream);
 }
@@ -622,7 +674,8 @@ size_t kvpop_fused_workspace_bytes(const int32_t* cu_seqlens, kvpop_shape shape)
   if (cu_seqlens == nullptr || shape.batch < 1 || shape.batch > kMaxSeqs || shape.n_q_heads < 1) return 0;
   const int64_t tiles = flag_tiles(cu_seqlens, shape.batch);
   if (tiles < 0) return 0;
-  return align256(static_cast<size_t>(shape.n_q_heads * tiles + 2) * sizeof(int32_t));
+  return align256(static_cast<size_t>(shape.n_q_heads * tiles + 2) * sizeof(int32_t)) +
+         align256(norm_rows_bytes(shape));
 }
 
 kvpop_status kvpop_future_targets_fused(const void* q, const void* k, const int32_t* cu_seqlens, kvpop_shape shape,
@@ -638,12 +691,9 @@ kvpop_status kvpop_future_targets_fused(const void* q, const void* k, const int3
   for (int b = 0; b < shape.batch; ++b)
     if (static_cast<int64_t>(budgets[b]) < static_cast<int64_t>(sinks) + window)
       return fail(KVPOP_ERR_INVALID_ARG, "budget[%d] = %d is below sinks + window", b, budgets[b]);
-  const size_t need = kvpop_fused_workspace_bytes(cu_seqlens, shape);
-  if (workspace == nullptr || workspace_bytes < need)
-    return fail(KVPOP_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu required", workspace_bytes,
-                need);
-  if ((reinterpret_cast<uintptr_t>(workspace) & 3u) != 0)
-    return fail(KVPOP_ERR_INVALID_ARG, "workspace must be 4-byte aligned");
+  if ((st = check_workspace(workspace, workspace_bytes, kvpop_fused_workspace_bytes(cu_seqlens, shape), 16)) !=
+      KVPOP_OK)
+    return st;
   if (static_cast<int64_t>(shape.n_q_heads) * flag_tiles(cu_seqlens, shape.batch) >= (int64_t(1) << 31))
     return fail(KVPOP_ERR_UNSUPPORTED, "too many (query head, tile) flags for one launch");
   if (shape.total_tokens == 0) return KVPOP_OK;
@@ -664,7 +714,6 @@ kvpop_status kvpop_future_targets_fused(const void* q, const void* k, const int3
   }
   fp.attn.window = std::min<int32_t>(window, kMaxLevels * kTileRows + 1);
   fp.attn.out = lse;
-  fp.attn.lse_in = lse;
   fp.attn.status = dev_status;
   fp.target = target;
   std::vector<int32_t> base(shape.batch + 1, 0);
@@ -675,6 +724,8 @@ kvpop_status kvpop_future_targets_fused(const void* q, const void* k, const int3
   fp.flags = static_cast<int32_t*>(workspace);
   fp.done = fp.flags + fp.n_flags;
   fp.lse_done = fp.done + 1;
+  // Pass 1 writes the normaliser rows after the counters; pass 2 reads them.
+  fp.attn.nrm_rows = static_cast<uint8_t*>(workspace) + align256(static_cast<size_t>(fp.n_flags + 2) * sizeof(int32_t));
   for (size_t r = 0; r < order_lse.size(); ++r) fp.tile_base_lse[r] = base[order_lse[r]];
   for (size_t r = 0; r < order_tgt.size(); ++r) fp.tile_base_target[r] = base[order_tgt[r]];
   if (fp.attn.sched.total_items > 0) {
@@ -698,10 +749,12 @@ size_t kvpop_host_workspace_bytes(kvpop_shape shape) {
     return 0;
   const size_t T = static_cast<size_t>(shape.total_tokens);
   const size_t G = static_cast<size_t>(shape.n_q_heads / shape.n_kv_heads);
-  const size_t partials = G * host_group_max(shape.n_kv_heads) * target_split_groups() * T * 4;
+  const size_t group_q_heads = G * host_group_max(shape.n_kv_heads);
+  const size_t partials = group_q_heads * target_split_groups() * T * 4;
+  const size_t rows = group_q_heads * T * 16;
   return align256(T * shape.n_q_heads * shape.head_dim * 2) + align256(T * shape.n_kv_heads * shape.head_dim * 2) +
          align256(T * shape.n_q_heads * 4) + align256(T * shape.n_kv_heads * 4) + align256(T * shape.n_kv_heads) +
-         align256(partials);
+         align256(rows) + align256(partials);
 }
 
 kvpop_status kvpop_future_targets_host(const void* q_host, const void* k_host, const int32_t* cu_seqlens,
@@ -735,10 +788,11 @@ kvpop_status kvpop_future_targets_host(const void* q_host, const void* k_host, c
   float* lse = reinterpret_cast<float*>(w + align256(qb) + align256(kb));
   float* target = reinterpret_cast<float*>(w + align256(qb) + align256(kb) + align256(lb));
   uint8_t* keep = w + align256(qb) + align256(kb) + align256(lb) + align256(tb);
-  float* partials = reinterpret_cast<float*>(w + align256(qb) + align256(kb) + align256(lb) + align256(tb) +
-                                             align256(T * shape.n_kv_heads));
-  const size_t partials_bytes = need - (align256(qb) + align256(kb) + align256(lb) + align256(tb) +
-                                        align256(T * shape.n_kv_heads));
+  uint8_t* rows = w + align256(qb) + align256(kb) + align256(lb) + align256(tb) + align256(T * shape.n_kv_heads);
+  float* partials = reinterpret_cast<float*>(rows + align256(static_cast<size_t>(G) * host_group_max(shape.n_kv_heads) *
+                                                             T * 16));
+  DeviceInfo dev;
+  if ((st = device_info(&dev)) != KVPOP_OK) return st;
   HostStreams hs;
   if ((st = host_streams(&hs)) != KVPOP_OK) return st;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -785,9 +839,10 @@ kvpop_status kvpop_future_targets_host(const void* q_host, const void* k_host, c
     sc.n_kv_heads = hn;
     float* lse_c = lse + static_cast<size_t>(h0) * G * T;
     float* target_c = target + static_cast<size_t>(h0) * T;
-    if ((st = kvpop_row_lse(qc, kc, cu_seqlens, sc, scale, lse_c, dev_status, stream)) != KVPOP_OK ||
-        (st = kvpop_future_target_split(qc, kc, cu_seqlens, sc, scale, window, lse_c, target_c, partials,
-                                        partials_bytes, dev_status, stream)) != KVPOP_OK ||
+    // Groups run one after another on `stream`, so they share the rows and partials.
+    if ((st = run_row_lse(qc, kc, cu_seqlens, sc, scale, lse_c, rows, dev_status, s, dev)) != KVPOP_OK ||
+        (st = run_target(qc, kc, cu_seqlens, sc, scale, window, rows, target_c, G > 1 ? partials : nullptr,
+                         dev_status, s, dev)) != KVPOP_OK ||
         (st = kvpop_keep_mask(target_c, cu_seqlens, sc, window, sinks, budgets, keep + static_cast<size_t>(h0) * T,
                               stream)) != KVPOP_OK)
       return st;

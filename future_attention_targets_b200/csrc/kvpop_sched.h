@@ -32,7 +32,8 @@ struct LevelSchedule {
 struct AttnParams {
   CUtensorMap tmap_q;     // bf16 [T, H_q * d], box {64, rows}
   CUtensorMap tmap_k;     // bf16 [T, H_kv * d], box {64, rows}
-  const float* lse_in;    // pass 2: [H_q, T]
+  void* nrm_rows;         // normaliser rows [H_q, T] x 16 bytes: pass 2 reads them, pass 1
+                          // writes them when non-null (next to lse)
   float* out;             // pass 1: lse [H_q, T]; pass 2: target [H_kv, T]
   int32_t* status;
   uint64_t wait_ns;

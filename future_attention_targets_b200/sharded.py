@@ -22,7 +22,8 @@ import math
 
 import numpy as np
 
-from ._binding import future_target, future_target_split, keep_mask, row_lse, target_split_workspace_bytes
+from ._binding import (future_target, future_target_split, keep_mask, row_lse, target_split_workspace_bytes,
+                       target_workspace_bytes)
 
 
 def head_range(n_kv_heads: int, world: int, rank: int) -> tuple[int, int]:
@@ -91,11 +92,12 @@ class HeadShardedTargets:
         self.keep = torch.empty((n_kv_heads, T), dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         # A shard holds few KV heads: its transposed pass takes one item per
-        # (key tile, query head), which needs a partial-sum workspace.
-        self.split_ws = None
+        # (key tile, query head), whose workspace also holds partial sums.
         if self.G > 1:
             n = target_split_workspace_bytes(T, self.n_local * self.G, self.n_local, head_dim)
-            self.split_ws = torch.empty(max(n, 16), dtype=torch.uint8, device=dev)
+        else:
+            n = target_workspace_bytes(T, self.n_local, self.n_local, head_dim)
+        self.ws = torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
 
     def __call__(self, q_local, k_local, stream=None):
         import torch
@@ -105,13 +107,12 @@ class HeadShardedTargets:
         stream = torch.cuda.current_stream(self.target.device) if stream is None else stream
         with torch.cuda.stream(stream):
             row_lse(q_local, k_local, self.cu_seqlens, self.scale, out=self.lse, status=self.status, stream=stream)
-            if self.split_ws is not None:
+            if self.G > 1:
                 future_target_split(q_local, k_local, self.cu_seqlens, self.window, self.lse, self.scale,
-                                    out=self.target_local, workspace=self.split_ws, status=self.status,
-                                    stream=stream)
+                                    out=self.target_local, workspace=self.ws, status=self.status, stream=stream)
             else:
                 future_target(q_local, k_local, self.cu_seqlens, self.window, self.lse, self.scale,
-                              out=self.target_local, status=self.status, stream=stream)
+                              out=self.target_local, workspace=self.ws, status=self.status, stream=stream)
             gather_targets(self.target_local, self.target, self.group)
             keep_mask(self.target, self.cu_seqlens, self.window, self.sinks, self.budgets, out=self.keep,
                       stream=stream)

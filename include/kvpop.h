@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define KVPOP_ABI_VERSION 1
+#define KVPOP_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define KVPOP_API __attribute__((visibility("default")))
@@ -93,36 +93,46 @@ KVPOP_API kvpop_status kvpop_row_lse(const void* q, const void* k, const int32_t
                            kvpop_shape shape, float scale, float* lse,
                            int32_t* dev_status, void* stream);
 
+/* Device workspace (bytes) of kvpop_future_target and kvpop_future_targets:
+ * the normaliser rows of the transposed pass, 16 bytes per (query head,
+ * token), rounded up to 256; 0 for T = 0. */
+KVPOP_API size_t kvpop_target_workspace_bytes(kvpop_shape shape);
+
 /* Future-attention target: the transposed pass.  Each CTA owns a tile of 128
  * keys of one KV head and streams the query tiles i >= j + W of all G query
  * heads of its group, so the sum over queries and over the GQA group stays
  * inside one thread per key (KVpop: "transposed-attention pass", aiweekly
- * article, second paragraph).
+ * article, second paragraph).  A first small kernel turns lse into the rows
+ * that the tensor cores subtract from every score (lse_i / s as three bf16
+ * parts, 16 bytes a row); they travel beside each query tile in one bulk copy.
  *   window      W >= 0, the protected recent window
  *   lse         device fp32 [n_q_heads, T] from kvpop_row_lse with the same q, k, scale
  *   target      device fp32 [n_kv_heads, T], written for every (h, j)
+ *   workspace   device, >= kvpop_target_workspace_bytes(shape) bytes, 16-byte
+ *               aligned; contents on entry are ignored
  * other arguments as for kvpop_row_lse. */
 KVPOP_API kvpop_status kvpop_future_target(const void* q, const void* k, const int32_t* cu_seqlens,
                                  kvpop_shape shape, float scale, int32_t window,
-                                 const float* lse, float* target,
-                                 int32_t* dev_status, void* stream);
+                                 const float* lse, float* target, void* workspace,
+                                 size_t workspace_bytes, int32_t* dev_status, void* stream);
 
-/* Device workspace (bytes) of kvpop_future_target_split:
- * n_q_heads * 4 * T floats (per query head and softmax column group). */
+/* Device workspace (bytes) of kvpop_future_target_split: the normaliser rows
+ * (kvpop_target_workspace_bytes) followed by n_q_heads * 4 * T floats of
+ * partial sums (per query head and softmax column group). */
 KVPOP_API size_t kvpop_target_split_workspace_bytes(kvpop_shape shape);
 
 /* kvpop_future_target with one work item per (key tile, query head) instead
  * of per (key tile, KV head): for few KV heads per call (a group of heads, a
  * tensor-parallel shard) the G-fold larger item count keeps every SM busy.
- * Each item writes per-head partial sums to `partials`; a second kernel adds
- * them in the order the one-item-per-KV-head pass uses, so `target` is
+ * Each item writes per-head partial sums to the workspace; a second kernel
+ * adds them in the order the one-item-per-KV-head pass uses, so `target` is
  * bit-identical to kvpop_future_target's.  With G = 1 it is that call.
- *   partials   device, >= kvpop_target_split_workspace_bytes(shape) bytes,
+ *   workspace  device, >= kvpop_target_split_workspace_bytes(shape) bytes,
  *              16-byte aligned; contents on entry are ignored
  * Other arguments as for kvpop_future_target. */
 KVPOP_API kvpop_status kvpop_future_target_split(const void* q, const void* k, const int32_t* cu_seqlens,
                                                  kvpop_shape shape, float scale, int32_t window, const float* lse,
-                                                 float* target, float* partials, size_t partials_bytes,
+                                                 float* target, void* workspace, size_t workspace_bytes,
                                                  int32_t* dev_status, void* stream);
 
 /* Sink + top-k + recent-window keep set (model card, introduction; French
@@ -238,14 +248,20 @@ KVPOP_API kvpop_status kvpop_decode_attention_noalloc(const void* q, const void*
                                                       float* out, float* lse, void* stream);
 
 /* The whole hot path on device buffers: row logsumexp, transposed pass, keep
- * mask, enqueued back to back on `stream`.  lse is written as a by-product. */
+ * mask, enqueued back to back on `stream`.  lse is written as a by-product;
+ * the row-logsumexp pass also writes the transposed pass's normaliser rows
+ * into `workspace` (device, >= kvpop_target_workspace_bytes(shape) bytes,
+ * 16-byte aligned, contents on entry ignored), so no conversion kernel runs. */
 KVPOP_API kvpop_status kvpop_future_targets(const void* q, const void* k, const int32_t* cu_seqlens,
                                   kvpop_shape shape, float scale, int32_t window, int32_t sinks,
                                   const int32_t* budgets, float* lse, float* target,
-                                  uint8_t* keep, int32_t* dev_status, void* stream);
+                                  uint8_t* keep, void* workspace, size_t workspace_bytes,
+                                  int32_t* dev_status, void* stream);
 
 /* Device workspace (bytes) of kvpop_future_targets_fused: one int32 readiness
- * counter per (query head, 128-row tile of each sequence) plus two. */
+ * counter per (query head, 128-row tile of each sequence) plus two, rounded
+ * up to 256 bytes (the counter block), then the normaliser rows
+ * (kvpop_target_workspace_bytes). */
 KVPOP_API size_t kvpop_fused_workspace_bytes(const int32_t* cu_seqlens, kvpop_shape shape);
 
 /* The same three results as kvpop_future_targets with both attention passes
@@ -256,10 +272,11 @@ KVPOP_API size_t kvpop_fused_workspace_bytes(const int32_t* cu_seqlens, kvpop_sh
  * counters in `workspace`.  lse, target and keep are bit-identical to those
  * of kvpop_future_targets.
  *   workspace  device, >= kvpop_fused_workspace_bytes(cu_seqlens, shape) bytes,
- *              4-byte aligned, ZERO-FILLED before the first call; a launch
- *              that completes leaves it zero-filled again (after a timeout
- *              or a failed launch, zero it again before reuse).  Calls that
- *              share one workspace must not overlap on the GPU.
+ *              16-byte aligned; its counter block must be ZERO-FILLED before
+ *              the first call, and a launch that completes leaves it
+ *              zero-filled again (after a timeout or a failed launch, zero
+ *              it again before reuse); the rows after it are scratch.  Calls
+ *              that share one workspace must not overlap on the GPU.
  * Other arguments as for kvpop_future_targets. */
 KVPOP_API kvpop_status kvpop_future_targets_fused(const void* q, const void* k, const int32_t* cu_seqlens,
                                                   kvpop_shape shape, float scale, int32_t window, int32_t sinks,

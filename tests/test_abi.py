@@ -17,14 +17,14 @@ def lib():
 
 def test_exports_every_header_symbol(lib):
     names = B.header_symbols()
-    assert len(names) == 20, names
+    assert len(names) == 21, names
     for name in names:
         assert hasattr(lib, name), f"{name} declared in kvpop.h but not exported"
     assert set(names) == set(B._SIGS), "binding signatures and header disagree"
 
 
 def test_version_and_strings(lib):
-    assert lib.kvpop_abi_version() == 1
+    assert lib.kvpop_abi_version() == 2
     for code, word in [(0, b"ok"), (1, b"invalid argument"), (2, b"unsupported"), (3, b"CUDA error"),
                        (4, b"device wait timed out")]:
         assert lib.kvpop_status_string(code) == word
@@ -78,9 +78,25 @@ def test_cu_seqlens_null(lib):
 
 def test_future_target_rejects(lib):
     cu, sh = _cu(0, 100), _shape()
-    assert lib.kvpop_future_target(FAKE, FAKE, cu, sh, 0.1, -1, FAKE, FAKE, None, None) == B.INVALID_ARG
-    assert lib.kvpop_future_target(FAKE, FAKE, cu, sh, 0.1, 4, None, FAKE, None, None) == B.INVALID_ARG
-    assert lib.kvpop_future_target(FAKE, FAKE, cu, sh, 0.1, 4, FAKE, None, None, None) == B.INVALID_ARG
+    need = lib.kvpop_target_workspace_bytes(sh)
+    F = lib.kvpop_future_target
+    assert F(FAKE, FAKE, cu, sh, 0.1, -1, FAKE, FAKE, FAKE, need, None, None) == B.INVALID_ARG      # window
+    assert F(FAKE, FAKE, cu, sh, 0.1, 4, None, FAKE, FAKE, need, None, None) == B.INVALID_ARG       # lse
+    assert F(FAKE, FAKE, cu, sh, 0.1, 4, FAKE, None, FAKE, need, None, None) == B.INVALID_ARG       # target
+    assert F(FAKE, FAKE, cu, sh, 0.1, 4, FAKE, FAKE, None, need, None, None) == B.INVALID_ARG       # no workspace
+    assert F(FAKE, FAKE, cu, sh, 0.1, 4, FAKE, FAKE, FAKE, need - 1, None, None) == B.INVALID_ARG   # too small
+    assert F(FAKE, FAKE, cu, sh, 0.1, 4, FAKE, FAKE, FAKE + 8, need, None, None) == B.INVALID_ARG   # misaligned
+    assert b"aligned" in lib.kvpop_last_error()
+    # T = 0 needs no workspace and enqueues nothing
+    assert F(FAKE, FAKE, _cu(0, 0), B.Shape(1, 0, 4, 2, 128), 0.1, 4, FAKE, FAKE, None, 0, None, None) == B.OK
+
+
+def test_target_workspace_bytes(lib):
+    # 16 bytes of normaliser row per (query head, token), rounded up to 256
+    r = lambda x: (x + 255) // 256 * 256
+    assert lib.kvpop_target_workspace_bytes(B.Shape(1, 16384, 32, 8, 128)) == 32 * 16384 * 16
+    assert lib.kvpop_target_workspace_bytes(B.Shape(3, 101, 4, 2, 64)) == r(4 * 101 * 16)
+    assert lib.kvpop_target_workspace_bytes(B.Shape(1, 0, 4, 2, 64)) == 0
 
 
 def test_keep_mask_rejects(lib):
@@ -134,8 +150,12 @@ def test_static_cache_rejects(lib):
 def test_pipeline_rejects(lib):
     cu, sh = _cu(0, 100), _shape()
     bud = _cu(50)
-    assert lib.kvpop_future_targets(FAKE, FAKE, cu, sh, 0.1, 16, 4, _cu(10), FAKE, FAKE, FAKE, None,
-                                    None) == B.INVALID_ARG
+    tneed = lib.kvpop_target_workspace_bytes(sh)
+    P = lib.kvpop_future_targets
+    assert P(FAKE, FAKE, cu, sh, 0.1, 16, 4, _cu(10), FAKE, FAKE, FAKE, FAKE, tneed, None, None) == B.INVALID_ARG
+    assert P(FAKE, FAKE, cu, sh, 0.1, 16, 4, bud, FAKE, FAKE, FAKE, FAKE, tneed - 16, None, None) == B.INVALID_ARG
+    assert P(FAKE, FAKE, cu, sh, 0.1, 16, 4, bud, FAKE, FAKE, FAKE, FAKE + 4, tneed, None, None) == B.INVALID_ARG
+    assert P(FAKE, FAKE, cu, sh, 0.1, 16, 4, bud, FAKE, FAKE, None, FAKE, tneed, None, None) == B.INVALID_ARG
     need = lib.kvpop_host_workspace_bytes(sh)
     assert lib.kvpop_future_targets_host(FAKE, FAKE, cu, sh, 0.1, 16, 4, bud, FAKE, FAKE, FAKE, need - 1, None,
                                          None) == B.INVALID_ARG
@@ -146,6 +166,7 @@ def test_pipeline_rejects(lib):
     assert F(FAKE, FAKE, cu, sh, 0.1, 16, 4, bud, FAKE, FAKE, FAKE, None, fneed, None, None) == B.INVALID_ARG
     assert F(FAKE, FAKE, cu, sh, 0.1, 16, 4, bud, FAKE, FAKE, FAKE, FAKE, fneed - 1, None, None) == B.INVALID_ARG
     assert F(FAKE, FAKE, cu, sh, 0.1, 16, 4, bud, FAKE, FAKE, FAKE, FAKE + 2, fneed, None, None) == B.INVALID_ARG
+    assert F(FAKE, FAKE, cu, sh, 0.1, 16, 4, bud, FAKE, FAKE, FAKE, FAKE + 4, fneed, None, None) == B.INVALID_ARG
     assert F(FAKE, FAKE, cu, sh, 0.1, 16, 4, _cu(10), FAKE, FAKE, FAKE, FAKE, fneed, None, None) == B.INVALID_ARG
     assert F(FAKE, FAKE, cu, sh, 0.1, 16, 4, bud, None, FAKE, FAKE, FAKE, fneed, None, None) == B.INVALID_ARG
     assert lib.kvpop_check_device_status(None, None) == B.INVALID_ARG
@@ -157,10 +178,11 @@ def test_workspace_bytes(lib):
     sh = B.Shape(1, 16384, 32, 8, 128)
     r = lambda x: (x + 255) // 256 * 256
     T = 16384
-    # q, k, lse, target, keep, and the split partials of the largest KV-head group
-    # (eight groups of one head: G = 4 query heads x 4 column groups x T floats)
+    # q, k, lse, target, keep, then for the largest KV-head group (eight groups
+    # of one head) the normaliser rows (G = 4 query heads x T x 16 bytes) and
+    # the split partials (4 query heads x 4 column groups x T floats)
     want = (r(T * 32 * 128 * 2) + r(T * 8 * 128 * 2) + r(T * 32 * 4) + r(T * 8 * 4) + r(T * 8) +
-            r(4 * 1 * 4 * T * 4))
+            r(4 * 1 * T * 16) + r(4 * 1 * 4 * T * 4))
     assert lib.kvpop_host_workspace_bytes(sh) == want
     assert lib.kvpop_host_workspace_bytes(B.Shape(1, 0, 32, 8, 128)) == 0
 
@@ -168,7 +190,9 @@ def test_workspace_bytes(lib):
 def test_split_target_rejects_and_sizes(lib):
     cu, sh = _cu(0, 100), _shape()                       # 4 query heads over 2 KV heads
     need = lib.kvpop_target_split_workspace_bytes(sh)
-    assert need == 4 * 4 * 100 * 4                      # query heads x column groups x T floats
+    # normaliser rows (query heads x T x 16 bytes, rounded up to 256), then
+    # query heads x column groups x T floats
+    assert need == 6400 + 4 * 4 * 100 * 4
     S = lib.kvpop_future_target_split
     assert S(FAKE, FAKE, cu, sh, 0.1, 16, FAKE, FAKE, None, need, None, None) == B.INVALID_ARG       # no workspace
     assert S(FAKE, FAKE, cu, sh, 0.1, 16, FAKE, FAKE, FAKE, need - 4, None, None) == B.INVALID_ARG   # too small
@@ -179,11 +203,14 @@ def test_split_target_rejects_and_sizes(lib):
 
 
 def test_fused_workspace_bytes(lib):
-    # one int32 per (query head, 128-row tile of each sequence), plus two completion counters
+    # one int32 per (query head, 128-row tile of each sequence), plus two
+    # completion counters, rounded up to 256; then 16 bytes of normaliser row
+    # per (query head, token)
     r = lambda x: (x + 255) // 256 * 256
-    assert lib.kvpop_fused_workspace_bytes(_cu(0, 16384), B.Shape(1, 16384, 32, 8, 128)) == r((32 * 128 + 2) * 4)
+    assert lib.kvpop_fused_workspace_bytes(_cu(0, 16384), B.Shape(1, 16384, 32, 8, 128)) == \
+        r((32 * 128 + 2) * 4) + 32 * 16384 * 16
     assert lib.kvpop_fused_workspace_bytes(_cu(0, 1, 129, 129, 300), B.Shape(4, 300, 4, 2, 64)) == \
-        r((4 * (1 + 1 + 0 + 2) + 2) * 4)
+        r((4 * (1 + 1 + 0 + 2) + 2) * 4) + r(4 * 300 * 16)
     assert lib.kvpop_fused_workspace_bytes(None, B.Shape(1, 10, 4, 2, 64)) == 0
     assert lib.kvpop_fused_workspace_bytes(_cu(0, 10), B.Shape(1, 10, 0, 2, 64)) == 0
 

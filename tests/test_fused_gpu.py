@@ -3,8 +3,8 @@
 Every work item runs the same arithmetic in the same order as in the
 two-launch path, so lse, target and keep must be bit-identical to
 future_targets; the small cases are also checked against the oracle
-directly.  The flag workspace must come back zero-filled after each call so
-that it can be reused.
+directly.  The flag counters (the workspace before its normaliser rows) must come back
+zero-filled after each call so that the workspace can be reused.
 """
 import math
 
@@ -13,7 +13,8 @@ import pytest
 import torch
 
 import oracle
-from future_attention_targets_b200 import (check_status, fused_workspace, future_targets, future_targets_fused)
+from future_attention_targets_b200 import (check_status, fused_workspace, future_targets, future_targets_fused,
+                                           target_workspace_bytes)
 from future_attention_targets_b200.workloads import make_inputs, random_qk
 
 pytestmark = pytest.mark.gpu
@@ -41,7 +42,9 @@ def run_both(q_bits, k_bits, cu, W, S, budgets, scale, calls=2):
     torch.cuda.synchronize()
     check_status(st1)
     check_status(st2)
-    assert int(torch.count_nonzero(ws)) == 0, "flag workspace not cleared by the launch"
+    counters = ws.numel() - target_workspace_bytes(q.shape[0], hq, hkv, d)
+    assert 0 < counters < ws.numel()
+    assert int(torch.count_nonzero(ws[:counters])) == 0, "flag counters not cleared by the launch"
     for out in outs:
         for a, b in zip(out, ref):
             assert torch.equal(a, b)

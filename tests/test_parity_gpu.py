@@ -105,6 +105,12 @@ def test_edge_shapes(case):
     assert rel_err(tgt, ref_tgt) <= TARGET_TOL
     assert np.max(np.abs(lse - ref_lse), initial=0.0) <= LSE_TOL
     np.testing.assert_array_equal(keep, oracle.keep_mask(tgt, cu, W, 4, budgets))
+    # The separate transposed pass builds its normaliser rows from lse in a
+    # kernel of its own; the pipeline's row-logsumexp pass writes them: the
+    # same rows, so the same targets, bit for bit (ragged last tiles included).
+    q, k = dev(q_bits), dev(k_bits)
+    t2 = future_target(q, k, cu, W, row_lse(q, k, cu, scale), scale)
+    np.testing.assert_array_equal(t2.cpu().numpy(), tgt)
 
 
 # ------------------------------------------------------------------ full size: closed forms, invariants
