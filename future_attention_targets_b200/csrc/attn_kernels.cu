@@ -523,13 +523,16 @@ __device__ __forceinline__ uint64_t f2_add_rm(uint64_t a, uint64_t b) {
 
 // 2^y for a pair, on the FMA pipe: Cody-Waite reduction y = n + f with
 // n = floor(y) (adding 1.5 * 2^23 rounded toward -inf leaves n in the low
-// mantissa bits), 2^f from a degree-4 minimax polynomial with p(0) = 1
-// (coefficients from fit_exp2_poly.py, max relative error 3.0e-6 in fp32),
+// mantissa bits), 2^f from a minimax polynomial with p(0) = 1 (coefficients
+// from fit_exp2_poly.py: degree 4, max relative error 3.0e-6 in fp32, for
+// the row logsumexp; degree 3, 8.6e-5, for the transposed pass, whose error
+// goes only into targets held to 2e-3),
 // and 2^n applied by adding n to the exponent field.  Inputs are clamped to
 // >= -126 so the exponent arithmetic cannot wrap; results below 2^-126 are
 // therefore at most 2^-125 instead of 0, far below any tolerance.
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
 constexpr float kP1 = 0x1.62d6c6p-1f, kP2 = 0x1.ee2450p-3f, kP3 = 0x1.abf868p-5f, kP4 = 0x1.b7f730p-7f;
+constexpr float kT1 = 0x1.63e658p-1f, kT2 = 0x1.d2378ap-3f, kT3 = 0x1.3baaa6p-4f;
 
 __device__ __forceinline__ uint64_t exp2_poly_pair(uint64_t y) {
   float y0, y1;
@@ -563,9 +566,8 @@ __device__ __forceinline__ uint64_t exp2_poly_pair_scaled(uint64_t x, uint64_t c
   float n0, n1;
   f2_unpack(n, n0, n1);
   const uint64_t f = f2_fma(xc, c2, f2_pack(-n0, -n1));
-  uint64_t q = f2_fma(f, f2_pack(kP4, kP4), f2_pack(kP3, kP3));
-  q = f2_fma(q, f, f2_pack(kP2, kP2));
-  q = f2_fma(q, f, f2_pack(kP1, kP1));
+  uint64_t q = f2_fma(f, f2_pack(kT3, kT3), f2_pack(kT2, kT2));
+  q = f2_fma(q, f, f2_pack(kT1, kT1));
   q = f2_fma(q, f, f2_pack(1.f, 1.f));
   float t0, t1, q0, q1;
   f2_unpack(t, t0, t1);
@@ -588,7 +590,7 @@ __device__ __forceinline__ uint64_t exp2_mufu_pair(uint64_t y) {
 #define KVPOP_POLY16_LSE 3
 #endif
 #ifndef KVPOP_POLY16_TARGET
-#define KVPOP_POLY16_TARGET 3
+#define KVPOP_POLY16_TARGET 5
 #endif
 
 template <int kPoly>
