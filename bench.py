@@ -46,11 +46,42 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+def strip_comments(src: str) -> str:
+    """C/C++ source without // and /* */ comments, trailing blanks and empty lines (string and character
+    literals kept intact), so that editing a comment leaves the code's fingerprint unchanged."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (line.rstrip() for line in "".join(out).splitlines())
+    return "\n".join(line for line in lines if line)
+
+
+def kernel_source_hash(read=None) -> str:
+    """First 16 hex digits of the sha256 of the attention kernels' sources, comments stripped.
+    read(name) -> text overrides how a source file is read (to fingerprint another revision)."""
     h = hashlib.sha256()
     for name in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, "future_attention_targets_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        if read is None:
+            with open(os.path.join(ROOT, "future_attention_targets_b200", "csrc", name)) as f:
+                text = f.read()
+        else:
+            text = read(name)
+        h.update(strip_comments(text).encode())
     return h.hexdigest()[:16]
 
 

@@ -923,7 +923,8 @@ __device__ __forceinline__ uint8_t* aligned_smem(uint8_t* raw) {
 }
 
 // Barriers, slab constants and TMEM of one CTA.  kSlab: the pass-2 layout
-// (normaliser slabs; B stages completed by 32 lane arrivals).
+// (the ones block of A; the normaliser block of every B stage zeroed, so
+// that its upper half stays zero under the bulk copies of the lower half).
 template <int HD, bool kSlab>
 __device__ __forceinline__ void cta_setup(uint8_t* smem, const Bars& bars, uint32_t* tmem_slot,
                                           volatile int* abort_flag) {

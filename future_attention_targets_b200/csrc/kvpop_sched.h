@@ -49,11 +49,11 @@ struct AttnParams {
 };
 
 // Both attention passes in one launch.  attn holds pass 1 (its tensor maps,
-// schedule and lse output, which is also attn.lse_in); pass 2 has its own
-// maps (A = 128 key rows, B = 256 query rows) and schedule.  flags counts,
-// per (query head, 128-row tile of a sequence), the pass-1 warps that have
-// written that tile's lse; it, done and lse_done are zero on entry and zero
-// again when the launch completes.
+// schedule, lse output and the normaliser rows it writes, which pass 2
+// reads); pass 2 has its own maps (A = 128 key rows, B = 256 query rows)
+// and schedule.  flags counts, per (query head, 128-row tile of a sequence),
+// the pass-1 warps that have written that tile's lse and rows; it, done and
+// lse_done are zero on entry and zero again when the launch completes.
 struct FusedParams {
   AttnParams attn;
   CUtensorMap tmap_q_stream;   // pass 2 B operand: Q, box {64, 256}
