@@ -706,6 +706,7 @@ __device__ void lse_softmax_phase(const AttnParams& p, const Phase& ph, uint8_t*
   const uint64_t c2 = f2_pack(c, c);
   const float kBig = 18446744073709551616.0f;   // 2^64: larger tile sums force an exact rescale
   const float kRebase = 4294967296.0f;          // 2^32: keep the running sum moderate
+  const float kTiny = 5.421010862427522e-20f;   // 2^-64: smaller first-tile sums take the exact max
   const LevelSchedule& sched = *ph.sched;
   const int32_t total = sched.total_items;
   for (int32_t k = 0; st.ok; ++k) {
@@ -733,13 +734,19 @@ __device__ void lse_softmax_phase(const AttnParams& p, const Phase& ph, uint8_t*
       if (!skip) {
         const uint32_t taddr = lane_addr + acc * kStreamRows;
         float ts = 0.f;
-        bool rescale = (off == -INFINITY);                 // first tile of the row: no offset yet
-        if (!rescale) {
+        // A row's first tile is summed with offset 0 instead of its exact max
+        // (one TMEM pass instead of two) and kept when the sum lands in
+        // [2^-64, 2^64): no overflow, and far from the fp32 underflow.
+        // Otherwise, as for any later tile past 2^64, the exact max is taken.
+        const bool first = (off == -INFINITY);
+        if (first) off = 0.f;
+        {
           const uint64_t nb = f2_pack(-off, -off);
           ts = masked ? group_exp_sum<true, 0>(taddr, c2, nb, 0, hi)
                       : group_exp_sum<false, KVPOP_POLY16_LSE>(taddr, c2, nb, 0, kGroupCols);
-          rescale = !(ts < kBig);
         }
+        const bool rescale = !(ts < kBig) || (first && !(ts >= kTiny));
+        if (rescale && first) off = -INFINITY;
         // Warp-uniform: the rescale path issues warp-collective TMEM loads.
         if (__any_sync(0xffffffffu, rescale)) {
           const float tm = group_max(taddr, c, 0, hi);
