@@ -395,15 +395,22 @@ class HostPipeline:
         self.h2d_bytes = T * (n_q_heads + n_kv_heads) * head_dim * 2
         self.d2h_bytes = T * n_kv_heads * 5
 
-    def __call__(self, q_host, k_host, stream=None):
-        """q_host, k_host: pinned CPU bf16 tensors.  Returns (target, keep) host tensors after syncing."""
+    def submit(self, q_host, k_host, stream=None):
+        """Enqueues one step on `stream` and returns at once; self.target and self.keep hold its results
+        once the stream has reached this point.  The workspace is reused by the next call on the same
+        stream only after this one's work there, so two pipelines on two streams let one step's copies in
+        overlap the other's compute."""
         import torch
         s = torch.cuda.current_stream(self.device) if stream is None else stream
         _check(lib().kvpop_future_targets_host(
             q_host.data_ptr(), k_host.data_ptr(), self.cu_c, self.shape, self.scale, self.window, self.sinks,
             self.budgets, self.target.data_ptr(), self.keep.data_ptr(), self.workspace.data_ptr(),
             self.workspace.numel(), self.status.data_ptr(), _stream_ptr(s)))
-        s.synchronize()
+        return s
+
+    def __call__(self, q_host, k_host, stream=None):
+        """q_host, k_host: pinned CPU bf16 tensors.  Returns (target, keep) host tensors after syncing."""
+        self.submit(q_host, k_host, stream).synchronize()
         return self.target, self.keep
 
 

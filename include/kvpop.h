@@ -297,7 +297,9 @@ KVPOP_API size_t kvpop_host_workspace_bytes(kvpop_shape shape);
  * two internal streams that the library creates once per device.  The
  * copies in wait for the work already queued on `stream` (which may still
  * read the workspace), and `stream` waits for the last copy back, so the
- * results are valid once `stream` has been synchronised.
+ * results are valid once `stream` has been synchronised.  Consecutive calls
+ * with two workspaces (and host outputs) on two streams overlap: the copies
+ * in of one run, in order on the internal stream, while the other computes.
  * Results are identical to kvpop_future_targets on device copies of q and k. */
 KVPOP_API kvpop_status kvpop_future_targets_host(const void* q_host, const void* k_host,
                                        const int32_t* cu_seqlens, kvpop_shape shape,

@@ -269,6 +269,36 @@ def test_host_pipeline_matches_device():
     np.testing.assert_array_equal(k_h.numpy(), keep)
 
 
+def test_host_pipelines_overlapped_on_two_streams():
+    """Steps submitted without synchronising, alternating between two pipelines (workspaces, pinned
+    outputs) on two streams, with different inputs per step: every step's results equal the device
+    pipeline's on that step's inputs."""
+    d = make_inputs("qwen3_4b_4k")
+    w = d["workload"]
+    args = (d["cu_seqlens"], w.n_q_heads, w.n_kv_heads, w.head_dim, w.window, w.sinks, d["budgets"], d["scale"])
+    pipes = [B.HostPipeline(*args) for _ in range(2)]
+    streams = [torch.cuda.current_stream(), torch.cuda.Stream()]
+    inputs = []
+    for seed in (0, 1, 2, 3):
+        q_bits, k_bits = random_qk(int(d["cu_seqlens"][-1]), w.n_q_heads, w.n_kv_heads, w.head_dim, seed=100 + seed)
+        inputs.append((torch.from_numpy(q_bits.view(np.int16)).view(torch.bfloat16).pin_memory(),
+                       torch.from_numpy(k_bits.view(np.int16)).view(torch.bfloat16).pin_memory(), q_bits, k_bits))
+    results = []
+    for step, (qh, kh, _, _) in enumerate(inputs):
+        pipe = pipes[step % 2]
+        if step >= 2:   # the outputs of the step two back are overwritten next: keep them
+            streams[step % 2].synchronize()
+            results[step - 2] = (results[step - 2][0].clone(), results[step - 2][1].clone())
+        pipe.submit(qh, kh, streams[step % 2])
+        results.append((pipe.target, pipe.keep))
+    torch.cuda.synchronize()
+    for step, (_, _, q_bits, k_bits) in enumerate(inputs):
+        _, t_ref, k_ref = future_targets(dev(q_bits), dev(k_bits), d["cu_seqlens"], w.window, w.sinks, d["budgets"],
+                                         scale=d["scale"])
+        assert torch.equal(results[step][0], t_ref.cpu()), step
+        assert torch.equal(results[step][1], k_ref.cpu()), step
+
+
 @pytest.mark.parametrize("seqlens,hq,hkv,d", [((700, 1, 300), 12, 6, 128),   # six groups of one KV head
                                                ((900,), 16, 8, 64),             # eight groups of one
                                                ((600,), 20, 10, 64),            # groups of 2, 2, 1, ... 1
