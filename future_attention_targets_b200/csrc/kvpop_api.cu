@@ -359,6 +359,16 @@ static kvpop_status run_target(const void* q, const void* k, const int32_t* cu_s
   return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "merge of the split partials");
 }
 
+// Every sequence's budget covers its sinks and window (budgets: host [batch]).
+static kvpop_status check_budgets(const int32_t* budgets, int batch, int32_t sinks, int32_t window) {
+  if (budgets == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "budgets is NULL");
+  for (int b = 0; b < batch; ++b)
+    if (static_cast<int64_t>(budgets[b]) < static_cast<int64_t>(sinks) + window)
+      return fail(KVPOP_ERR_INVALID_ARG, "budget[%d] = %d is below sinks + window = %lld", b, budgets[b],
+                  static_cast<long long>(sinks) + window);
+  return KVPOP_OK;
+}
+
 static kvpop_status check_workspace(const void* ws, size_t bytes, size_t need, size_t align) {
   if (ws == nullptr || bytes < need)
     return fail(KVPOP_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu required", bytes, need);
@@ -447,11 +457,7 @@ kvpop_status kvpop_keep_mask(const float* score, const int32_t* cu_seqlens, kvpo
   if (budgets == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "budgets is NULL");
   if (window < 0 || sinks < 0) return fail(KVPOP_ERR_INVALID_ARG, "window and sinks must be >= 0");
   if ((st = check_shape(cu_seqlens, shape, false)) != KVPOP_OK) return st;
-  for (int b = 0; b < shape.batch; ++b) {
-    if (static_cast<int64_t>(budgets[b]) < static_cast<int64_t>(sinks) + window)
-      return fail(KVPOP_ERR_INVALID_ARG, "budget[%d] = %d is below sinks + window = %lld", b, budgets[b],
-                  static_cast<long long>(sinks) + window);
-  }
+  if ((st = check_budgets(budgets, shape.batch, sinks, window)) != KVPOP_OK) return st;
   if (shape.total_tokens == 0) return KVPOP_OK;
   DeviceInfo dev;
   if ((st = device_info(&dev)) != KVPOP_OK) return st;
@@ -481,12 +487,7 @@ kvpop_status kvpop_prefix_topk_thresholds(const float* score, const int32_t* cu_
   if (budgets == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "budgets is NULL");
   if (window < 0 || sinks < 0) return fail(KVPOP_ERR_INVALID_ARG, "window and sinks must be >= 0");
   if ((st = check_shape(cu_seqlens, shape, false)) != KVPOP_OK) return st;
-  for (int b = 0; b < shape.batch; ++b) {
-    const int64_t k = static_cast<int64_t>(budgets[b]) - sinks - window;
-    if (k < 0)
-      return fail(KVPOP_ERR_INVALID_ARG, "budget[%d] = %d is below sinks + window = %lld", b, budgets[b],
-                  static_cast<long long>(sinks) + window);
-  }
+  if ((st = check_budgets(budgets, shape.batch, sinks, window)) != KVPOP_OK) return st;
   if (shape.total_tokens == 0) return KVPOP_OK;
   DeviceInfo dev;
   if ((st = device_info(&dev)) != KVPOP_OK) return st;
@@ -653,9 +654,7 @@ kvpop_status kvpop_future_targets(const void* q, const void* k, const int32_t* c
     return fail(KVPOP_ERR_INVALID_ARG, "lse, target, keep or budgets is NULL");
   if (window < 0 || sinks < 0) return fail(KVPOP_ERR_INVALID_ARG, "window and sinks must be >= 0");
   if ((st = check_shape(cu_seqlens, shape, true)) != KVPOP_OK) return st;
-  for (int b = 0; b < shape.batch; ++b)
-    if (static_cast<int64_t>(budgets[b]) < static_cast<int64_t>(sinks) + window)
-      return fail(KVPOP_ERR_INVALID_ARG, "budget[%d] = %d is below sinks + window", b, budgets[b]);
+  if ((st = check_budgets(budgets, shape.batch, sinks, window)) != KVPOP_OK) return st;
   if (shape.total_tokens == 0) return KVPOP_OK;
   if ((st = check_workspace(workspace, workspace_bytes, kvpop_target_workspace_bytes(shape), 16)) != KVPOP_OK)
     return st;
@@ -688,9 +687,7 @@ kvpop_status kvpop_future_targets_fused(const void* q, const void* k, const int3
     return fail(KVPOP_ERR_INVALID_ARG, "lse, target, keep or budgets is NULL");
   if (window < 0 || sinks < 0) return fail(KVPOP_ERR_INVALID_ARG, "window and sinks must be >= 0");
   if ((st = check_shape(cu_seqlens, shape, true)) != KVPOP_OK) return st;
-  for (int b = 0; b < shape.batch; ++b)
-    if (static_cast<int64_t>(budgets[b]) < static_cast<int64_t>(sinks) + window)
-      return fail(KVPOP_ERR_INVALID_ARG, "budget[%d] = %d is below sinks + window", b, budgets[b]);
+  if ((st = check_budgets(budgets, shape.batch, sinks, window)) != KVPOP_OK) return st;
   if ((st = check_workspace(workspace, workspace_bytes, kvpop_fused_workspace_bytes(cu_seqlens, shape), 16)) !=
       KVPOP_OK)
     return st;
@@ -768,9 +765,7 @@ kvpop_status kvpop_future_targets_host(const void* q_host, const void* k_host, c
   if (budgets == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "budgets is NULL");
   if (window < 0 || sinks < 0) return fail(KVPOP_ERR_INVALID_ARG, "window and sinks must be >= 0");
   if ((st = check_shape(cu_seqlens, shape, true)) != KVPOP_OK) return st;
-  for (int b = 0; b < shape.batch; ++b)
-    if (static_cast<int64_t>(budgets[b]) < static_cast<int64_t>(sinks) + window)
-      return fail(KVPOP_ERR_INVALID_ARG, "budget[%d] = %d is below sinks + window", b, budgets[b]);
+  if ((st = check_budgets(budgets, shape.batch, sinks, window)) != KVPOP_OK) return st;
   if (shape.total_tokens == 0) return KVPOP_OK;
   const size_t need = kvpop_host_workspace_bytes(shape);
   if (workspace == nullptr || workspace_bytes < need)
