@@ -35,7 +35,7 @@ def _worker(rank, world, port, out):
 
 def test_two_gloo_ranks():
     world, port = 2, _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()   # no fork of this (threaded) process
     out = mgr.dict()
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
     assert out[0][0] == out[1][0] == 2.5                  # both ranks see the slowest
