@@ -18,7 +18,7 @@
 namespace kvpop {
 cudaError_t launch_row_lse(const AttnParams& p, int head_dim, int grid, cudaStream_t stream);
 cudaError_t launch_future_target(const AttnParams& p, int head_dim, int grid, cudaStream_t stream);
-cudaError_t launch_keep_mask(const KeepParams& p, int n_kv_heads, cudaStream_t stream);
+cudaError_t launch_keep_mask(const KeepParams& p, int n_kv_heads, int sm_count, cudaStream_t stream);
 cudaError_t launch_selftest_wait(int32_t* status, uint64_t limit_ns, cudaStream_t stream);
 cudaError_t launch_prefix_thresholds(const ThresholdParams& p, int n_kv_heads, int max_len, cudaStream_t stream);
 cudaError_t launch_compact_kv(const CompactParams& p, cudaStream_t stream);
@@ -474,7 +474,7 @@ kvpop_status kvpop_keep_mask(const float* score, const int32_t* cu_seqlens, kvpo
     p.seq_len[b] = cu_seqlens[b + 1] - cu_seqlens[b];
     p.budget[b] = budgets[b];
   }
-  cudaError_t e = launch_keep_mask(p, shape.n_kv_heads, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_keep_mask(p, shape.n_kv_heads, dev.sm_count, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "keep_mask launch");
 }
 
