@@ -13,8 +13,8 @@ import pytest
 import torch
 
 import oracle
-from future_attention_targets_b200 import (check_status, fused_workspace, future_targets, future_targets_fused,
-                                           target_workspace_bytes)
+from future_attention_targets_b200 import (KvpopError, check_status, fused_workspace, future_targets,
+                                           future_targets_fused, target_workspace_bytes)
 from future_attention_targets_b200.workloads import make_inputs, random_qk
 
 pytestmark = pytest.mark.gpu
@@ -83,3 +83,29 @@ def test_fused_full_size_16k():
     lse, tgt, keep = run_both(d["q_bits"], d["k_bits"], d["cu_seqlens"], d["window"], d["sinks"], d["budgets"],
                               d["scale"], calls=3)
     assert int(keep.sum()) == 8 * 4032
+
+
+def test_flag_wait_times_out_and_the_context_survives():
+    """Counters that can never reach their thresholds (a workspace that was not zero-filled, which the
+    contract rules out) leave every transposed-pass producer waiting for lse tiles: each wait gives up
+    after its 1 s limit, the status word reports a timeout, the launch ends, and
+    after zero-filling the workspace the same call gives the right results."""
+    d = make_inputs("tiny")
+    q, k = dev(d["q_bits"]), dev(d["k_bits"])
+    hq, hkv, hd = q.shape[1], k.shape[1], q.shape[2]
+    cu, W, S, budgets, scale = d["cu_seqlens"], d["window"], d["sinks"], d["budgets"], d["scale"]
+    ws = fused_workspace(cu, hq, hkv, hd)
+    counters = ws.numel() - target_workspace_bytes(q.shape[0], hq, hkv, hd)
+    ws[:counters].view(torch.int32).fill_(-(1 << 30))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    future_targets_fused(q, k, cu, W, S, budgets, scale=scale, workspace=ws, status=status)
+    with pytest.raises(KvpopError, match="TIMEOUT"):
+        check_status(status)
+    # A timeout code; the site is the first wait to give up (the flag wait, or a wait downstream of it).
+    assert int(status.item()) & 0xff == 4
+    ws.zero_()
+    status.zero_()
+    out = future_targets_fused(q, k, cu, W, S, budgets, scale=scale, workspace=ws, status=status)
+    check_status(status)
+    for a, b in zip(out, future_targets(q, k, cu, W, S, budgets, scale=scale)):
+        assert torch.equal(a, b)
