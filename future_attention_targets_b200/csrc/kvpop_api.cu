@@ -3,8 +3,10 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -38,6 +40,30 @@ using namespace kvpop;
 namespace {
 
 thread_local std::string g_last_error;
+
+// An NVTX range named after the entry point around its host work and
+// launches: Nsight tools show (and ncu can filter by) it when attached; a
+// no-op otherwise.
+struct TraceRange {
+  explicit TraceRange(const char* name) { nvtxRangePushA(name); }
+  ~TraceRange() { nvtxRangePop(); }
+  TraceRange(const TraceRange&) = delete;
+  TraceRange& operator=(const TraceRange&) = delete;
+};
+#define KVPOP_TRACE() TraceRange kvpop_trace_range_(__func__)
+
+// Time limit of every bounded on-chip wait: KVPOP_WAIT_NS nanoseconds when
+// that environment variable holds a number in [1e3, 6e10] at the call, else
+// 1 s.
+uint64_t wait_limit_ns() {
+  const char* v = getenv("KVPOP_WAIT_NS");
+  if (v != nullptr && *v != 0) {
+    char* end = nullptr;
+    const unsigned long long x = strtoull(v, &end, 10);
+    if (end != nullptr && *end == 0 && x >= 1000ull && x <= 60000000000ull) return x;
+  }
+  return kDefaultWaitNs;
+}
 
 kvpop_status fail(kvpop_status st, const char* fmt, ...) {
   char buf[512];
@@ -215,7 +241,7 @@ kvpop_status fill_attn_common(AttnParams* p, const void* q, const void* k, const
   if ((st = make_map(&p->tmap_k, k, static_cast<int64_t>(sh.n_kv_heads) * sh.head_dim, T,
                      target_pass ? kTileRows : kStreamRows)) != KVPOP_OK)
     return st;
-  p->wait_ns = kDefaultWaitNs;
+  p->wait_ns = wait_limit_ns();
   p->total_tokens = sh.total_tokens;
   p->n_q_heads = sh.n_q_heads;
   p->n_kv_heads = sh.n_kv_heads;
@@ -379,6 +405,7 @@ static kvpop_status check_workspace(const void* ws, size_t bytes, size_t need, s
 
 kvpop_status kvpop_row_lse(const void* q, const void* k, const int32_t* cu_seqlens, kvpop_shape shape, float scale,
                            float* lse, int32_t* dev_status, void* stream) {
+  KVPOP_TRACE();
   kvpop_status st;
   if ((st = check_qk(q, k, scale)) != KVPOP_OK) return st;
   if (lse == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "lse is NULL");
@@ -398,6 +425,7 @@ size_t kvpop_target_workspace_bytes(kvpop_shape shape) {
 kvpop_status kvpop_future_target(const void* q, const void* k, const int32_t* cu_seqlens, kvpop_shape shape,
                                  float scale, int32_t window, const float* lse, float* target, void* workspace,
                                  size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  KVPOP_TRACE();
   kvpop_status st;
   if ((st = check_qk(q, k, scale)) != KVPOP_OK) return st;
   if (lse == nullptr || target == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "lse or target is NULL");
@@ -427,6 +455,7 @@ size_t kvpop_target_split_workspace_bytes(kvpop_shape shape) {
 kvpop_status kvpop_future_target_split(const void* q, const void* k, const int32_t* cu_seqlens, kvpop_shape shape,
                                        float scale, int32_t window, const float* lse, float* target, void* workspace,
                                        size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  KVPOP_TRACE();
   kvpop_status st;
   if ((st = check_qk(q, k, scale)) != KVPOP_OK) return st;
   if (lse == nullptr || target == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "lse or target is NULL");
@@ -452,6 +481,7 @@ kvpop_status kvpop_future_target_split(const void* q, const void* k, const int32
 
 kvpop_status kvpop_keep_mask(const float* score, const int32_t* cu_seqlens, kvpop_shape shape, int32_t window,
                              int32_t sinks, const int32_t* budgets, uint8_t* keep, void* stream) {
+  KVPOP_TRACE();
   kvpop_status st;
   if (score == nullptr || keep == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "score or keep is NULL");
   if (budgets == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "budgets is NULL");
@@ -481,6 +511,7 @@ kvpop_status kvpop_keep_mask(const float* score, const int32_t* cu_seqlens, kvpo
 kvpop_status kvpop_prefix_topk_thresholds(const float* score, const int32_t* cu_seqlens, kvpop_shape shape,
                                           int32_t window, int32_t sinks, const int32_t* budgets, float* thr_score,
                                           int32_t* thr_pos, void* stream) {
+  KVPOP_TRACE();
   kvpop_status st;
   if (score == nullptr || thr_score == nullptr || thr_pos == nullptr)
     return fail(KVPOP_ERR_INVALID_ARG, "score, thr_score or thr_pos is NULL");
@@ -514,6 +545,7 @@ kvpop_status kvpop_prefix_topk_thresholds(const float* score, const int32_t* cu_
 kvpop_status kvpop_compact_kv(const void* k, const void* v, const uint8_t* keep, const int32_t* cu_seqlens,
                               kvpop_shape shape, int32_t capacity, void* k_cache, void* v_cache, int32_t* pos,
                               int32_t* count, void* stream) {
+  KVPOP_TRACE();
   kvpop_status st;
   if (k == nullptr || v == nullptr || keep == nullptr || k_cache == nullptr || v_cache == nullptr ||
       pos == nullptr || count == nullptr)
@@ -565,6 +597,7 @@ size_t kvpop_decode_workspace_bytes(kvpop_cache_shape shape) {
 kvpop_status kvpop_decode_attention(const void* q, const void* k_cache, const void* v_cache, const int32_t* count,
                                     kvpop_cache_shape shape, float scale, float* out, float* lse, void* workspace,
                                     size_t workspace_bytes, void* stream) {
+  KVPOP_TRACE();
   kvpop_status st;
   if (q == nullptr || k_cache == nullptr || v_cache == nullptr || count == nullptr || out == nullptr)
     return fail(KVPOP_ERR_INVALID_ARG, "a pointer argument is NULL");
@@ -603,6 +636,7 @@ kvpop_status kvpop_decode_attention(const void* q, const void* k_cache, const vo
 kvpop_status kvpop_decode_attention_noalloc(const void* q, const void* k_cache, const void* v_cache,
                                             const int32_t* count, kvpop_cache_shape shape, float scale, float* out,
                                             float* lse, void* stream) {
+  KVPOP_TRACE();
   kvpop_status st;
   if (q == nullptr || k_cache == nullptr || v_cache == nullptr || count == nullptr || out == nullptr)
     return fail(KVPOP_ERR_INVALID_ARG, "a pointer argument is NULL");
@@ -647,6 +681,7 @@ kvpop_status kvpop_future_targets(const void* q, const void* k, const int32_t* c
                                   float scale, int32_t window, int32_t sinks, const int32_t* budgets, float* lse,
                                   float* target, uint8_t* keep, void* workspace, size_t workspace_bytes,
                                   int32_t* dev_status, void* stream) {
+  KVPOP_TRACE();
   kvpop_status st;
   // Validate everything before the first launch.
   if ((st = check_qk(q, k, scale)) != KVPOP_OK) return st;
@@ -681,6 +716,7 @@ kvpop_status kvpop_future_targets_fused(const void* q, const void* k, const int3
                                         float scale, int32_t window, int32_t sinks, const int32_t* budgets,
                                         float* lse, float* target, uint8_t* keep, void* workspace,
                                         size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  KVPOP_TRACE();
   kvpop_status st;
   if ((st = check_qk(q, k, scale)) != KVPOP_OK) return st;
   if (lse == nullptr || target == nullptr || keep == nullptr || budgets == nullptr)
@@ -758,6 +794,7 @@ kvpop_status kvpop_future_targets_host(const void* q_host, const void* k_host, c
                                        kvpop_shape shape, float scale, int32_t window, int32_t sinks,
                                        const int32_t* budgets, float* target_host, uint8_t* keep_host,
                                        void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  KVPOP_TRACE();
   kvpop_status st;
   if (q_host == nullptr || k_host == nullptr || target_host == nullptr || keep_host == nullptr)
     return fail(KVPOP_ERR_INVALID_ARG, "a host buffer is NULL");

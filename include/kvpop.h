@@ -38,11 +38,17 @@
  * Errors: a call returns KVPOP_ERR_INVALID_ARG or KVPOP_ERR_UNSUPPORTED before
  * touching the device when an argument is bad; KVPOP_ERR_CUDA when the CUDA
  * runtime reports an error (cudaGetLastError after the launch).  Kernels that
- * wait on on-chip barriers give every wait a time limit; when one runs out the
- * kernel writes a nonzero code into *dev_status, stops its work early and
- * exits cleanly; kvpop_check_device_status() maps that word to
- * KVPOP_ERR_TIMEOUT.  kvpop_last_error() gives a one-line description of the
- * last failure on the calling thread.
+ * wait on on-chip barriers give every wait a time limit (1 s, or the number
+ * of nanoseconds in the environment variable KVPOP_WAIT_NS, 1e3 .. 6e10, when
+ * it is set at the call); when one runs out the kernel writes a nonzero code
+ * into *dev_status, stops its work early and exits cleanly;
+ * kvpop_check_device_status() maps that word to KVPOP_ERR_TIMEOUT.
+ * kvpop_last_error() gives a one-line description of the last failure on the
+ * calling thread.
+ *
+ * Tracing: every call that enqueues work wraps its host work and launches in
+ * an NVTX range named after the call (seen by Nsight tools when one is
+ * attached, a no-op otherwise).
  */
 #ifndef KVPOP_H_
 #define KVPOP_H_

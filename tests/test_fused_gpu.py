@@ -85,11 +85,12 @@ def test_fused_full_size_16k():
     assert int(keep.sum()) == 8 * 4032
 
 
-def test_flag_wait_times_out_and_the_context_survives():
+def test_flag_wait_times_out_and_the_context_survives(monkeypatch):
     """Counters that can never reach their thresholds (a workspace that was not zero-filled, which the
     contract rules out) leave every transposed-pass producer waiting for lse tiles: each wait gives up
-    after its 1 s limit, the status word reports a timeout, the launch ends, and
-    after zero-filling the workspace the same call gives the right results."""
+    after its limit (50 ms here, through KVPOP_WAIT_NS), the status word reports a timeout, the launch
+    ends, and after zero-filling the workspace the same call gives the right results."""
+    monkeypatch.setenv("KVPOP_WAIT_NS", "50000000")
     d = make_inputs("tiny")
     q, k = dev(d["q_bits"]), dev(d["k_bits"])
     hq, hkv, hd = q.shape[1], k.shape[1], q.shape[2]
