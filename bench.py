@@ -602,6 +602,11 @@ def run_ours(args):
             "pct_of_bf16_peak": 100.0 * value / world / peak,
             "pct_of_bf16_peak_sustained": 100.0 * value / world / peak_sus,
             "keys_per_s": keys / (attn_ms * 1e-3),
+            "keys_per_s_with_keep_mask": keys / ((attn_ms + avg["keep_mask"]) * 1e-3),
+            # The transposed pass on its own, per GPU (its call also runs the normaliser-row kernel).
+            "target_pass_only": {"value": fl["target"] / (avg["future_target"] * 1e-3) / 1e12, "unit": UNIT,
+                                 "pct_of_bf16_peak": 100.0 * fl["target"] / (avg["future_target"] * 1e-3) / 1e12
+                                 / peak},
             "kernel_ms": {n: round(v, 4) for n, v in avg.items()},
             "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": f"{peak_kind} bf16 burst",
