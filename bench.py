@@ -608,6 +608,8 @@ def run_ours(args):
                                  "pct_of_bf16_peak": 100.0 * fl["target"] / (avg["future_target"] * 1e-3) / 1e12
                                  / peak},
             "kernel_ms": {n: round(v, 4) for n, v in avg.items()},
+            "kernel_ms_median": {n: round(statistics.median(v), 4) for n, v in per_kernel.items()},
+            "kernel_ms_best": {n: round(min(v), 4) for n, v in per_kernel.items()},
             "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": f"{peak_kind} bf16 burst",
                          "traffic": recorded_traffic(dom),
