@@ -423,8 +423,11 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
 
 // One CTA per (sequence, query head): merge the splits.  Launched as a
 // programmatic dependent of the split kernel, so it waits (griddepcontrol)
-// until that grid has finished and its writes are visible.  The split loops
-// are strided over the threads or unrolled so that their loads overlap.
+// until that grid has finished and its writes are visible.  Up to 64 splits
+// the whole partial block is staged in shared memory with every load issued
+// at once (one round trip instead of three dependent ones); beyond that the
+// split loops are strided over the threads or unrolled so that their loads
+// overlap.
 __device__ __forceinline__ float block_reduce_128(float x, float* red, bool is_max) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -440,8 +443,51 @@ __device__ __forceinline__ float block_reduce_128(float x, float* red, bool is_m
   return t;
 }
 
+// Splits whose partials are staged whole in shared memory (one round of
+// loads); more splits take the streaming path below.
+constexpr int kCombineStagedSplits = 64;
+
 __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_constant__ DecodeParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ float2 staged[kCombineStagedSplits * 65];       // ns x (d + 2) floats, d <= 128
+  __shared__ float wsm[kCombineStagedSplits];
+  __shared__ float red2[2];
+  if (p.n_split <= kCombineStagedSplits) {
+    const int bg = blockIdx.x, tid = threadIdx.x;
+    const int d = p.head_dim, ns = p.n_split, stride = d + 2, half = stride / 2;
+    const float2* part = reinterpret_cast<const float2*>(p.partial + static_cast<int64_t>(bg) * ns * stride);
+    for (int i = tid; i < ns * half; i += 128) staged[i] = part[i];     // every load issued before any use
+    __syncthreads();
+    const float* st = reinterpret_cast<const float*>(staged);
+    if (tid < 32) {
+      float m = -INFINITY;
+      for (int s2 = tid; s2 < ns; s2 += 32) m = fmaxf(m, st[s2 * stride + d]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      float l = 0.f;
+      for (int s2 = tid; s2 < ns; s2 += 32) {
+        const float ms = st[s2 * stride + d];
+        const float w = (m > -INFINITY && ms > -INFINITY) ? exp2f(ms - m) : 0.f;
+        wsm[s2] = w;
+        l += st[s2 * stride + d + 1] * w;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+      if (tid == 0) {
+        red2[0] = m;
+        red2[1] = l;
+      }
+    }
+    __syncthreads();
+    const float mm = red2[0], ll = red2[1];
+    for (int e = tid; e < d; e += 128) {
+      float oo = 0.f;
+      for (int s2 = 0; s2 < ns; ++s2) oo = fmaf(st[s2 * stride + e], wsm[s2], oo);
+      p.out[static_cast<int64_t>(bg) * d + e] = (ll > 0.f) ? oo / ll : 0.f;
+    }
+    if (tid == 0 && p.lse != nullptr) p.lse[bg] = (ll > 0.f) ? (mm + log2f(ll)) * 0.6931471805599453f : -INFINITY;
+    return;
+  }
   constexpr int kMaxSplitsInSmem = 1024;      // split weights kept in shared memory (more splits: recomputed)
   __shared__ float red[4];
   __shared__ float wsplit[kMaxSplitsInSmem];

@@ -73,7 +73,10 @@ def test_compaction_clustered_masks(seqlens, C):
                                         (8, 64, 513, [513, 512, 1, 2]),
                                         # warp (32-slot) and CTA (128-slot) boundaries, several sequences
                                         (4, 128, 300, [[129, 32, 33, 95], [1, 300, 128, 31], [0, 0, 0, 64]]),
-                                        (2, 64, 130, [[127, 128], [129, 130]])])
+                                        (2, 64, 130, [[127, 128], [129, 130]]),
+                                        # the merge stages up to 64 splits in shared memory, streams beyond
+                                        (4, 128, 8192, [8192, 8191, 1, 0]),
+                                        (2, 64, 9000, [9000, 8193, 4, 0])])
 def test_decode_attention_random_cache(G, d, C, fill):
     fill = fill if isinstance(fill[0], list) else [fill]
     B, Hkv = len(fill), len(fill[0])
