@@ -150,6 +150,28 @@ def _ptr(t) -> int | None:
     return None if t is None else t.data_ptr()
 
 
+def _tensor(t, shape, dtype, device, name):
+    """t, checked: the kernels read or write it through its pointer alone, so its dtype, shape, device and
+    layout must be exactly what the call describes."""
+    import torch
+    if (not isinstance(t, torch.Tensor) or t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_cuda
+            or t.device != device or not t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous {dtype} CUDA tensor of shape {tuple(shape)} on {device}")
+    return t
+
+
+def _out(t, shape, dtype, device, name):
+    """A fresh output tensor when t is None, else t after _tensor's checks."""
+    import torch
+    if t is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    return _tensor(t, shape, dtype, device, name)
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
 # ------------------------------------------------------------------ entry points
 
 def row_lse(q, k, cu_seqlens, scale: float | None = None, out=None, status=None, stream=None):
@@ -159,19 +181,22 @@ def row_lse(q, k, cu_seqlens, scale: float | None = None, out=None, status=None,
     cu, cu_c = _cu_host(cu_seqlens)
     sh = _shape(q, k, cu)
     scale = 1.0 / math.sqrt(sh.head_dim) if scale is None else float(scale)
-    if out is None:
-        out = torch.empty((sh.n_q_heads, sh.total_tokens), dtype=torch.float32, device=q.device)
+    out = _out(out, (sh.n_q_heads, sh.total_tokens), torch.float32, q.device, "out")
     _check(lib().kvpop_row_lse(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, out.data_ptr(), _ptr(status),
                                _stream_ptr(stream)))
     return out
 
 
 def _workspace(nbytes: int, device, workspace):
-    """The caller's workspace if given, else a fresh uint8 CUDA tensor of nbytes (at least 256)."""
+    """The caller's workspace (a contiguous CUDA tensor on `device`; the library checks its size in bytes)
+    if given, else a fresh uint8 CUDA tensor of nbytes (at least 256)."""
     import torch
-    if workspace is not None:
-        return workspace
-    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    if workspace is None:
+        return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    if (not isinstance(workspace, torch.Tensor) or not workspace.is_cuda or workspace.device != device
+            or not workspace.is_contiguous()):
+        raise ValueError(f"workspace must be a contiguous CUDA tensor on {device}")
+    return workspace
 
 
 def future_target(q, k, cu_seqlens, window: int, lse, scale: float | None = None, out=None, workspace=None,
@@ -182,14 +207,12 @@ def future_target(q, k, cu_seqlens, window: int, lse, scale: float | None = None
     cu, cu_c = _cu_host(cu_seqlens)
     sh = _shape(q, k, cu)
     scale = 1.0 / math.sqrt(sh.head_dim) if scale is None else float(scale)
-    if lse.dtype != torch.float32 or not lse.is_cuda or tuple(lse.shape) != (sh.n_q_heads, sh.total_tokens):
-        raise ValueError("lse must be a fp32 CUDA tensor [H_q, T]")
-    if out is None:
-        out = torch.empty((sh.n_kv_heads, sh.total_tokens), dtype=torch.float32, device=q.device)
+    _tensor(lse, (sh.n_q_heads, sh.total_tokens), torch.float32, q.device, "lse")
+    out = _out(out, (sh.n_kv_heads, sh.total_tokens), torch.float32, q.device, "out")
     workspace = _workspace(lib().kvpop_target_workspace_bytes(sh), q.device, workspace)
     _check(lib().kvpop_future_target(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, int(window),
-                                     lse.contiguous().data_ptr(), out.data_ptr(), workspace.data_ptr(),
-                                     workspace.numel(), _ptr(status), _stream_ptr(stream)))
+                                     lse.data_ptr(), out.data_ptr(), workspace.data_ptr(),
+                                     _nbytes(workspace), _ptr(status), _stream_ptr(stream)))
     return out
 
 
@@ -201,14 +224,12 @@ def future_target_split(q, k, cu_seqlens, window: int, lse, scale: float | None 
     cu, cu_c = _cu_host(cu_seqlens)
     sh = _shape(q, k, cu)
     scale = 1.0 / math.sqrt(sh.head_dim) if scale is None else float(scale)
-    if lse.dtype != torch.float32 or not lse.is_cuda or tuple(lse.shape) != (sh.n_q_heads, sh.total_tokens):
-        raise ValueError("lse must be a fp32 CUDA tensor [H_q, T]")
-    if out is None:
-        out = torch.empty((sh.n_kv_heads, sh.total_tokens), dtype=torch.float32, device=q.device)
+    _tensor(lse, (sh.n_q_heads, sh.total_tokens), torch.float32, q.device, "lse")
+    out = _out(out, (sh.n_kv_heads, sh.total_tokens), torch.float32, q.device, "out")
     workspace = _workspace(lib().kvpop_target_split_workspace_bytes(sh), q.device, workspace)
     _check(lib().kvpop_future_target_split(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, int(window),
-                                           lse.contiguous().data_ptr(), out.data_ptr(), workspace.data_ptr(),
-                                           workspace.numel(), _ptr(status), _stream_ptr(stream)))
+                                           lse.data_ptr(), out.data_ptr(), workspace.data_ptr(),
+                                           _nbytes(workspace), _ptr(status), _stream_ptr(stream)))
     return out
 
 
@@ -232,8 +253,7 @@ def keep_mask(score, cu_seqlens, window: int, sinks: int, budgets, out=None, str
     bud = _i32_host(budgets)
     if len(bud) != sh.batch:
         raise ValueError("one budget per sequence is needed")
-    if out is None:
-        out = torch.empty((Hkv, T), dtype=torch.uint8, device=score.device)
+    out = _out(out, (Hkv, T), torch.uint8, score.device, "out")
     _check(lib().kvpop_keep_mask(score.data_ptr(), cu_c, sh, int(window), int(sinks), bud, out.data_ptr(),
                                  _stream_ptr(stream)))
     return out
@@ -250,10 +270,9 @@ def prefix_topk_thresholds(score, cu_seqlens, window: int, sinks: int, budgets, 
     bud = _i32_host(budgets)
     if len(bud) != sh.batch:
         raise ValueError("one budget per sequence is needed")
-    if out is None:
-        out = (torch.empty((Hkv, T), dtype=torch.float32, device=score.device),
-               torch.empty((Hkv, T), dtype=torch.int32, device=score.device))
-    thr_s, thr_p = out
+    out = (None, None) if out is None else out
+    thr_s = _out(out[0], (Hkv, T), torch.float32, score.device, "out[0]")
+    thr_p = _out(out[1], (Hkv, T), torch.int32, score.device, "out[1]")
     _check(lib().kvpop_prefix_topk_thresholds(score.data_ptr(), cu_c, sh, int(window), int(sinks), bud,
                                               thr_s.data_ptr(), thr_p.data_ptr(), _stream_ptr(stream)))
     return thr_s, thr_p
@@ -265,18 +284,17 @@ def compact_kv(k, v, keep, cu_seqlens, capacity: int, out=None, stream=None):
     for name, t in (("k", k), ("v", v)):
         if t.dtype != torch.bfloat16 or not t.is_cuda or t.dim() != 3 or not t.is_contiguous():
             raise TypeError(f"{name} must be a contiguous 3-D bf16 CUDA tensor [T, H_kv, d]")
-    if keep.dtype != torch.uint8 or not keep.is_cuda or not keep.is_contiguous():
-        raise TypeError("keep must be a contiguous uint8 CUDA tensor [H_kv, T]")
     cu, cu_c = _cu_host(cu_seqlens)
     T, Hkv, d = k.shape
+    _tensor(v, (T, Hkv, d), torch.bfloat16, k.device, "v")
+    _tensor(keep, (Hkv, T), torch.uint8, k.device, "keep")
     B = len(cu) - 1
     sh = Shape(B, T, Hkv, Hkv, d)
-    if out is None:
-        out = (torch.empty((B, Hkv, capacity, d), dtype=torch.bfloat16, device=k.device),
-               torch.empty((B, Hkv, capacity, d), dtype=torch.bfloat16, device=k.device),
-               torch.empty((B, Hkv, capacity), dtype=torch.int32, device=k.device),
-               torch.empty((B, Hkv), dtype=torch.int32, device=k.device))
-    kc, vc, pos, cnt = out
+    out = (None,) * 4 if out is None else out
+    kc = _out(out[0], (B, Hkv, capacity, d), torch.bfloat16, k.device, "out[0]")
+    vc = _out(out[1], (B, Hkv, capacity, d), torch.bfloat16, k.device, "out[1]")
+    pos = _out(out[2], (B, Hkv, capacity), torch.int32, k.device, "out[2]")
+    cnt = _out(out[3], (B, Hkv), torch.int32, k.device, "out[3]")
     _check(lib().kvpop_compact_kv(k.data_ptr(), v.data_ptr(), keep.data_ptr(), cu_c, sh, int(capacity),
                                   kc.data_ptr(), vc.data_ptr(), pos.data_ptr(), cnt.data_ptr(), _stream_ptr(stream)))
     return kc, vc, pos, cnt
@@ -293,19 +311,20 @@ def decode_attention(q, k_cache, v_cache, count, scale: float | None = None, out
     if q.dtype != torch.bfloat16 or not q.is_cuda or q.dim() != 3 or not q.is_contiguous():
         raise TypeError("q must be a contiguous 3-D bf16 CUDA tensor [B, H_q, d]")
     B, Hq, d = q.shape
+    if not isinstance(k_cache, torch.Tensor) or k_cache.dim() != 4:
+        raise TypeError("k_cache must be a 4-D bf16 CUDA tensor [B, H_kv, C, d]")
     _, Hkv, C, _ = k_cache.shape
+    _tensor(k_cache, (B, Hkv, C, d), torch.bfloat16, q.device, "k_cache")
+    _tensor(v_cache, (B, Hkv, C, d), torch.bfloat16, q.device, "v_cache")
+    _tensor(count, (B, Hkv), torch.int32, q.device, "count")
     sh = CacheShape(B, Hq, Hkv, d, C)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    if out is None:
-        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
-    if lse is None:
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
-    need = int(lib().kvpop_decode_workspace_bytes(sh))
-    if workspace is None:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    out = _out(out, (B, Hq, d), torch.float32, q.device, "out")
+    lse = _out(lse, (B, Hq), torch.float32, q.device, "lse")
+    workspace = _workspace(lib().kvpop_decode_workspace_bytes(sh), q.device, workspace)
     _check(lib().kvpop_decode_attention(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), count.data_ptr(), sh,
                                         scale, out.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
-                                        workspace.numel(), _stream_ptr(stream)))
+                                        _nbytes(workspace), _stream_ptr(stream)))
     return out, lse
 
 
@@ -318,17 +337,14 @@ def future_targets(q, k, cu_seqlens, window: int, sinks: int, budgets, scale: fl
     sh = _shape(q, k, cu)
     scale = 1.0 / math.sqrt(sh.head_dim) if scale is None else float(scale)
     dev = q.device
-    if lse is None:
-        lse = torch.empty((sh.n_q_heads, sh.total_tokens), dtype=torch.float32, device=dev)
-    if target is None:
-        target = torch.empty((sh.n_kv_heads, sh.total_tokens), dtype=torch.float32, device=dev)
-    if keep is None:
-        keep = torch.empty((sh.n_kv_heads, sh.total_tokens), dtype=torch.uint8, device=dev)
+    lse = _out(lse, (sh.n_q_heads, sh.total_tokens), torch.float32, dev, "lse")
+    target = _out(target, (sh.n_kv_heads, sh.total_tokens), torch.float32, dev, "target")
+    keep = _out(keep, (sh.n_kv_heads, sh.total_tokens), torch.uint8, dev, "keep")
     bud = _i32_host(budgets)
     workspace = _workspace(lib().kvpop_target_workspace_bytes(sh), dev, workspace)
     _check(lib().kvpop_future_targets(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, int(window), int(sinks), bud,
                                       lse.data_ptr(), target.data_ptr(), keep.data_ptr(), workspace.data_ptr(),
-                                      workspace.numel(), _ptr(status), _stream_ptr(stream)))
+                                      _nbytes(workspace), _ptr(status), _stream_ptr(stream)))
     return lse, target, keep
 
 
@@ -353,18 +369,16 @@ def future_targets_fused(q, k, cu_seqlens, window: int, sinks: int, budgets, sca
     sh = _shape(q, k, cu)
     scale = 1.0 / math.sqrt(sh.head_dim) if scale is None else float(scale)
     dev = q.device
-    if lse is None:
-        lse = torch.empty((sh.n_q_heads, sh.total_tokens), dtype=torch.float32, device=dev)
-    if target is None:
-        target = torch.empty((sh.n_kv_heads, sh.total_tokens), dtype=torch.float32, device=dev)
-    if keep is None:
-        keep = torch.empty((sh.n_kv_heads, sh.total_tokens), dtype=torch.uint8, device=dev)
+    lse = _out(lse, (sh.n_q_heads, sh.total_tokens), torch.float32, dev, "lse")
+    target = _out(target, (sh.n_kv_heads, sh.total_tokens), torch.float32, dev, "target")
+    keep = _out(keep, (sh.n_kv_heads, sh.total_tokens), torch.uint8, dev, "keep")
     if workspace is None:
         workspace = fused_workspace(cu, sh.n_q_heads, sh.n_kv_heads, sh.head_dim, device=dev)
+    workspace = _workspace(0, dev, workspace)
     bud = _i32_host(budgets)
     _check(lib().kvpop_future_targets_fused(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, int(window), int(sinks),
                                             bud, lse.data_ptr(), target.data_ptr(), keep.data_ptr(),
-                                            workspace.data_ptr(), workspace.numel(), _ptr(status),
+                                            workspace.data_ptr(), _nbytes(workspace), _ptr(status),
                                             _stream_ptr(stream)))
     return lse, target, keep
 
@@ -401,6 +415,11 @@ class HostPipeline:
         stream only after this one's work there, so two pipelines on two streams let one step's copies in
         overlap the other's compute."""
         import torch
+        T, Hq, Hkv, d = self.shape.total_tokens, self.shape.n_q_heads, self.shape.n_kv_heads, self.shape.head_dim
+        for name, t, shape in (("q_host", q_host, (T, Hq, d)), ("k_host", k_host, (T, Hkv, d))):
+            if (not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or t.is_cuda
+                    or tuple(t.shape) != shape or not t.is_contiguous()):
+                raise ValueError(f"{name} must be a contiguous bf16 CPU tensor of shape {shape}")
         s = torch.cuda.current_stream(self.device) if stream is None else stream
         _check(lib().kvpop_future_targets_host(
             q_host.data_ptr(), k_host.data_ptr(), self.cu_c, self.shape, self.scale, self.window, self.sinks,

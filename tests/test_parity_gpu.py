@@ -345,3 +345,21 @@ def test_binding_rejects_bad_tensors():
     with pytest.raises(KvpopError) as ei:
         row_lse(q.bfloat16(), k, [0, 9])                 # cu_seqlens[batch] != T
     assert ei.value.status == B.INVALID_ARG
+    # Buffers the kernels write through their pointer alone are checked in the binding, before any launch.
+    qb = q.bfloat16()
+    with pytest.raises(ValueError, match="out"):
+        row_lse(qb, k, [0, 10], out=torch.empty((4, 9), dtype=torch.float32, device="cuda"))
+    lse = row_lse(qb, k, [0, 10])
+    with pytest.raises(ValueError, match="lse"):
+        future_target(qb, k, [0, 10], 2, lse.t().contiguous().t())           # right shape, not contiguous
+    with pytest.raises(ValueError, match="out"):
+        keep_mask(torch.zeros((2, 10), device="cuda"), [0, 10], 2, 1, [5],
+                  out=torch.empty((2, 10), dtype=torch.int32, device="cuda"))
+    with pytest.raises(ValueError, match="count"):
+        B.decode_attention(torch.zeros((1, 4, 128), dtype=torch.bfloat16, device="cuda"),
+                           torch.zeros((1, 2, 8, 128), dtype=torch.bfloat16, device="cuda"),
+                           torch.zeros((1, 2, 8, 128), dtype=torch.bfloat16, device="cuda"),
+                           torch.zeros((1, 2), dtype=torch.int64, device="cuda"))
+    pipe = B.HostPipeline([0, 10], 4, 2, 128, 2, 1, [5])
+    with pytest.raises(ValueError, match="q_host"):
+        pipe(torch.zeros((10, 2, 128), dtype=torch.bfloat16), torch.zeros((10, 2, 128), dtype=torch.bfloat16))
