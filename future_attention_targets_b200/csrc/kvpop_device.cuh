@@ -23,19 +23,9 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
-__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-__device__ __forceinline__ float lg2_approx(float x) {
-  float y;
-  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
@@ -129,26 +119,6 @@ __device__ __forceinline__ int32_t flag_arrive_count(int32_t* f) {
   int32_t old;
   asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(f) : "memory");
   return old;
-}
-
-// One thread waits until *f >= want.  Gives up like wait_bounded: when the
-// CTA is aborting, or after ctl.limit_ns (then it raises the abort flag and
-// records a timeout at `site`).
-__device__ __noinline__ bool wait_flag_bounded(const int32_t* f, int32_t want, const WaitCtl& ctl, int32_t site) {
-  if (flag_acquire_load(f) >= want) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    __nanosleep(64);
-    if (flag_acquire_load(f) >= want) return true;
-    if ((it & 15u) == 0u) {
-      if (*ctl.abort_flag) return false;
-      if (global_timer_ns() - t0 > ctl.limit_ns) {
-        *ctl.abort_flag = 1;
-        if (ctl.status != nullptr) atomicCAS(ctl.status, 0, 4 | (site << 8));
-        return false;
-      }
-    }
-  }
 }
 
 // ------------------------------------------------------------------ TMA
