@@ -239,6 +239,30 @@ def pin_budget_from_pages(orc):
     assert np.all(mid.sum(axis=1) == g["scored_top_k"])
 
 
+def pin_keep_protected_positions(orc):
+    """The scored top-k is drawn only from [S, L - W): sinks and recent-window
+    tokens are kept by position, so giving them the highest scores must not
+    let them take a scored slot (model card introduction: sink + scored top-k +
+    recent window, each its own share of the budget)."""
+    W, S = 5, 3
+    seqlens = (40, 25, 21)                        # L = budget + 1 in the last: exactly one token evicted
+    budgets = [20, 14, 20]
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    rng = np.random.default_rng(5)
+    score = rng.random((2, int(cu[-1]))).astype(np.float32)
+    for b, L in enumerate(seqlens):
+        s = int(cu[b])
+        score[:, s:s + S] = np.inf                 # sinks score highest
+        score[0, s + L - W:s + L] = 1e30           # so does the whole recent window
+        score[1, s + L - W] = 1e30                 # only its first position (the candidate range's edge)
+    got = orc.keep_mask(score, cu, W, S, budgets)
+    np.testing.assert_array_equal(got, keep_mask_by_sorting(score, cu, W, S, budgets))
+    for b, L in enumerate(seqlens):
+        s = int(cu[b])
+        assert np.all(got[:, s:s + L].sum(axis=1) == budgets[b])
+        assert np.all(got[:, s + S:s + L - W].sum(axis=1) == budgets[b] - S - W)
+
+
 # ------------------------------------------------------------ restrictions
 
 def pin_restrictions(orc):
@@ -268,6 +292,7 @@ ALL_PINS = [
     pin_dominant_key,
     pin_keep_mask,
     pin_budget_from_pages,
+    pin_keep_protected_positions,
     pin_restrictions,
 ]
 
@@ -375,6 +400,55 @@ def pin_threshold_steps(orc):
 
 
 ALL_PINS.append(pin_threshold_steps)
+
+
+
+def pin_threshold_onset(orc):
+    """The steps where the threshold starts to exist.  With k = budget - S - W
+    scored slots, step t has t - W - S + 1 candidates.  While fewer than k
+    compete nothing is evicted: (-inf, -1).  At the step where exactly k
+    compete the threshold is the k-th best of them, i.e. the worst one in the
+    keep order (computed here with sorted()).  With k = 0 the first candidate
+    already makes it (+inf, -1): nothing is kept."""
+    W, S = 4, 2
+    budgets = [W + S + 6, W + S, W + S + 1]
+    seqlens = (30, 12, 20)
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    rng = np.random.default_rng(17)
+    score = rng.random((2, int(cu[-1]))).astype(np.float32)
+    score[1, :] = 0.5                                  # all tied: position order decides
+    thr_s, thr_p = orc.prefix_topk_thresholds(score, cu, W, S, budgets)
+    for b, L in enumerate(seqlens):
+        s0, k_top = int(cu[b]), budgets[b] - S - W
+        onset = S + W + max(k_top, 1) - 1              # first step with max(k, 1) candidates
+        for h in range(2):
+            for t in range(onset):
+                assert thr_s[h, s0 + t] == -np.inf and thr_p[h, s0 + t] == -1, (b, h, t)
+            if k_top == 0:
+                assert thr_s[h, s0 + onset] == np.inf and thr_p[h, s0 + onset] == -1
+                continue
+            cand = sorted((-float(score[h, s0 + p]), p) for p in range(S, onset - W + 1))
+            assert len(cand) == k_top
+            worst = cand[-1]
+            assert thr_p[h, s0 + onset] == worst[1] and thr_s[h, s0 + onset] == -worst[0], (b, h)
+
+
+def pin_budget_below_protected(orc):
+    """A budget smaller than sinks + window leaves no room for the protected
+    tokens; both the keep mask and the thresholds reject it."""
+    cu = np.array([0, 50], dtype=np.int32)
+    score = np.zeros((1, 50), dtype=np.float32)
+    for fn in (orc.keep_mask, orc.prefix_topk_thresholds):
+        try:
+            fn(score, cu, 8, 4, [11])
+        except ValueError:
+            pass
+        else:
+            raise AssertionError(f"{fn.__name__} accepted a budget below sinks + window")
+        fn(score, cu, 8, 4, [12])                      # exactly sinks + window is allowed
+
+
+ALL_PINS.extend([pin_threshold_onset, pin_budget_below_protected])
 
 
 # ------------------------------------------------------------ static cache: compaction + decode attention

@@ -52,6 +52,27 @@ MUTANTS = [
     ("decode_wrong_group", "            h = g // G\n            n = int(count[b, h])", "            h = g % Hkv\n            n = int(count[b, h])"),
     ("decode_unnormalised", "out[b, g] = (w / Z) @ vc[b, h, :n]", "out[b, g] = w @ vc[b, h, :n]"),
     ("decode_scale_dropped", "logits = scale * (kc[b, h, :n] @ q[b, g])", "logits = (kc[b, h, :n] @ q[b, g])"),
+    ("bf16_decoded_wrongly", "<< np.uint32(16)", "<< np.uint32(15)"),
+    ("target_overwritten_not_summed", "target[h, s + j_lo:s + r1] += col_sum[j_lo:]",
+     "target[h, s + j_lo:s + r1] = col_sum[j_lo:]"),
+    ("target_last_row_dropped", "for r0 in range(i_start, L, ROW_BLOCK):\n                r1 = min(r0 + ROW_BLOCK, L)",
+     "for r0 in range(i_start, L, ROW_BLOCK):\n                r1 = min(r0 + ROW_BLOCK, L - 1)"),
+    ("far_mass_unwindowed", "far[g, s + r0:s + r1] = F.sum(axis=1)", "far[g, s + r0:s + r1] = A.sum(axis=1)"),
+    ("key_lo_rows_skipped", "i_start = min(L, j_lo + W) if key_lo", "i_start = min(L, j_lo + W + 1) if key_lo"),
+    ("keep_candidates_overlap_window", "lo, hi = S, L - W ", "lo, hi = S, L - W + 1 "),
+    ("keep_nan_ranked_first",
+     "sc = score[h, s + lo:s + hi].astype(np.float64)\n            order",
+     "sc = np.nan_to_num(score[h, s + lo:s + hi].astype(np.float64), nan=np.inf)\n            order"),
+    ("keep_budget_unchecked", "if B < S + W:", "if B < 0:"),
+    ("threshold_defined_one_step_late", "if len(pos) < k_top:", "if len(pos) <= k_top:"),
+    ("threshold_k0_keeps_all", "thr_s[h, s0 + t] = np.inf", "thr_s[h, s0 + t] = -np.inf"),
+    ("threshold_nan_ranked_first", "sc = score[h, s0 + S:s0 + hi + 1].astype(np.float64)",
+     "sc = np.nan_to_num(score[h, s0 + S:s0 + hi + 1].astype(np.float64), nan=np.inf)"),
+    ("threshold_budget_unchecked", "if k_top < 0:", "if k_top < -10**9:"),
+    ("compact_count_capped", "cnt[b, h] = len(p)\n            p = p[:capacity]",
+     "p = p[:capacity]\n            cnt[b, h] = len(p)"),
+    ("decode_count_ignored", "n = int(count[b, h])\n            if n == 0", "n = kc.shape[2]\n            if int(count[b, h]) == 0"),
+    ("decode_lse_max_dropped", "lse[b, g] = m + np.log(Z)", "lse[b, g] = np.log(Z)"),
 ]
 
 
