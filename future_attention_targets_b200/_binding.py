@@ -123,10 +123,40 @@ def _cu_host(cu_seqlens):
 
 
 def _stream_ptr(stream) -> int:
+    """The raw cudaStream_t of `stream` (a torch.cuda.Stream, a raw handle, or None for the current stream).
+    A torch stream must belong to the current device, on which the library launches."""
     import torch
     if stream is None:
         stream = torch.cuda.current_stream()
-    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+    if hasattr(stream, "cuda_stream"):
+        dev = getattr(stream, "device", None)
+        cur = torch.cuda.current_device()
+        if dev is not None and dev.index is not None and dev.index != cur:
+            raise ValueError(f"stream belongs to {dev} but the current CUDA device is cuda:{cur}")
+        return int(stream.cuda_stream)
+    return int(stream)
+
+
+def _on_current_device(t, name) -> None:
+    """The library launches on the calling thread's current CUDA device and takes raw pointers, so every
+    tensor it is given must live on that device (a pointer into another GPU would be read as a peer
+    address)."""
+    import torch
+    cur = torch.cuda.current_device()
+    if t.device.index != cur:
+        raise ValueError(f"{name} is on {t.device} but the current CUDA device is cuda:{cur}; "
+                         f"call under torch.cuda.device({t.device})")
+
+
+def _status_ptr(status, device):
+    """Pointer of the optional int32 status word (a CUDA tensor on `device` with at least one element)."""
+    import torch
+    if status is None:
+        return None
+    if (not isinstance(status, torch.Tensor) or status.dtype != torch.int32 or not status.is_cuda
+            or status.device != device or status.numel() < 1):
+        raise ValueError(f"status must be an int32 CUDA tensor on {device} with at least one element")
+    return status.data_ptr()
 
 
 def _shape(q, k, cu) -> Shape:
@@ -144,10 +174,9 @@ def _check_qk(q, k):
             raise ValueError(f"{name} must be contiguous")
     if q.shape[0] != k.shape[0] or q.shape[2] != k.shape[2]:
         raise ValueError("q [T, H_q, d] and k [T, H_kv, d] disagree on T or d")
-
-
-def _ptr(t) -> int | None:
-    return None if t is None else t.data_ptr()
+    if k.device != q.device:
+        raise ValueError(f"q is on {q.device} and k on {k.device}")
+    _on_current_device(q, "q")
 
 
 def _tensor(t, shape, dtype, device, name):
@@ -182,8 +211,8 @@ def row_lse(q, k, cu_seqlens, scale: float | None = None, out=None, status=None,
     sh = _shape(q, k, cu)
     scale = 1.0 / math.sqrt(sh.head_dim) if scale is None else float(scale)
     out = _out(out, (sh.n_q_heads, sh.total_tokens), torch.float32, q.device, "out")
-    _check(lib().kvpop_row_lse(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, out.data_ptr(), _ptr(status),
-                               _stream_ptr(stream)))
+    _check(lib().kvpop_row_lse(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, out.data_ptr(),
+                               _status_ptr(status, q.device), _stream_ptr(stream)))
     return out
 
 
@@ -212,7 +241,7 @@ def future_target(q, k, cu_seqlens, window: int, lse, scale: float | None = None
     workspace = _workspace(lib().kvpop_target_workspace_bytes(sh), q.device, workspace)
     _check(lib().kvpop_future_target(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, int(window),
                                      lse.data_ptr(), out.data_ptr(), workspace.data_ptr(),
-                                     _nbytes(workspace), _ptr(status), _stream_ptr(stream)))
+                                     _nbytes(workspace), _status_ptr(status, q.device), _stream_ptr(stream)))
     return out
 
 
@@ -229,7 +258,7 @@ def future_target_split(q, k, cu_seqlens, window: int, lse, scale: float | None 
     workspace = _workspace(lib().kvpop_target_split_workspace_bytes(sh), q.device, workspace)
     _check(lib().kvpop_future_target_split(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, int(window),
                                            lse.data_ptr(), out.data_ptr(), workspace.data_ptr(),
-                                           _nbytes(workspace), _ptr(status), _stream_ptr(stream)))
+                                           _nbytes(workspace), _status_ptr(status, q.device), _stream_ptr(stream)))
     return out
 
 
@@ -247,6 +276,7 @@ def keep_mask(score, cu_seqlens, window: int, sinks: int, budgets, out=None, str
     import torch
     if score.dtype != torch.float32 or not score.is_cuda or score.dim() != 2 or not score.is_contiguous():
         raise TypeError("score must be a contiguous 2-D fp32 CUDA tensor [H_kv, T]")
+    _on_current_device(score, "score")
     cu, cu_c = _cu_host(cu_seqlens)
     Hkv, T = score.shape
     sh = Shape(len(cu) - 1, T, Hkv, Hkv, 128)
@@ -264,6 +294,7 @@ def prefix_topk_thresholds(score, cu_seqlens, window: int, sinks: int, budgets, 
     import torch
     if score.dtype != torch.float32 or not score.is_cuda or score.dim() != 2 or not score.is_contiguous():
         raise TypeError("score must be a contiguous 2-D fp32 CUDA tensor [H_kv, T]")
+    _on_current_device(score, "score")
     cu, cu_c = _cu_host(cu_seqlens)
     Hkv, T = score.shape
     sh = Shape(len(cu) - 1, T, Hkv, Hkv, 128)
@@ -284,6 +315,7 @@ def compact_kv(k, v, keep, cu_seqlens, capacity: int, out=None, stream=None):
     for name, t in (("k", k), ("v", v)):
         if t.dtype != torch.bfloat16 or not t.is_cuda or t.dim() != 3 or not t.is_contiguous():
             raise TypeError(f"{name} must be a contiguous 3-D bf16 CUDA tensor [T, H_kv, d]")
+    _on_current_device(k, "k")
     cu, cu_c = _cu_host(cu_seqlens)
     T, Hkv, d = k.shape
     _tensor(v, (T, Hkv, d), torch.bfloat16, k.device, "v")
@@ -310,6 +342,7 @@ def decode_attention(q, k_cache, v_cache, count, scale: float | None = None, out
     import torch
     if q.dtype != torch.bfloat16 or not q.is_cuda or q.dim() != 3 or not q.is_contiguous():
         raise TypeError("q must be a contiguous 3-D bf16 CUDA tensor [B, H_q, d]")
+    _on_current_device(q, "q")
     B, Hq, d = q.shape
     if not isinstance(k_cache, torch.Tensor) or k_cache.dim() != 4:
         raise TypeError("k_cache must be a 4-D bf16 CUDA tensor [B, H_kv, C, d]")
@@ -344,7 +377,7 @@ def future_targets(q, k, cu_seqlens, window: int, sinks: int, budgets, scale: fl
     workspace = _workspace(lib().kvpop_target_workspace_bytes(sh), dev, workspace)
     _check(lib().kvpop_future_targets(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, int(window), int(sinks), bud,
                                       lse.data_ptr(), target.data_ptr(), keep.data_ptr(), workspace.data_ptr(),
-                                      _nbytes(workspace), _ptr(status), _stream_ptr(stream)))
+                                      _nbytes(workspace), _status_ptr(status, q.device), _stream_ptr(stream)))
     return lse, target, keep
 
 
@@ -378,8 +411,8 @@ def future_targets_fused(q, k, cu_seqlens, window: int, sinks: int, budgets, sca
     bud = _i32_host(budgets)
     _check(lib().kvpop_future_targets_fused(q.data_ptr(), k.data_ptr(), cu_c, sh, scale, int(window), int(sinks),
                                             bud, lse.data_ptr(), target.data_ptr(), keep.data_ptr(),
-                                            workspace.data_ptr(), _nbytes(workspace), _ptr(status),
-                                            _stream_ptr(stream)))
+                                            workspace.data_ptr(), _nbytes(workspace),
+                                            _status_ptr(status, q.device), _stream_ptr(stream)))
     return lse, target, keep
 
 
@@ -420,6 +453,7 @@ class HostPipeline:
             if (not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or t.is_cuda
                     or tuple(t.shape) != shape or not t.is_contiguous()):
                 raise ValueError(f"{name} must be a contiguous bf16 CPU tensor of shape {shape}")
+        _on_current_device(self.workspace, "the pipeline's workspace")
         s = torch.cuda.current_stream(self.device) if stream is None else stream
         _check(lib().kvpop_future_targets_host(
             q_host.data_ptr(), k_host.data_ptr(), self.cu_c, self.shape, self.scale, self.window, self.sinks,
@@ -435,8 +469,11 @@ class HostPipeline:
 
 def check_status(status, stream=None) -> None:
     """Raises KvpopError(TIMEOUT) when a kernel recorded a wait that ran out."""
-    _check(lib().kvpop_check_device_status(status.data_ptr(), _stream_ptr(stream)))
+    _on_current_device(status, "status")
+    _check(lib().kvpop_check_device_status(_status_ptr(status, status.device), _stream_ptr(stream)))
 
 
 def selftest_bounded_wait(status, limit_ns: int, stream=None) -> None:
-    _check(lib().kvpop_selftest_bounded_wait(status.data_ptr(), int(limit_ns), _stream_ptr(stream)))
+    _on_current_device(status, "status")
+    _check(lib().kvpop_selftest_bounded_wait(_status_ptr(status, status.device), int(limit_ns),
+                                             _stream_ptr(stream)))

@@ -360,6 +360,10 @@ def test_binding_rejects_bad_tensors():
                            torch.zeros((1, 2, 8, 128), dtype=torch.bfloat16, device="cuda"),
                            torch.zeros((1, 2, 8, 128), dtype=torch.bfloat16, device="cuda"),
                            torch.zeros((1, 2), dtype=torch.int64, device="cuda"))
+    for bad in (torch.zeros(1, dtype=torch.float32, device="cuda"), torch.zeros(0, dtype=torch.int32, device="cuda"),
+                torch.zeros(1, dtype=torch.int32)):
+        with pytest.raises(ValueError, match="status"):
+            row_lse(qb, k, [0, 10], status=bad)
     pipe = B.HostPipeline([0, 10], 4, 2, 128, 2, 1, [5])
     with pytest.raises(ValueError, match="q_host"):
         pipe(torch.zeros((10, 2, 128), dtype=torch.bfloat16), torch.zeros((10, 2, 128), dtype=torch.bfloat16))
