@@ -32,6 +32,9 @@
  * valid until the enqueued work has finished.  Calls are stream-ordered: they
  * validate on the host, enqueue on `stream` (a cudaStream_t, NULL = legacy
  * default stream) on the current device and return without synchronising.
+ * Device pointers must point into the current device's memory and `stream`
+ * must belong to that device; the library does not look a pointer's device
+ * up, so memory of another GPU would be read as a peer address.
  * The library allocates no device memory and keeps no mutable state besides
  * per-device caches (SM count, capability, kernel attributes).
  *
