@@ -7,8 +7,9 @@ inputs from it without sharing any of the computation.
 
 The five workloads mirror the shapes the KVpop pages work at: a tiny GQA-2
 case, a Qwen3-4B-shaped layer at 4k context, the Qwen3-8B-shaped 16k
-distillation layer (KVpop model card, intro: "distilled at a 16,384-token
-context", budget 4 sink + 3,772 scored + 256 recent = 4,032 per head), a
+distillation layer (KVpop model card, introduction: the model was distilled
+with a 16,384-token context and a per-head budget of 4 + 3,772 + 256 = 4,032
+entries), a
 packed variable-length batch, and a 64k long-context layer.  Q and K are
 given post-QK-norm (unit RMS per row), as bf16 bit patterns (uint16).
 """

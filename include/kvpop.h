@@ -1,10 +1,11 @@
 /*
  * kvpop.h -- C ABI for KVpop future-attention targets on NVIDIA B200 (sm_100a).
  *
- * KVpop trains a per-KV-head token scorer against a "future-attention
- * target": the attention mass a token will receive from later queries once it
- * has left a small protected recent window, computed during training with a
- * transposed attention pass so that the dense attention map is never formed
+ * KVpop trains a per-KV-head token scorer against a future-attention target:
+ * the softmax probability that later queries give a token, counted only from
+ * the step at which the token is no longer among the W most recent positions.
+ * The target is computed during training by a transposed attention pass, so
+ * the dense attention map is never formed
  * (aiweekly article "KVpop shrinks Qwen3 KV cache 88%", second paragraph;
  * KVpop paper summary; French article, second paragraph).  At inference the
  * cache keeps sink tokens, the protected recent window and the scored top-k
@@ -110,8 +111,8 @@ KVPOP_API size_t kvpop_target_workspace_bytes(kvpop_shape shape);
 /* Future-attention target: the transposed pass.  Each CTA owns a tile of 128
  * keys of one KV head and streams the query tiles i >= j + W of all G query
  * heads of its group, so the sum over queries and over the GQA group stays
- * inside one thread per key (KVpop: "transposed-attention pass", aiweekly
- * article, second paragraph).  A first small kernel turns lse into the rows
+ * inside one thread per key (the pages name the target's computation a
+ * transposed attention pass: aiweekly article, second paragraph).  A first small kernel turns lse into the rows
  * that the tensor cores subtract from every score (lse_i / s as three bf16
  * parts, 16 bytes a row); they travel beside each query tile in one bulk copy.
  *   window      W >= 0, the protected recent window
@@ -181,8 +182,9 @@ KVPOP_API kvpop_status kvpop_prefix_topk_thresholds(const float* score, const in
                                                     const int32_t* budgets, float* thr_score,
                                                     int32_t* thr_pos, void* stream);
 
-/* Static fixed-budget cache (model card, "Cache backends": fixed-size buffers
- * with the same sink + scored top-k + sliding-window budget). */
+/* Static fixed-budget cache (model card, "Cache backends": a cache of fixed
+ * size whose slots hold the same three shares as the keep mask: sinks, the
+ * scored top-k and the recent window). */
 typedef struct {
   int32_t batch;          /* sequences, 1 .. 512 */
   int32_t n_q_heads;      /* a multiple of n_kv_heads, at most 16 per KV head, group a power of two */

@@ -13,17 +13,17 @@ materialised causal softmax (one block of query rows at a time):
   the GQA mapping ``h(g) = g // G``, ``G = H_q / H_kv``.
 * Future-attention target (KVpop paper summary; the aiweekly article
   "KVpop shrinks Qwen3 KV cache 88%", second paragraph; its French
-  edition, second paragraph).  The target of key j is the attention mass it
-  receives from queries that come after it has left the protected recent
-  window of W positions.  At query i the window holds positions
+  edition, second paragraph).  Key j is labelled with the softmax
+  probability that queries give it once it is outside the window of the W
+  most recent positions.  At query i the window holds positions
   i-W+1 .. i, so key j has left it exactly when i >= j + W.  The mass is
   the softmax probability ``A[i, j] = exp(S[i, j] - lse[i])`` and the
   target of a KV head is summed over the G query heads that share it:
   ``target[h, j] = sum_{g in group(h)} sum_{i = j+W}^{L-1} A_g[i, j]``.
-* Keep mask (KVpop model card, intro: "a bounded sink + scored top-k +
-  recent-window cache", 4,032 = 4 sink + 3,772 scored + 256 recent; the
-  French article, second paragraph: sinks + protected recent window +
-  learned top-k over the older tokens).  Per sequence and KV head: keep
+* Keep mask (KVpop model card, introduction: the cache is bounded and made
+  of initial sink tokens, scored older tokens and recent tokens, with 4,032 =
+  4 + 3,772 + 256 per head; the French article, second paragraph: the same
+  three parts, the older tokens picked by a learned top-k).  Per sequence and KV head: keep
   p < S (sinks), keep p >= L - W (recent window), and among p in [S, L-W)
   keep the k = budget - S - W largest scores; equal scores go to the
   smaller position first.  Everything is kept when L <= budget.
@@ -37,8 +37,8 @@ materialised causal softmax (one block of query rows at a time):
   this is exactly online eviction of the worst token whenever the scored
   slots overflow, and at the last step it gives the keep mask above.
 
-* Static sparse cache (model card, "Cache backends": fixed-size buffers
-  holding the same sink + scored top-k + sliding-window budget).  Compaction
+* Static sparse cache (model card, "Cache backends": a cache of fixed size
+  whose slots hold the same three shares as the keep mask).  Compaction
   gathers, per sequence and KV head, the kept positions in increasing order
   into fixed slots; a decode step attends one new query per query head over
   the filled slots of its KV head: ``out = sum_s softmax_s(s q.k_s) v_s``.

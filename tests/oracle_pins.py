@@ -242,8 +242,8 @@ def pin_budget_from_pages(orc):
 def pin_keep_protected_positions(orc):
     """The scored top-k is drawn only from [S, L - W): sinks and recent-window
     tokens are kept by position, so giving them the highest scores must not
-    let them take a scored slot (model card introduction: sink + scored top-k +
-    recent window, each its own share of the budget)."""
+    let them take a scored slot (model card introduction: sinks, scored older
+    tokens and recent tokens each have their own share of the budget)."""
     W, S = 5, 3
     seqlens = (40, 25, 21)                        # L = budget + 1 in the last: exactly one token evicted
     budgets = [20, 14, 20]
