@@ -4,6 +4,7 @@
 // Both are memory-bound (a gather, and a GEMV with G query heads per KV
 // head), so they run on CUDA cores with 16-byte vector accesses; the grid is
 // split along the sequence / the cache slots so that every SM streams.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -565,23 +566,56 @@ static __device__ __align__(256) float g_decode_scratch[kDecodeScratchBytes / si
 
 size_t decode_scratch_bytes() { return kDecodeScratchBytes; }
 
+// Unique id of the calling thread's current CUDA context, or 0 when no
+// context is current or the driver cannot say.  Ids are never reused, so a
+// context created after cudaDeviceReset has a new one.
+static unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(p);
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
 // Device address of g_decode_scratch on the current device.  In host code the
-// symbol's name is only a stand-in, so the address is looked up once per
-// device (with that device current) and cached.
+// symbol's name is only a stand-in, so the address is looked up with the
+// device current, once per device, and cached together with the id of the
+// context it belongs to.  If that context has since been destroyed (by
+// cudaDeviceReset, say), the module is loaded anew at a possibly different
+// address, so a changed context id triggers a fresh lookup.
 cudaError_t decode_scratch_address(float** out) {
   constexpr int kMaxDevices = 64;
   static std::mutex mu;
   static void* addr[kMaxDevices] = {};
+  static unsigned long long ctx_of[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (addr[dev] == nullptr || ctx == 0 || ctx != ctx_of[dev]) {
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
     if (e != cudaSuccess) return e;
     addr[dev] = ptr;
+    ctx_of[dev] = current_context_id();   // the lookup makes the device's primary context current
   }
   *out = static_cast<float*>(addr[dev]);
   return cudaSuccess;

@@ -246,8 +246,10 @@ KVPOP_API kvpop_status kvpop_decode_attention(const void* q, const void* k_cache
  * return KVPOP_ERR_UNSUPPORTED; use kvpop_decode_attention for them.
  *
  * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress) and caches it; make that first call before any
- * stream capture.  The call never calls cudaMalloc or cudaFree.  Every call
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture.  The cache remembers which context
+ * the address belongs to: the first call after that context is destroyed
+ * (cudaDeviceReset, say) looks the address up again.  The call never calls cudaMalloc or cudaFree.  Every call
  * uses the same array and leaves its partials there; nothing in it needs to
  * start at zero, because each call writes every partial it later reads.
  * Calls that overlap on the GPU (for example on two streams at once) race on
