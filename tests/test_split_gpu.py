@@ -37,8 +37,13 @@ def both(q_bits, k_bits, cu, W, scale):
 
 @pytest.mark.parametrize("name", ["tiny", "qwen3_4b_4k", "varlen_8x"])
 def test_split_is_bit_identical_on_workloads(name):
+    """Every key of the split pass against the fp64 oracle, and bit for bit against the plain pass."""
+    from oracle_cache import oracle_full
     d = make_inputs(name)
     plain, split = both(d["q_bits"], d["k_bits"], d["cu_seqlens"], d["window"], d["scale"])
+    ref = oracle_full(name, d)["target"]
+    got = split.cpu().numpy().astype(np.float64)
+    assert float(np.max(np.abs(got - ref) / np.maximum(np.abs(ref), 1e-3))) <= 2e-3
     assert torch.equal(plain, split)
 
 
