@@ -34,6 +34,14 @@ def test_rank0_prints_one_reference_line():
     assert d["metric"].startswith("future-attn target TFLOP/s")
     assert d["unit"] == "TFLOP/s" and d["higher_is_better"] is True and d["value"] > 0
     assert d["steps"] == 1 and d["config"]["workload"] == "qwen3_8b_16k"
+    # The sample is one KV-head group (1/8 of the step's flops), the one the GPU arm's cpu_baseline times;
+    # ms_per_step scales its time to a whole step.
+    assert "KV head 0" in d["cpu_baseline"]["sample"] and "all 16384 positions" in d["cpu_baseline"]["sample"]
+    assert abs(d["ms_per_step"] / d["sample_ms_per_step"] - 8.0) < 0.05
+    sys.path.insert(0, ROOT)
+    import bench
+    from future_attention_targets_b200.workloads import WORKLOADS
+    assert d["config"] == bench.workload_config(WORKLOADS["qwen3_8b_16k"], 1)
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == d["value"]
     e2e = d["e2e"]
