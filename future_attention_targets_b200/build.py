@@ -47,7 +47,7 @@ def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | N
         return LIB
     tmp = LIB + ".tmp"
     cmd = [_nvcc(), *NVCC_FLAGS, *(extra_flags or []), "-I", INCLUDE, "-I", CSRC, "-shared",
-           *sources(), "-o", tmp, "-lcuda" if False else "-lcudart_static", "-ldl", "-lrt", "-lpthread"]
+           *sources(), "-o", tmp, "-lcudart_static", "-ldl", "-lrt", "-lpthread"]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
