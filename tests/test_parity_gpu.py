@@ -70,12 +70,15 @@ def _near_tie_check(d, tgt, keep, ref_tgt, heads):
     cu, W, S, budgets = d["cu_seqlens"], d["window"], d["sinks"], d["budgets"]
     ref_keep = oracle.keep_mask(ref_tgt, cu, W, S, budgets)
     diff = np.argwhere(ref_keep[heads] != keep[heads])
+    kths = {}
     for hi, p in diff:
         h = heads[hi]
         b = int(np.searchsorted(cu, p, side="right")) - 1
         lo, hi_ = int(cu[b]) + S, int(cu[b + 1]) - W
-        k_top = int(budgets[b]) - S - W
-        kth = np.sort(ref_tgt[h, lo:hi_])[::-1][k_top - 1]
+        if (h, b) not in kths:
+            k_top = int(budgets[b]) - S - W
+            kths[h, b] = np.sort(ref_tgt[h, lo:hi_])[::-1][k_top - 1]
+        kth = kths[h, b]
         assert lo <= p < hi_ and abs(ref_tgt[h, p] - kth) <= TARGET_TOL * max(abs(kth), 1e-3), (h, p)
     return len(diff)
 

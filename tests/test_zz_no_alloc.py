@@ -90,31 +90,40 @@ def run_checks():
                                                 lse.data_ptr(), stream)
         assert st == B.OK, lib.kvpop_last_error()
 
-    # Warm-up: the first call on the device looks up the array's address.
-    shape, scale, dv, _, _, _, _, _, outs = cases[0]
+    def workspace_version(shape, scale, dv, ws, out, lse):
+        st = lib.kvpop_decode_attention(dv["q"].data_ptr(), dv["k"].data_ptr(), dv["v"].data_ptr(),
+                                        dv["count"].data_ptr(), shape, scale, out.data_ptr(), lse.data_ptr(),
+                                        ws.data_ptr(), ws.numel(), stream)
+        assert st == B.OK, lib.kvpop_last_error()
+
+    # Warm-up, before any free-memory reading: the first call on the device looks up the array's address,
+    # and the first launch of each torch kernel used below (fill, copy to host) loads it lazily, which
+    # takes device memory of its own.
+    shape, scale, dv, _, _, ws, w_out, w_lse, outs = cases[0]
     noalloc(shape, scale, dv, *outs[0])
+    workspace_version(shape, scale, dv, ws, w_out, w_lse)
+    outs[0][0].fill_(float("nan"))
+    outs[0][1].fill_(float("nan"))
+    outs[0][0].cpu()
     torch.cuda.synchronize()
-    free_before, _ = torch.cuda.mem_get_info()
     for shape, scale, dv, ref_out, ref_lse, ws, w_out, w_lse, outs in cases:
         for out, lse in outs:
             out.fill_(float("nan"))
             lse.fill_(float("nan"))
         torch.cuda.synchronize()
-        for out, lse in outs:                # two calls in a row
+        free_before, _ = torch.cuda.mem_get_info()
+        for out, lse in outs:                # two calls in a row, nothing else in between
             noalloc(shape, scale, dv, out, lse)
         torch.cuda.synchronize()
-        st = lib.kvpop_decode_attention(dv["q"].data_ptr(), dv["k"].data_ptr(), dv["v"].data_ptr(),
-                                        dv["count"].data_ptr(), shape, scale, w_out.data_ptr(), w_lse.data_ptr(),
-                                        ws.data_ptr(), ws.numel(), stream)
-        assert st == B.OK, lib.kvpop_last_error()
+        free_after, _ = torch.cuda.mem_get_info()
+        assert free_after >= free_before, (shape.batch, free_before, free_after)
+        workspace_version(shape, scale, dv, ws, w_out, w_lse)
         torch.cuda.synchronize()
         for call, (out, lse) in enumerate(outs):
             what = f"batch {shape.batch}, capacity {shape.capacity}, call {call}"
             o, l = out.cpu().numpy(), lse.cpu().numpy()
             _check_against(o, l, w_out.cpu().numpy(), w_lse.cpu().numpy(), what + " vs workspace version")
             _check_against(o, l, ref_out, ref_lse, what + " vs oracle")
-    free_after, _ = torch.cuda.mem_get_info()
-    assert free_after >= free_before, (free_before, free_after)
 
 
 @pytest.mark.gpu
