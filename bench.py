@@ -35,7 +35,7 @@ METRIC = "future-attn target TFLOP/s & % BF16 tensor peak, Qwen3-8B shape, 16k c
 UNIT = "TFLOP/s"
 WORKLOAD = "qwen3_8b_16k"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["attn_kernels.cu", "kvpop_device.cuh", "kvpop_sched.h"]
+KERNEL_SOURCES = ["attn_kernels.cu", "kvpop_device.cuh", "kvpop_sched.h", "kvpop_debug.cuh"]
 
 
 def load_peaks():
@@ -459,8 +459,11 @@ def run_ours(args):
         extras["fused_single_launch"] = {
             "ms_per_step": ms_f, "value": fl["total"] / (ms_f * 1e-3) / 1e12, "unit": UNIT,
             "vs_two_launch_step": ms_per_step / ms_f,
-            "identical_to_two_launch": bool(torch.equal(tgt_f, tgt) and torch.equal(keep_f, keep)
-                                            and torch.equal(lse_f, lse)),
+            # one CTA per item here, CTA pairs in the two-launch step: the same lse bits, the targets
+            # equal up to fp32 rounding (a different grouping of each key's query tiles)
+            "lse_identical_to_two_launch": bool(torch.equal(lse_f, lse)),
+            "target_max_rel_diff_vs_two_launch": float(((tgt_f.double() - tgt.double()).abs()
+                                                        / tgt.double().abs().clamp_min(1e-3)).max()),
             "launches_per_step": 2}
         del ws_f, lse_f, tgt_f, keep_f
 

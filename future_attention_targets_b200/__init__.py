@@ -9,6 +9,8 @@ from ._binding import (  # noqa: F401
     KvpopError,
     check_status,
     compact_kv,
+    debug_selftest,
+    debug_set_word,
     decode_attention,
     decode_workspace_bytes,
     future_target,
@@ -25,7 +27,8 @@ from ._binding import (  # noqa: F401
     target_workspace_bytes,
 )
 
-__all__ = ["HostPipeline", "KvpopError", "check_status", "compact_kv", "decode_attention",
+__all__ = ["HostPipeline", "KvpopError", "check_status", "compact_kv", "debug_selftest", "debug_set_word",
+           "decode_attention",
            "decode_workspace_bytes", "future_target", "future_target_split", "future_targets", "future_targets_fused",
            "fused_workspace", "keep_mask", "lib", "prefix_topk_thresholds", "row_lse", "selftest_bounded_wait",
            "target_split_workspace_bytes", "target_workspace_bytes"]

@@ -18,9 +18,11 @@ PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG_DIR, "libkvpop.so")
 HEADER_PATH = os.path.join(os.path.dirname(PKG_DIR), "include", "kvpop.h")
 
-OK, INVALID_ARG, UNSUPPORTED, CUDA_ERROR, TIMEOUT = 0, 1, 2, 3, 4
+DEBUG_LIB_PATH = os.path.join(PKG_DIR, "libkvpop_debug.so")
+
+OK, INVALID_ARG, UNSUPPORTED, CUDA_ERROR, TIMEOUT, BOUNDS = 0, 1, 2, 3, 4, 5
 STATUS_NAMES = {OK: "KVPOP_OK", INVALID_ARG: "KVPOP_ERR_INVALID_ARG", UNSUPPORTED: "KVPOP_ERR_UNSUPPORTED",
-                CUDA_ERROR: "KVPOP_ERR_CUDA", TIMEOUT: "KVPOP_ERR_TIMEOUT"}
+                CUDA_ERROR: "KVPOP_ERR_CUDA", TIMEOUT: "KVPOP_ERR_TIMEOUT", BOUNDS: "KVPOP_ERR_BOUNDS"}
 
 
 class KvpopError(RuntimeError):
@@ -67,6 +69,8 @@ _SIGS = {
                                                  ctypes.c_int32, _I32P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
     "kvpop_check_device_status": (ctypes.c_int, [_P, _P]),
     "kvpop_selftest_bounded_wait": (ctypes.c_int, [_P, ctypes.c_uint64, _P]),
+    "kvpop_debug_set_word": (ctypes.c_int, [_P]),
+    "kvpop_debug_selftest": (ctypes.c_int, [_P, _P]),
     "kvpop_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "kvpop_last_error": (ctypes.c_char_p, []),
     "kvpop_abi_version": (ctypes.c_int32, []),
@@ -91,6 +95,18 @@ def lib() -> ctypes.CDLL:
                 fn.argtypes = args
             _handle = h
     return _handle
+
+
+def use_library(path: str) -> str:
+    """Makes later calls go to another build of the same C ABI (for example the
+    bounds-checking debug build, DEBUG_LIB_PATH); returns the previous path.
+    The library at `path` must exist: nothing falls back to anything else."""
+    global LIB_PATH, _handle
+    with _lock:
+        old = LIB_PATH
+        LIB_PATH, _handle = path, None
+    lib()
+    return old
 
 
 def header_symbols() -> list[str]:
@@ -477,3 +493,19 @@ def selftest_bounded_wait(status, limit_ns: int, stream=None) -> None:
     _on_current_device(status, "status")
     _check(lib().kvpop_selftest_bounded_wait(_status_ptr(status, status.device), int(limit_ns),
                                              _stream_ptr(stream)))
+
+
+def debug_set_word(word) -> None:
+    """Debug build: registers a zero-filled one-word int32 CUDA tensor that the kernels' bounds checks
+    write (None stops recording).  The ordinary build raises KVPOP_ERR_UNSUPPORTED."""
+    if word is None:
+        _check(lib().kvpop_debug_set_word(None))
+        return
+    _on_current_device(word, "word")
+    _check(lib().kvpop_debug_set_word(_status_ptr(word, word.device)))
+
+
+def debug_selftest(word, stream=None) -> None:
+    """Debug build: one kernel makes an index check that fails by design and records its code in word."""
+    _on_current_device(word, "word")
+    _check(lib().kvpop_debug_selftest(_status_ptr(word, word.device), _stream_ptr(stream)))

@@ -12,6 +12,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libkvpop.so")
+DEBUG_LIB = os.path.join(PKG, "libkvpop_debug.so")   # the same sources with KVPOP_DEBUG bounds checks
 
 NVCC_FLAGS = [
     "-std=c++17", "-O3", "-lineinfo",
@@ -32,30 +33,34 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) \
         + glob.glob(os.path.join(INCLUDE, "*.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None) -> str:
-    """Compiles every CUDA source into libkvpop.so (skipped when up to date)."""
-    if not force and not _stale():
-        return LIB
-    tmp = LIB + ".tmp"
-    cmd = [_nvcc(), *NVCC_FLAGS, *(extra_flags or []), "-I", INCLUDE, "-I", CSRC, "-shared",
+def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None,
+          debug: bool = False) -> str:
+    """Compiles every CUDA source into libkvpop.so, or with debug=True into libkvpop_debug.so (the same
+    sources with every kernel's bounds checks compiled in, KVPOP_DEBUG); skipped when up to date."""
+    lib = DEBUG_LIB if debug else LIB
+    if not force and not _stale(lib):
+        return lib
+    tmp = lib + ".tmp"
+    flags = [*NVCC_FLAGS, *(["-DKVPOP_DEBUG"] if debug else []), *(extra_flags or [])]
+    cmd = [_nvcc(), *flags, "-I", INCLUDE, "-I", CSRC, "-shared",
            *sources(), "-o", tmp, "-lcudart_static", "-ldl", "-lrt", "-lpthread"]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     force = "--force" in sys.argv
     extra = ["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else []
-    print(build(force=force or bool(extra), verbose=True, extra_flags=extra))
+    print(build(force=force or bool(extra), verbose=True, extra_flags=extra, debug="--debug" in sys.argv))

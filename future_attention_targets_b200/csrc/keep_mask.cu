@@ -19,6 +19,7 @@
 
 #include <algorithm>
 
+#include "kvpop_debug.cuh"
 #include "kvpop_sched.h"
 
 namespace kvpop {
@@ -57,21 +58,29 @@ __global__ void __launch_bounds__(kKeepThreads, 2) keep_mask_kernel(const __grid
   const int32_t s = p.seq_start[b], L = p.seq_len[b], B = p.budget[b];
   const float* score = p.score + static_cast<int64_t>(h) * p.total_tokens + s;
   uint8_t* keep = p.keep + static_cast<int64_t>(h) * p.total_tokens + s;
+  // Debug build: positions i of this row must lie inside [0, T) once offset by s.
+  auto in_row = [&](int32_t i, int32_t site) {
+    return KVPOP_IN(i >= 0 && i < L && s >= 0 && s + i < p.total_tokens, p.dbg, DBG_KEEP, site);
+  };
 
   // Every branch below depends only on (b, h): all CTAs of a cluster take it.
   if (L <= B) {
-    for (int32_t i = r * kKeepThreads + tid; i < L; i += kKeepCluster * kKeepThreads) keep[i] = 1;
+    for (int32_t i = r * kKeepThreads + tid; i < L; i += kKeepCluster * kKeepThreads)
+      if (in_row(i, 1)) keep[i] = 1;
     return;
   }
   const int32_t S = p.sinks, W = p.window;
   const int32_t lo = S, hi = L - W;          // candidates; hi > lo because L > B >= S + W
   const int32_t chunk = (hi - lo + kKeepCluster - 1) / kKeepCluster;
   const int32_t s0 = min(hi, lo + r * chunk), s1 = min(hi, s0 + chunk);
-  for (int32_t i = s0 + tid; i < s1; i += kKeepThreads) keys[i - s0] = order_key(__ldg(score + i));
+  for (int32_t i = s0 + tid; i < s1; i += kKeepThreads)
+    if (in_row(i, 2) && KVPOP_IN(i - s0 < p.key_cap, p.dbg, DBG_KEEP, 3)) keys[i - s0] = order_key(__ldg(score + i));
   if (r == 0)
-    for (int32_t i = tid; i < S; i += kKeepThreads) keep[i] = 1;
+    for (int32_t i = tid; i < S; i += kKeepThreads)
+      if (in_row(i, 4)) keep[i] = 1;
   if (r == kKeepCluster - 1)
-    for (int32_t i = hi + tid; i < L; i += kKeepThreads) keep[i] = 1;
+    for (int32_t i = hi + tid; i < L; i += kKeepThreads)
+      if (in_row(i, 4)) keep[i] = 1;
   __syncthreads();
 
   uint32_t need = static_cast<uint32_t>(B - S - W);  // rank (1-based) of the threshold among candidates
@@ -82,6 +91,7 @@ __global__ void __launch_bounds__(kKeepThreads, 2) keep_mask_kernel(const __grid
     for (int i = tid; i < kKeepWarps * 256; i += kKeepThreads) (&hist[0][0])[i] = 0;
     __syncthreads();
     for (int32_t i = tid; i < s1 - s0; i += kKeepThreads) {
+      if (!KVPOP_IN(i < p.key_cap, p.dbg, DBG_KEEP, 5)) break;
       const uint32_t u = keys[i];
       if ((u & pmask) == prefix) atomicAdd(&hist[warp][(u >> shift) & 255u], 1u);
     }
@@ -139,7 +149,8 @@ __global__ void __launch_bounds__(kKeepThreads, 2) keep_mask_kernel(const __grid
   const uint32_t tau = prefix, keep_eq = need;
   {
     uint32_t c = 0;
-    for (int32_t i = tid; i < s1 - s0; i += kKeepThreads) c += keys[i] == tau;
+    for (int32_t i = tid; i < s1 - s0 && KVPOP_IN(i < p.key_cap, p.dbg, DBG_KEEP, 5); i += kKeepThreads)
+      c += keys[i] == tau;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
     if (lane == 0) warp_tot[warp] = c;
@@ -155,7 +166,7 @@ __global__ void __launch_bounds__(kKeepThreads, 2) keep_mask_kernel(const __grid
   for (int q = 0; q < r; ++q) seen_eq += *cluster.map_shared_rank(&eq_count, q);
   for (int32_t base = s0; base < s1; base += kKeepThreads) {
     const int32_t i = base + tid;
-    const bool in = i < s1;
+    const bool in = i < s1 && KVPOP_IN(i - s0 < p.key_cap, p.dbg, DBG_KEEP, 5);
     const uint32_t u = in ? keys[i - s0] : 0u;
     const bool eq = in && u == tau;
     const uint32_t m = __ballot_sync(0xffffffffu, eq);
@@ -174,7 +185,7 @@ __global__ void __launch_bounds__(kKeepThreads, 2) keep_mask_kernel(const __grid
     }
     __syncthreads();
     const uint32_t rank = seen_eq + warp_off[warp] + __popc(m & ((1u << lane) - 1u));
-    if (in) keep[i] = (u > tau || (eq && rank < keep_eq)) ? 1 : 0;
+    if (in && in_row(i, 6)) keep[i] = (u > tau || (eq && rank < keep_eq)) ? 1 : 0;
     seen_eq += warp_off[kKeepWarps];
     __syncthreads();
   }
@@ -214,11 +225,13 @@ cudaError_t launch_keep_mask(const KeepParams& p, int n_kv_heads, int sm_count, 
   while (c < kKeepMaxCluster && (max_cand + c - 1) / c > kKeepSliceMax) c <<= 1;
   const int slice = (max_cand + c - 1) / c;
   const int smem = ((slice + 3) / 4) * 16;
+  KeepParams q = p;
+  q.key_cap = smem / 4;
   switch (c) {
-    case 1: return launch_keep_cluster<1>(p, n_kv_heads, smem, stream);
-    case 2: return launch_keep_cluster<2>(p, n_kv_heads, smem, stream);
-    case 4: return launch_keep_cluster<4>(p, n_kv_heads, smem, stream);
-    default: return launch_keep_cluster<8>(p, n_kv_heads, smem, stream);
+    case 1: return launch_keep_cluster<1>(q, n_kv_heads, smem, stream);
+    case 2: return launch_keep_cluster<2>(q, n_kv_heads, smem, stream);
+    case 4: return launch_keep_cluster<4>(q, n_kv_heads, smem, stream);
+    default: return launch_keep_cluster<8>(q, n_kv_heads, smem, stream);
   }
 }
 

@@ -10,6 +10,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -18,8 +19,8 @@
 #include "kvpop_cache.h"
 
 namespace kvpop {
-cudaError_t launch_row_lse(const AttnParams& p, int head_dim, int grid, cudaStream_t stream);
-cudaError_t launch_future_target(const AttnParams& p, int head_dim, int grid, cudaStream_t stream);
+cudaError_t launch_row_lse(const AttnParams& p, int head_dim, int sm_count, cudaStream_t stream);
+cudaError_t launch_future_target(const AttnParams& p, int head_dim, int sm_count, cudaStream_t stream);
 cudaError_t launch_keep_mask(const KeepParams& p, int n_kv_heads, int sm_count, cudaStream_t stream);
 cudaError_t launch_selftest_wait(int32_t* status, uint64_t limit_ns, cudaStream_t stream);
 cudaError_t launch_prefix_thresholds(const ThresholdParams& p, int n_kv_heads, int max_len, cudaStream_t stream);
@@ -27,12 +28,13 @@ cudaError_t launch_compact_kv(const CompactParams& p, cudaStream_t stream);
 cudaError_t launch_decode_attention(const DecodeParams& p, int batch, cudaStream_t stream);
 cudaError_t launch_fused_targets(const FusedParams& fp, int head_dim, int grid, cudaStream_t stream);
 cudaError_t launch_merge_partials(const float* part, float* target, int group, int n_kv_heads, int total_tokens,
-                                  int sm_count, cudaStream_t stream);
+                                  int sm_count, int32_t* dbg, cudaStream_t stream);
 int target_split_groups();
-cudaError_t launch_norm_rows(const float* lse, void* rows, int64_t n, float inv_scale, int sm_count,
+cudaError_t launch_norm_rows(const float* lse, void* rows, int64_t n, float inv_scale, int sm_count, int32_t* dbg,
                              cudaStream_t stream);
 size_t decode_scratch_bytes();
 cudaError_t decode_scratch_address(float** out);
+cudaError_t launch_debug_selftest(int32_t* word, cudaStream_t stream);
 }  // namespace kvpop
 
 using namespace kvpop;
@@ -40,6 +42,15 @@ using namespace kvpop;
 namespace {
 
 thread_local std::string g_last_error;
+
+// Debug build: the device word that kernels' bounds checks write
+// (kvpop_debug_set_word); every launch passes it in its parameter block.
+#ifdef KVPOP_DEBUG
+std::atomic<int32_t*> g_debug_word{nullptr};
+int32_t* debug_word() { return g_debug_word.load(std::memory_order_relaxed); }
+#else
+int32_t* debug_word() { return nullptr; }
+#endif
 
 // An NVTX range named after the entry point around its host work and
 // launches: Nsight tools show (and ncu can filter by) it when attached; a
@@ -146,6 +157,23 @@ kvpop_status make_map(CUtensorMap* m, const void* base, int64_t cols, int64_t ro
   return KVPOP_OK;
 }
 
+// Normaliser rows [n_heads][T] of 16 bytes (8 bf16 values each) read as boxes
+// of 128 rows of one head: rows past T read as 0 (CTA pairs, pass 2).
+kvpop_status make_rows_map(CUtensorMap* m, const void* rows, int64_t T, int64_t n_heads) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return fail(KVPOP_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
+  cuuint64_t dims[3] = {8, static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(n_heads)};
+  cuuint64_t strides[2] = {16, static_cast<cuuint64_t>(T) * 16};
+  cuuint32_t box[3] = {8, static_cast<cuuint32_t>(kTileRows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(rows), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(KVPOP_ERR_CUDA, "cuTensorMapEncodeTiled (normaliser rows) failed (CUresult %d)", static_cast<int>(r));
+  return KVPOP_OK;
+}
+
 // ---------------------------------------------------------------- validation
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -190,13 +218,14 @@ kvpop_status check_qk(const void* q, const void* k, float scale) {
 // ---------------------------------------------------------------- schedule
 
 // Items (level, sequence, head), heaviest level first.  Sequences with t
-// 128-row tiles take part in levels 0 .. t-1.
+// blocks of block_rows rows take part in levels 0 .. t-1.
 // order (optional) receives the original index of each scheduled sequence.
-void build_schedule(const int32_t* cu, int batch, int n_heads, LevelSchedule* s, std::vector<int>* order = nullptr) {
+void build_schedule(const int32_t* cu, int batch, int n_heads, LevelSchedule* s, std::vector<int>* order = nullptr,
+                    int block_rows = kTileRows) {
   std::vector<std::pair<int, int>> seqs;  // (tiles, index)
   for (int b = 0; b < batch; ++b) {
     const int L = cu[b + 1] - cu[b];
-    const int t = (L + kTileRows - 1) / kTileRows;
+    const int t = (L + block_rows - 1) / block_rows;
     if (t > 0) seqs.emplace_back(t, b);
   }
   std::stable_sort(seqs.begin(), seqs.end(), [](const std::pair<int, int>& a, const std::pair<int, int>& b) {
@@ -228,19 +257,24 @@ void build_schedule(const int32_t* cu, int batch, int n_heads, LevelSchedule* s,
 
 int grid_for(int items, int sm_count) { return std::max(1, std::min(items, sm_count)); }
 
+// cta = 1: one CTA per work item, resident (A) tiles of 128 rows and
+// streamed (B) tiles of 256; cta = 2: a CTA pair per item of 256 rows, each
+// CTA loading 128 rows of A and 128 rows of every B tile.
 kvpop_status fill_attn_common(AttnParams* p, const void* q, const void* k, const int32_t* cu,
                               const kvpop_shape& sh, float scale, bool target_pass,
-                              std::vector<int>* order = nullptr) {
+                              std::vector<int>* order = nullptr, int cta = 1) {
   memset(p, 0, sizeof(*p));
+  p->dbg = debug_word();
   const int64_t T = sh.total_tokens;
   kvpop_status st;
-  // Resident (A) tiles are 128 rows, streamed (B) tiles 256 rows.
+  const uint32_t a_rows = kTileRows, b_rows = kStreamRows / cta;
   if ((st = make_map(&p->tmap_q, q, static_cast<int64_t>(sh.n_q_heads) * sh.head_dim, T,
-                     target_pass ? kStreamRows : kTileRows)) != KVPOP_OK)
+                     target_pass ? b_rows : a_rows)) != KVPOP_OK)
     return st;
   if ((st = make_map(&p->tmap_k, k, static_cast<int64_t>(sh.n_kv_heads) * sh.head_dim, T,
-                     target_pass ? kTileRows : kStreamRows)) != KVPOP_OK)
+                     target_pass ? a_rows : b_rows)) != KVPOP_OK)
     return st;
+  p->cta = cta;
   p->wait_ns = wait_limit_ns();
   p->total_tokens = sh.total_tokens;
   p->n_q_heads = sh.n_q_heads;
@@ -249,9 +283,17 @@ kvpop_status fill_attn_common(AttnParams* p, const void* q, const void* k, const
   p->scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p->inv_scale = static_cast<float>(1.0 / static_cast<double>(scale));
   p->g_split = 1;
-  build_schedule(cu, sh.batch, target_pass ? sh.n_kv_heads : sh.n_q_heads, &p->sched, order);
+  build_schedule(cu, sh.batch, target_pass ? sh.n_kv_heads : sh.n_q_heads, &p->sched, order, kTileRows * cta);
   return KVPOP_OK;
 }
+
+// The standalone passes run on CTA pairs (cta = 2): each M = 256 MMA is
+// shared by two SMs, which halves the B tiles every SM reads from L2 and
+// feeds to its tensor core.  The single-launch variant keeps one CTA per SM.
+#ifndef KVPOP_PAIR_CTAS
+#define KVPOP_PAIR_CTAS 1
+#endif
+constexpr int kPassCtas = KVPOP_PAIR_CTAS ? 2 : 1;
 
 // 128-row tiles of every sequence (the lse readiness flags of the single
 // launch are one per query head and tile), -1 for a malformed cu_seqlens.
@@ -332,6 +374,7 @@ const char* kvpop_status_string(kvpop_status s) {
     case KVPOP_ERR_UNSUPPORTED: return "unsupported";
     case KVPOP_ERR_CUDA: return "CUDA error";
     case KVPOP_ERR_TIMEOUT: return "device wait timed out";
+    case KVPOP_ERR_BOUNDS: return "a bounds check of the debug build failed";
   }
   return "unknown status";
 }
@@ -349,12 +392,12 @@ static kvpop_status run_row_lse(const void* q, const void* k, const int32_t* cu_
                                 const DeviceInfo& dev) {
   AttnParams p;
   kvpop_status st;
-  if ((st = fill_attn_common(&p, q, k, cu_seqlens, shape, scale, false)) != KVPOP_OK) return st;
+  if ((st = fill_attn_common(&p, q, k, cu_seqlens, shape, scale, false, nullptr, kPassCtas)) != KVPOP_OK) return st;
   p.out = lse;
   p.nrm_rows = rows;
   p.status = dev_status;
   if (p.sched.total_items == 0) return KVPOP_OK;
-  cudaError_t e = launch_row_lse(p, shape.head_dim, grid_for(p.sched.total_items, dev.sm_count), stream);
+  cudaError_t e = launch_row_lse(p, shape.head_dim, dev.sm_count, stream);
   return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "row_lse launch");
 }
 
@@ -365,10 +408,13 @@ static kvpop_status run_target(const void* q, const void* k, const int32_t* cu_s
                                int32_t* dev_status, cudaStream_t stream, const DeviceInfo& dev) {
   AttnParams p;
   kvpop_status st;
-  if ((st = fill_attn_common(&p, q, k, cu_seqlens, shape, scale, true)) != KVPOP_OK) return st;
+  if ((st = fill_attn_common(&p, q, k, cu_seqlens, shape, scale, true, nullptr, kPassCtas)) != KVPOP_OK) return st;
+  if (kPassCtas == 2 &&
+      (st = make_rows_map(&p.tmap_rows, rows, shape.total_tokens, shape.n_q_heads)) != KVPOP_OK)
+    return st;
   const int G = shape.n_q_heads / shape.n_kv_heads;
   if (partials != nullptr) {
-    build_schedule(cu_seqlens, shape.batch, shape.n_kv_heads * G, &p.sched);
+    build_schedule(cu_seqlens, shape.batch, shape.n_kv_heads * G, &p.sched, nullptr, kTileRows * kPassCtas);
     p.g_split = G;
   }
   // A window longer than any sequence leaves every target at zero; clamp it
@@ -378,10 +424,11 @@ static kvpop_status run_target(const void* q, const void* k, const int32_t* cu_s
   p.out = partials != nullptr ? partials : target;
   p.status = dev_status;
   if (p.sched.total_items == 0) return KVPOP_OK;
-  cudaError_t e = launch_future_target(p, shape.head_dim, grid_for(p.sched.total_items, dev.sm_count), stream);
+  cudaError_t e = launch_future_target(p, shape.head_dim, dev.sm_count, stream);
   if (e != cudaSuccess) return cuda_fail(e, "future_target launch");
   if (partials == nullptr) return KVPOP_OK;
-  e = launch_merge_partials(partials, target, G, shape.n_kv_heads, shape.total_tokens, dev.sm_count, stream);
+  e = launch_merge_partials(partials, target, G, shape.n_kv_heads, shape.total_tokens, dev.sm_count, debug_word(),
+                            stream);
   return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "merge of the split partials");
 }
 
@@ -439,7 +486,7 @@ kvpop_status kvpop_future_target(const void* q, const void* k, const int32_t* cu
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   const float inv_scale = static_cast<float>(1.0 / static_cast<double>(scale));
   cudaError_t e = launch_norm_rows(lse, workspace, static_cast<int64_t>(shape.n_q_heads) * shape.total_tokens,
-                                   inv_scale, dev.sm_count, s);
+                                   inv_scale, dev.sm_count, debug_word(), s);
   if (e != cudaSuccess) return cuda_fail(e, "normaliser rows launch");
   return run_target(q, k, cu_seqlens, shape, scale, window, workspace, target, nullptr, dev_status, s, dev);
 }
@@ -473,7 +520,7 @@ kvpop_status kvpop_future_target_split(const void* q, const void* k, const int32
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   const float inv_scale = static_cast<float>(1.0 / static_cast<double>(scale));
   cudaError_t e = launch_norm_rows(lse, workspace, static_cast<int64_t>(shape.n_q_heads) * shape.total_tokens,
-                                   inv_scale, dev.sm_count, s);
+                                   inv_scale, dev.sm_count, debug_word(), s);
   if (e != cudaSuccess) return cuda_fail(e, "normaliser rows launch");
   float* partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kvpop_target_workspace_bytes(shape));
   return run_target(q, k, cu_seqlens, shape, scale, window, workspace, target, partials, dev_status, s, dev);
@@ -493,6 +540,7 @@ kvpop_status kvpop_keep_mask(const float* score, const int32_t* cu_seqlens, kvpo
   if ((st = device_info(&dev)) != KVPOP_OK) return st;
   KeepParams p;
   memset(&p, 0, sizeof(p));
+  p.dbg = debug_word();
   p.score = score;
   p.keep = keep;
   p.total_tokens = shape.total_tokens;
@@ -524,6 +572,7 @@ kvpop_status kvpop_prefix_topk_thresholds(const float* score, const int32_t* cu_
   if ((st = device_info(&dev)) != KVPOP_OK) return st;
   ThresholdParams p;
   memset(&p, 0, sizeof(p));
+  p.dbg = debug_word();
   p.score = score;
   p.thr_score = thr_score;
   p.thr_pos = thr_pos;
@@ -560,6 +609,7 @@ kvpop_status kvpop_compact_kv(const void* k, const void* v, const uint8_t* keep,
   if ((st = device_info(&dev)) != KVPOP_OK) return st;
   CompactParams p;
   memset(&p, 0, sizeof(p));
+  p.dbg = debug_word();
   p.k = static_cast<const uint16_t*>(k);
   p.v = static_cast<const uint16_t*>(v);
   p.keep = keep;
@@ -616,6 +666,7 @@ kvpop_status kvpop_decode_attention(const void* q, const void* k_cache, const vo
   if ((st = device_info(&dev)) != KVPOP_OK) return st;
   DecodeParams p;
   memset(&p, 0, sizeof(p));
+  p.dbg = debug_word();
   p.q = static_cast<const uint16_t*>(q);
   p.k_cache = static_cast<const uint16_t*>(k_cache);
   p.v_cache = static_cast<const uint16_t*>(v_cache);
@@ -660,6 +711,7 @@ kvpop_status kvpop_decode_attention_noalloc(const void* q, const void* k_cache, 
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the decode scratch");
   DecodeParams p;
   memset(&p, 0, sizeof(p));
+  p.dbg = debug_word();
   p.q = static_cast<const uint16_t*>(q);
   p.k_cache = static_cast<const uint16_t*>(k_cache);
   p.v_cache = static_cast<const uint16_t*>(v_cache);
@@ -908,6 +960,8 @@ kvpop_status kvpop_check_device_status(const int32_t* dev_status, void* stream) 
   if (v == 0) return KVPOP_OK;
   if ((v & 0xff) == KVPOP_ERR_TIMEOUT)
     return fail(KVPOP_ERR_TIMEOUT, "a kernel wait timed out (site %d)", (v >> 8) & 0xff);
+  if ((v & 0xff) == KVPOP_ERR_BOUNDS)
+    return fail(KVPOP_ERR_BOUNDS, "bounds check failed in kernel %d at site %d", (v >> 16) & 0xff, (v >> 8) & 0xff);
   return fail(KVPOP_ERR_CUDA, "device status word holds %d", v);
 }
 
@@ -919,6 +973,31 @@ kvpop_status kvpop_selftest_bounded_wait(int32_t* dev_status, uint64_t limit_ns,
   if ((st = device_info(&dev)) != KVPOP_OK) return st;
   cudaError_t e = launch_selftest_wait(dev_status, limit_ns, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "selftest launch");
+}
+
+kvpop_status kvpop_debug_set_word(int32_t* dev_word) {
+#ifdef KVPOP_DEBUG
+  g_debug_word.store(dev_word, std::memory_order_relaxed);
+  return KVPOP_OK;
+#else
+  (void)dev_word;
+  return fail(KVPOP_ERR_UNSUPPORTED, "this library was built without bounds checks (KVPOP_DEBUG)");
+#endif
+}
+
+kvpop_status kvpop_debug_selftest(int32_t* dev_word, void* stream) {
+#ifdef KVPOP_DEBUG
+  if (dev_word == nullptr) return fail(KVPOP_ERR_INVALID_ARG, "dev_word is NULL");
+  DeviceInfo dev;
+  kvpop_status st;
+  if ((st = device_info(&dev)) != KVPOP_OK) return st;
+  cudaError_t e = launch_debug_selftest(dev_word, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "debug self-test launch");
+#else
+  (void)dev_word;
+  (void)stream;
+  return fail(KVPOP_ERR_UNSUPPORTED, "this library was built without bounds checks (KVPOP_DEBUG)");
+#endif
 }
 
 }  // extern "C"

@@ -12,6 +12,7 @@ struct ThresholdParams {
   const float* score;     // [H_kv, T]
   float* thr_score;       // [H_kv, T]
   int32_t* thr_pos;       // [H_kv, T]
+  int32_t* dbg;           // debug build: bounds-check word, else unused
   int32_t total_tokens;
   int32_t window;
   int32_t sinks;
@@ -29,6 +30,7 @@ struct CompactParams {
   uint16_t* v_cache;
   int32_t* pos;             // [B, H_kv, C]
   int32_t* count;           // [B, H_kv]
+  int32_t* dbg;             // debug build: bounds-check word, else unused
   int32_t total_tokens, n_kv_heads, head_dim, capacity;
   int32_t n_seqs;
   int32_t seq_start[kMaxSeqs];
@@ -43,6 +45,7 @@ struct DecodeParams {
   float* partial;           // workspace [B, H_q, n_split, d + 2]: o[d], m, l
   float* out;               // [B, H_q, d]
   float* lse;               // [B, H_q] (may be null)
+  int32_t* dbg;             // debug build: bounds-check word, else unused
   int32_t n_q_heads, n_kv_heads, head_dim, capacity, n_split;
   float scale_log2;
 };

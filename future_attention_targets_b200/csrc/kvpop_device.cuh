@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "kvpop_debug.cuh"
 #include "kvpop_sched.h"
 
 namespace kvpop {
@@ -77,7 +78,13 @@ struct WaitCtl {
   volatile int* abort_flag;  // shared memory; set by the first wait that gives up
   int32_t* status;           // device status word (may be null)
   uint64_t limit_ns;         // per-wait time limit
+  volatile int* peer_abort = nullptr;  // CTA pairs: the other CTA's abort flag (distributed shared memory)
 };
+
+__device__ __forceinline__ void raise_abort(const WaitCtl& ctl) {
+  *ctl.abort_flag = 1;
+  if (ctl.peer_abort != nullptr) *ctl.peer_abort = 1;
+}
 
 // Waits for the phase of `bar` with parity `parity` to complete.  Returns
 // false when the CTA is aborting or the wait ran past its limit (then the
@@ -91,7 +98,7 @@ __device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const 
     if ((it & 15u) == 0u) {
       if (*ctl.abort_flag) return false;
       if (global_timer_ns() - t0 > ctl.limit_ns) {
-        *ctl.abort_flag = 1;
+        raise_abort(ctl);
         if (ctl.status != nullptr) atomicCAS(ctl.status, 0, 4 | (site << 8));
         return false;
       }
@@ -139,6 +146,57 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// CTA pairs (a cluster of two CTAs sharing one tcgen05 MMA): the same
+// shared-memory offset in the pair's first CTA.  A shared::cta address of
+// this CTA, used as a shared::cluster address, names this CTA's own memory;
+// clearing bit 24 names the first CTA's.
+constexpr uint32_t kPairLeaderMask = 0xFEFFFFFFu;
+__device__ __forceinline__ uint32_t leader_addr(const void* p) { return smem_u32(p) & kPairLeaderMask; }
+
+// 2-D tiled load into this CTA's shared memory whose completion bytes count
+// on the mbarrier at `bar`'s offset in the pair's first CTA (`.cta_group::2`).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, const uint64_t* bar, int32_t x,
+                                                 int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_addr(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// The same for a 3-D map (coordinates x, y, z).
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, const uint64_t* bar, int32_t x,
+                                                 int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_addr(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+// Arrive on the mbarrier at `bar`'s offset in the pair's first CTA.  Used to
+// hand an accumulator back after this warp's TMEM reads, which
+// tcgen05.wait::ld and tcgen05.fence::before_thread_sync already order; no
+// generic memory write needs releasing, so the arrive keeps its default
+// (CTA-scope) semantics: a cluster-scope release costs a memory barrier per
+// warp and tile.
+__device__ __forceinline__ void mbar_arrive_leader(const uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(leader_addr(bar)) : "memory");
+}
+
+// All threads of both CTAs of the cluster.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Generic pointer to the same shared-memory object in CTA `rank` of the cluster.
+template <class T>
+__device__ __forceinline__ T* cluster_map(T* p, uint32_t rank) {
+  uint64_t out;
+  asm volatile("mapa.u64 %0, %1, %2;" : "=l"(out) : "l"(reinterpret_cast<uint64_t>(p)), "r"(rank));
+  return reinterpret_cast<T*>(out);
+}
+
 // Contiguous bulk copy global -> shared: both addresses 16-byte aligned,
 // bytes a multiple of 16; completion counted in bytes on `bar`.
 __device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -149,16 +207,32 @@ __device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_
 
 // ------------------------------------------------------------------ tcgen05
 
+// kCta = 1: this CTA's TMEM; kCta = 2: the same columns in both CTAs of a
+// pair (issued by the same warp in each).
+template <int kCta = 1>
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
-               "r"(ncols)
-               : "memory");
+  if constexpr (kCta == 1)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+  else
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
 }
+template <int kCta = 1>
 __device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  if constexpr (kCta == 1)
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  else
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
 }
+template <int kCta = 1>
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+  if constexpr (kCta == 1)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+  else
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 __device__ __forceinline__ void tc_fence_before_sync() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -207,6 +281,30 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    smem_u32(bar))
                : "memory");
+}
+
+// CTA pairs: D[tmem] (+)= A * B^T with M = 256 (128 rows of A from each CTA's
+// shared memory), B's N rows split in halves between the two CTAs, and the
+// accumulator rows of each CTA in its own TMEM; issued by one thread of the
+// first CTA.
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// CTA pairs: arrive on the mbarrier at `bar`'s offset in both CTAs once every
+// tcgen05 operation issued so far by this thread has completed.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
 }
 
 // kW (16 or 32) consecutive fp32 columns of this thread's TMEM lane

@@ -32,6 +32,7 @@ struct LevelSchedule {
 struct AttnParams {
   CUtensorMap tmap_q;     // bf16 [T, H_q * d], box {64, rows}
   CUtensorMap tmap_k;     // bf16 [T, H_kv * d], box {64, rows}
+  CUtensorMap tmap_rows;  // CTA pairs, pass 2: normaliser rows [H_q][T][8 x bf16], box {8, 128, 1}
   void* nrm_rows;         // normaliser rows [H_q, T] x 16 bytes: pass 2 reads them, pass 1
                           // writes them when non-null (next to lse)
   float* out;             // pass 1: lse [H_q, T]; pass 2: target [H_kv, T]
@@ -45,6 +46,8 @@ struct AttnParams {
   float scale_log2;       // softmax scale * log2(e)
   float inv_scale;        // 1 / softmax scale (pass 2 normaliser slab)
   int32_t g_split;        // pass 2: 1 = an item covers the G query heads; G = one query head per item
+  int32_t cta;            // 1: one CTA per item (128-row blocks); 2: a CTA pair per item (256-row blocks)
+  int32_t* dbg;           // debug build: bounds-check word (kvpop_debug_set_word), else unused
   LevelSchedule sched;
 };
 
@@ -72,6 +75,8 @@ struct FusedParams {
 struct KeepParams {
   const float* score;     // [H_kv, T]
   uint8_t* keep;          // [H_kv, T]
+  int32_t* dbg;           // debug build: bounds-check word, else unused
+  int32_t key_cap;        // keys of one slice the shared-memory cache holds (set by the launcher)
   int32_t total_tokens;
   int32_t window;
   int32_t sinks;

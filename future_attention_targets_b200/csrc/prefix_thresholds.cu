@@ -28,6 +28,7 @@
 #include <stdint.h>
 
 #include "kvpop_cache.h"
+#include "kvpop_debug.cuh"
 
 namespace kvpop {
 
@@ -236,11 +237,16 @@ __global__ void __launch_bounds__(kThrThreads, 1) prefix_thresholds_kernel(const
   const float* score = p.score + static_cast<int64_t>(h) * p.total_tokens + s0;
   float* out_s = p.thr_score + static_cast<int64_t>(h) * p.total_tokens + s0;
   int32_t* out_p = p.thr_pos + static_cast<int64_t>(h) * p.total_tokens + s0;
+  // Debug build: a step or position t of this row lies inside the row and the [H_kv, T] arrays.
+  auto in_row = [&](int32_t t, int32_t site) {
+    return KVPOP_IN(t >= 0 && t < L && s0 >= 0 && s0 + t < p.total_tokens, p.dbg, DBG_THRESHOLDS, site);
+  };
 
   // Steps before the first candidate leaves the window: no eviction.
   if (c == 0) {
     const int32_t first = min(L, S + W);
     for (int32_t t = tid; t < first; t += kThrThreads) {
+      if (!in_row(t, 1)) continue;
       out_s[t] = -INFINITY;
       out_p[t] = -1;
     }
@@ -251,6 +257,7 @@ __global__ void __launch_bounds__(kThrThreads, 1) prefix_thresholds_kernel(const
   const int nb = min(kBlock, n - base);
   if (k == 0) {                                 // no scored slots: every candidate is evicted at once
     for (int32_t i = tid; i < nb; i += kThrThreads) {
+      if (!in_row(S + W + base + i, 1)) continue;
       out_s[S + W + base + i] = INFINITY;
       out_p[S + W + base + i] = -1;
     }
@@ -260,9 +267,13 @@ __global__ void __launch_bounds__(kThrThreads, 1) prefix_thresholds_kernel(const
   const int ksz = min(base, k);                 // |K|
   const bool cached = base <= kKeyCache;
   if (cached)
-    for (int32_t i = tid; i < base; i += kThrThreads) keys[i] = score_key(__ldg(score + S + i));
+    for (int32_t i = tid; i < base; i += kThrThreads)
+      if (in_row(S + i, 2) && KVPOP_IN(i < kKeyCache, p.dbg, DBG_THRESHOLDS, 3)) keys[i] = score_key(__ldg(score + S + i));
   __syncthreads();
-  auto key_at = [&](int32_t i) -> uint32_t { return cached ? keys[i] : score_key(__ldg(score + S + i)); };
+  auto key_at = [&](int32_t i) -> uint32_t {
+    if (cached) return KVPOP_IN(i >= 0 && i < kKeyCache, p.dbg, DBG_THRESHOLDS, 3) ? keys[i] : 0u;
+    return in_row(S + i, 2) ? score_key(__ldg(score + S + i)) : 0u;
+  };
 
   // ---- 1. K's minimum: the ksz-th largest key of the prefix.
   const uint64_t kmin = (ksz > 0) ? select_rank(key_at, base, static_cast<uint32_t>(ksz), S, sh) : 0ull;
@@ -271,7 +282,7 @@ __global__ void __launch_bounds__(kThrThreads, 1) prefix_thresholds_kernel(const
   const uint64_t tau = (ksz >= k) ? kmin : 0ull;      // every key is > 0
   uint64_t v = 0;
   bool beats = false;
-  if (tid < nb) {
+  if (tid < nb && in_row(S + base + tid, 2)) {
     v = compose_key(score_key(__ldg(score + S + base + tid)), S + base + tid);
     beats = v > tau;
   }
@@ -279,8 +290,9 @@ __global__ void __launch_bounds__(kThrThreads, 1) prefix_thresholds_kernel(const
   const int d_j = block_rank(beats, warp_tot, &d_total);   // inclusive
   int np2 = 1;
   while (np2 < d_total) np2 <<= 1;
-  if (beats) dsort[d_j - 1] = v;
-  for (int i = d_total + tid; i < np2; i += kThrThreads) dsort[i] = ~0ull;
+  if (beats && KVPOP_IN(d_j >= 1 && d_j <= kBlock, p.dbg, DBG_THRESHOLDS, 4)) dsort[d_j - 1] = v;
+  for (int i = d_total + tid; i < np2; i += kThrThreads)
+    if (KVPOP_IN(i < kBlock, p.dbg, DBG_THRESHOLDS, 4)) dsort[i] = ~0ull;
   __syncthreads();
   bitonic_sort(dsort, np2);
 
@@ -305,7 +317,8 @@ __global__ void __launch_bounds__(kThrThreads, 1) prefix_thresholds_kernel(const
     __syncthreads();
     int bp2 = 1;
     while (bp2 < m) bp2 <<= 1;
-    for (int i = m + tid; i < bp2; i += kThrThreads) band[i] = ~0ull;
+    for (int i = m + tid; i < bp2; i += kThrThreads)
+      if (KVPOP_IN(i < kSortMax, p.dbg, DBG_THRESHOLDS, 5)) band[i] = ~0ull;
     __syncthreads();
     bitonic_sort(band, bp2);
   }
@@ -317,15 +330,18 @@ __global__ void __launch_bounds__(kThrThreads, 1) prefix_thresholds_kernel(const
   const int n_padded = (n_merged + 7) & ~7;
   for (int a = tid; a < m; a += kThrThreads) {
     const int at = a + lower_bound_u64(dsort, d_total, band[a]);
+    if (!KVPOP_IN(at >= 0 && at < kMergedMax, p.dbg, DBG_THRESHOLDS, 6)) continue;
     merged[at] = band[a];
     tags[at] = -1;
   }
   for (int r = tid; r < d_total; r += kThrThreads) {
     const int at = r + lower_bound_u64(band, m, dsort[r]);
+    if (!KVPOP_IN(at >= 0 && at < kMergedMax, p.dbg, DBG_THRESHOLDS, 6)) continue;
     merged[at] = dsort[r];
     tags[at] = static_cast<int16_t>(key_pos(dsort[r]) - (S + base));
   }
-  for (int i = n_merged + tid; i < n_padded; i += kThrThreads) tags[i] = kNeverTag;
+  for (int i = n_merged + tid; i < n_padded; i += kThrThreads)
+    if (KVPOP_IN(i < kMergedMax, p.dbg, DBG_THRESHOLDS, 6)) tags[i] = kNeverTag;
   __syncthreads();
 
   // ---- 4. threshold of this thread's step: its rank among the entries
@@ -333,14 +349,15 @@ __global__ void __launch_bounds__(kThrThreads, 1) prefix_thresholds_kernel(const
   if (tid < nb) {
     const int t = S + W + base + tid;
     const int total = ksz + d_j;
-    if (total < k) {
+    if (!in_row(t, 1)) {
+    } else if (total < k) {
       out_s[t] = -INFINITY;
       out_p[t] = -1;
     } else {
       const int want = total - k + 1;
       const uint32_t me2 = (static_cast<uint32_t>(tid) & 0xffffu) * 0x10001u;   // this step in both halves
       int cnt = 0, i = 0;
-      for (; i < n_padded; i += 8) {
+      for (; i < n_padded && KVPOP_IN(i + 8 <= kMergedMax, p.dbg, DBG_THRESHOLDS, 7); i += 8) {
         const uint4 w = *reinterpret_cast<const uint4*>(tags + i);
         const int here = (__popc(__vcmples2(w.x, me2)) + __popc(__vcmples2(w.y, me2)) +
                           __popc(__vcmples2(w.z, me2)) + __popc(__vcmples2(w.w, me2))) >> 4;
@@ -348,7 +365,7 @@ __global__ void __launch_bounds__(kThrThreads, 1) prefix_thresholds_kernel(const
         cnt += here;
       }
       uint64_t x = 0;
-      for (int q = 0; q < 8; ++q) {
+      for (int q = 0; q < 8 && KVPOP_IN(i + q < kMergedMax, p.dbg, DBG_THRESHOLDS, 7); ++q) {
         if (tags[i + q] <= tid && ++cnt == want) {
           x = merged[i + q];
           break;

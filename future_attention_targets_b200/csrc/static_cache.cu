@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "kvpop_cache.h"
+#include "kvpop_debug.cuh"
 
 namespace kvpop {
 
@@ -121,13 +122,15 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_kv_kernel(const __
 
   const int chunk = (L + kCompactThreads - 1) / kCompactThreads;
   const int c0 = min(L, tid * chunk), c1 = min(L, c0 + chunk);
+  // Debug build: the mask row [s0, s0 + L) of head h lies inside [H_kv, T].
+  KVPOP_CHECK(s0 >= 0 && s0 + L <= p.total_tokens && h < p.n_kv_heads, p.dbg, DBG_COMPACT, 1);
   const int mine = count_kept(mask, c0, c1);
   int total = 0;
   const int first = block_exclusive_scan(mine, warp_sums, &total);
   if (first < S1 && first + mine > S0) {
     int slot = first;
     for_each_kept(mask, c0, c1, [&](int i) {
-      if (slot >= S0 && slot < S1) list_pos[slot - S0] = i;
+      if (slot >= S0 && slot < S1 && KVPOP_IN(slot - S0 < kCompactSlots, p.dbg, DBG_COMPACT, 2)) list_pos[slot - S0] = i;
       ++slot;
     });
   }
@@ -147,7 +150,10 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_kv_kernel(const __
         const bool is_v = rem >= kWords;
         const int w = is_v ? rem - kWords : rem;
         const int64_t src = (static_cast<int64_t>(s0 + list_pos[e]) * p.n_kv_heads + h) * d + w * 8;
-        buf[u] = __ldg(reinterpret_cast<const uint4*>((is_v ? p.v : p.k) + src));
+        buf[u] = KVPOP_IN(list_pos[e] >= 0 && list_pos[e] < L && s0 + list_pos[e] < p.total_tokens, p.dbg,
+                          DBG_COMPACT, 3)
+                     ? __ldg(reinterpret_cast<const uint4*>((is_v ? p.v : p.k) + src))
+                     : make_uint4(0, 0, 0, 0);
       }
     }
 #pragma unroll
@@ -157,20 +163,24 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_kv_kernel(const __
         const int e = idx / kRowWords, rem = idx - e * kRowWords;
         const bool is_v = rem >= kWords;
         const int w = is_v ? rem - kWords : rem;
-        *reinterpret_cast<uint4*>((is_v ? p.v_cache : p.k_cache) + (row0 + S0 + e) * d + w * 8) = buf[u];
+        if (KVPOP_IN(S0 + e < p.capacity, p.dbg, DBG_COMPACT, 4))
+          *reinterpret_cast<uint4*>((is_v ? p.v_cache : p.k_cache) + (row0 + S0 + e) * d + w * 8) = buf[u];
       }
     }
   }
   // Slot positions (-1 when unused) and zeros in the unused rows.
-  for (int e = tid; e < S1 - S0; e += kCompactThreads) p.pos[row0 + S0 + e] = (e < n_fill) ? list_pos[e] : -1;
+  for (int e = tid; e < S1 - S0; e += kCompactThreads)
+    if (KVPOP_IN(S0 + e < p.capacity && e < kCompactSlots, p.dbg, DBG_COMPACT, 5))
+      p.pos[row0 + S0 + e] = (e < n_fill) ? list_pos[e] : -1;
   const int clear_words = (S1 - S0 - n_fill) * kWords;
+  KVPOP_CHECK(S0 + n_fill + clear_words / kWords <= p.capacity, p.dbg, DBG_COMPACT, 4);
   uint4* kz = reinterpret_cast<uint4*>(p.k_cache + (row0 + S0 + n_fill) * d);
   uint4* vz = reinterpret_cast<uint4*>(p.v_cache + (row0 + S0 + n_fill) * d);
   for (int i = tid; i < clear_words; i += kCompactThreads) {
     kz[i] = make_uint4(0, 0, 0, 0);
     vz[i] = make_uint4(0, 0, 0, 0);
   }
-  if (c == 0 && tid == 0) p.count[b * p.n_kv_heads + h] = total;
+  if (c == 0 && tid == 0 && KVPOP_IN(b < p.n_seqs, p.dbg, DBG_COMPACT, 6)) p.count[b * p.n_kv_heads + h] = total;
 }
 
 cudaError_t launch_compact_kv(const CompactParams& p, cudaStream_t stream) {
@@ -265,10 +275,13 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
   const int rows = max(0, min(kDecRowsPerWarp, n - w_lo));
   uint16_t* sk = dec_smem + warp * kDecRowsPerWarp * HD;
   uint16_t* sv = dec_smem + kDecSplit * HD + warp * kDecRowsPerWarp * HD;
+  [[maybe_unused]] const int batch = static_cast<int>(gridDim.x) / p.n_kv_heads;
   {
     const int64_t g0 = ((static_cast<int64_t>(b) * p.n_kv_heads + h) * p.capacity + w_lo) * HD;
     for (int idx = lane; idx < rows * kChunks; idx += 32) {
       const int r = idx / kChunks, c = idx - r * kChunks;
+      // Debug build: the staged row is one of this (sequence, KV head)'s filled slots.
+      if (!KVPOP_IN(w_lo + r < p.capacity && r < kDecRowsPerWarp && b < batch, p.dbg, DBG_DECODE, 1)) continue;
       cp_async16(swz<HD>(sk, r, c), p.k_cache + g0 + idx * 8);
       cp_async16(swz<HD>(sv, r, c), p.v_cache + g0 + idx * 8);
     }
@@ -283,6 +296,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
   // q as the A operand: rows = query heads (>= G read as 0), cols = head dims.
   uint32_t qa[KS][4];
   {
+    KVPOP_CHECK(h * G + G <= p.n_q_heads && G <= 16, p.dbg, DBG_DECODE, 2);
     const uint16_t* qb = p.q + (static_cast<int64_t>(b) * p.n_q_heads + h * G) * HD;
 #pragma unroll
     for (int kk = 0; kk < KS; ++kk) {
@@ -413,7 +427,11 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
         oo += so[(w * G + g) * HD + e] * c;
       }
     }
-    float* dst = p.partial + ((static_cast<int64_t>(b) * p.n_q_heads + h * G + g) * p.n_split + split) * (HD + 2);
+    const int64_t at = ((static_cast<int64_t>(b) * p.n_q_heads + h * G + g) * p.n_split + split) * (HD + 2);
+    if (!KVPOP_IN(split < p.n_split && at + HD + 2 <= static_cast<int64_t>(batch) * p.n_q_heads * p.n_split * (HD + 2),
+                  p.dbg, DBG_DECODE, 3))
+      continue;
+    float* dst = p.partial + at;
     dst[e] = oo;
     if (e == 0) {
       dst[HD] = mm;
@@ -457,7 +475,8 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
     const int bg = blockIdx.x, tid = threadIdx.x;
     const int d = p.head_dim, ns = p.n_split, stride = d + 2, half = stride / 2;
     const float2* part = reinterpret_cast<const float2*>(p.partial + static_cast<int64_t>(bg) * ns * stride);
-    for (int i = tid; i < ns * half; i += 128) staged[i] = part[i];     // every load issued before any use
+    for (int i = tid; i < ns * half; i += 128)                          // every load issued before any use
+      if (KVPOP_IN(i < kCombineStagedSplits * 65 && (stride & 1) == 0, p.dbg, DBG_COMBINE, 1)) staged[i] = part[i];
     __syncthreads();
     const float* st = reinterpret_cast<const float*>(staged);
     if (tid < 32) {
@@ -484,7 +503,8 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
     for (int e = tid; e < d; e += 128) {
       float oo = 0.f;
       for (int s2 = 0; s2 < ns; ++s2) oo = fmaf(st[s2 * stride + e], wsm[s2], oo);
-      p.out[static_cast<int64_t>(bg) * d + e] = (ll > 0.f) ? oo / ll : 0.f;
+      if (KVPOP_IN(bg < static_cast<int>(gridDim.x) && e < d, p.dbg, DBG_COMBINE, 2))
+        p.out[static_cast<int64_t>(bg) * d + e] = (ll > 0.f) ? oo / ll : 0.f;
     }
     if (tid == 0 && p.lse != nullptr) p.lse[bg] = (ll > 0.f) ? (mm + log2f(ll)) * 0.6931471805599453f : -INFINITY;
     return;
@@ -495,6 +515,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
   const int bg = blockIdx.x, tid = threadIdx.x;
   const int d = p.head_dim, ns = p.n_split, stride = d + 2;
   const float* part = p.partial + static_cast<int64_t>(bg) * ns * stride;
+  KVPOP_CHECK(ns > kCombineStagedSplits && d <= 128, p.dbg, DBG_COMBINE, 3);
   // Split maxima, their maximum, then each split's weight exp2(m_s - m) and the total sum.
   float mm = -INFINITY;
   for (int s = tid; s < ns; s += 128) mm = fmaxf(mm, part[s * stride + d]);

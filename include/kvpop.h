@@ -64,7 +64,7 @@
 extern "C" {
 #endif
 
-#define KVPOP_ABI_VERSION 2
+#define KVPOP_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define KVPOP_API __attribute__((visibility("default")))
@@ -77,7 +77,8 @@ typedef enum {
   KVPOP_ERR_INVALID_ARG = 1,   /* null pointer, bad size, inconsistent cu_seqlens, ... */
   KVPOP_ERR_UNSUPPORTED = 2,   /* head_dim not 64/128, too many sequences or tokens, non-sm_100 device */
   KVPOP_ERR_CUDA = 3,          /* CUDA runtime error (launch, copy, device query) */
-  KVPOP_ERR_TIMEOUT = 4        /* a kernel's bounded on-chip wait ran out (from kvpop_check_device_status) */
+  KVPOP_ERR_TIMEOUT = 4,       /* a kernel's bounded on-chip wait ran out (from kvpop_check_device_status) */
+  KVPOP_ERR_BOUNDS = 5         /* debug build only: a kernel's index check failed (see kvpop_debug_set_word) */
 } kvpop_status;
 
 /* Problem shape.  cu_seqlens (host memory, int32 [batch + 1]) holds the packed
@@ -98,6 +99,12 @@ typedef struct {
  *   scale       softmax scale s (finite, > 0; 1/sqrt(head_dim) for the workloads)
  *   lse         device fp32 [n_q_heads, T], written for every (g, i)
  *   dev_status  device int32 or NULL; receives a nonzero code if a wait times out
+ * Accuracy: the exponentials are fp32, 5 of every 16 from a degree-3
+ * polynomial (relative error at most 8.6e-5), the rest from the hardware
+ * exp2; sums in fp32.  |lse - exact| stays within 2e-4 (tested on every row
+ * of the workloads and edge shapes); a target moves by about that relative
+ * amount, well inside its 2e-3 bound.
+ * Runs as CTA pairs: each M = 256 MMA is shared by two SMs.
  */
 KVPOP_API kvpop_status kvpop_row_lse(const void* q, const void* k, const int32_t* cu_seqlens,
                            kvpop_shape shape, float scale, float* lse,
@@ -331,6 +338,26 @@ KVPOP_API kvpop_status kvpop_check_device_status(const int32_t* dev_status, void
  * and writes its timeout code into *dev_status.  Used by the tests to show a
  * wait that runs out ends in an error status, not a hang. */
 KVPOP_API kvpop_status kvpop_selftest_bounded_wait(int32_t* dev_status, uint64_t limit_ns, void* stream);
+
+/* Bounds checks of the debug build (libkvpop_debug.so, the same sources
+ * compiled with KVPOP_DEBUG; future_attention_targets_b200/build.py builds
+ * it beside libkvpop.so).  There, every kernel checks the index of each
+ * data-dependent global or shared-memory access against the extent it may
+ * touch before making it; a failed check skips the access (nothing traps)
+ * and writes, if the word is still 0,
+ *   KVPOP_ERR_BOUNDS | check site << 8 | kernel << 16
+ * into the device word registered here.  One word per process, used by
+ * every later launch on any device until replaced (NULL stops recording);
+ * it must be device memory of the device the kernels run on, zero-filled
+ * by the caller, and read after the launches finish (or passed to
+ * kvpop_check_device_status).  Not part of the method: a testing aid.
+ * The ordinary library returns KVPOP_ERR_UNSUPPORTED from both calls. */
+KVPOP_API kvpop_status kvpop_debug_set_word(int32_t* dev_word);
+
+/* Debug build: one kernel makes a single index check that fails by design
+ * (an index one past the extent it declares; the access it guards is
+ * skipped) so that a test can see the code arrive in *dev_word. */
+KVPOP_API kvpop_status kvpop_debug_selftest(int32_t* dev_word, void* stream);
 
 KVPOP_API const char* kvpop_status_string(kvpop_status status);
 KVPOP_API const char* kvpop_last_error(void);

@@ -17,17 +17,23 @@ def lib():
 
 def test_exports_every_header_symbol(lib):
     names = B.header_symbols()
-    assert len(names) == 21, names
+    assert len(names) == 23, names
     for name in names:
         assert hasattr(lib, name), f"{name} declared in kvpop.h but not exported"
     assert set(names) == set(B._SIGS), "binding signatures and header disagree"
 
 
 def test_version_and_strings(lib):
-    assert lib.kvpop_abi_version() == 2
+    assert lib.kvpop_abi_version() == 3
     for code, word in [(0, b"ok"), (1, b"invalid argument"), (2, b"unsupported"), (3, b"CUDA error"),
-                       (4, b"device wait timed out")]:
+                       (4, b"device wait timed out"), (5, b"a bounds check of the debug build failed")]:
         assert lib.kvpop_status_string(code) == word
+
+
+def test_ordinary_build_has_no_bounds_checks(lib):
+    """The debug calls exist in every build; the ordinary library refuses them before touching a device."""
+    assert lib.kvpop_debug_set_word(FAKE) == B.UNSUPPORTED
+    assert lib.kvpop_debug_selftest(FAKE, None) == B.UNSUPPORTED
 
 
 FAKE = 0x10000  # never dereferenced: every call below fails validation first

@@ -22,4 +22,4 @@ def test_c99_client_builds_links_and_passes(tmp_path):
                     f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True, capture_output=True, text=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert out.returncode == 0, out.stdout + out.stderr
-    assert "c client ok: abi 2" in out.stdout
+    assert "c client ok: abi 3" in out.stdout

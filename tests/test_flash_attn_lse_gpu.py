@@ -19,7 +19,7 @@ from future_attention_targets_b200.workloads import make_inputs
 pytestmark = pytest.mark.gpu
 flash_attn = pytest.importorskip("flash_attn")
 
-LSE_TOL = 1e-4
+LSE_TOL = 2e-4   # the row logsumexp's own bound (see test_parity_gpu)
 
 
 @pytest.mark.parametrize("name", ["qwen3_4b_4k", "qwen3_8b_16k", "varlen_8x"])

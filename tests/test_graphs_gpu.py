@@ -79,8 +79,13 @@ def test_attention_pipeline_in_a_graph(fused):
         q.copy_(dev(other["q_bits"]))
         k.copy_(dev(other["k_bits"]))
 
-    # The eager reference runs the plain device pipeline on separate outputs.
+    # The eager reference runs the same entry point on separate outputs (and, for the single launch, its own
+    # workspace).
+    ws_eager = fused_workspace(cu, w.n_q_heads, w.n_kv_heads, w.head_dim) if fused else None
+
     def eager():
+        if fused:
+            return future_targets_fused(q, k, cu, W, S, budgets, scale=scale, workspace=ws_eager)
         return future_targets(q, k, cu, W, S, budgets, scale=scale)
 
     _replays_match(graph, eager, (lse, tgt, keep), refill, status)

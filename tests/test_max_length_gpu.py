@@ -25,7 +25,7 @@ pytestmark = pytest.mark.gpu
 L_MAX = 131072
 HQ, HKV, D = 2, 1, 64
 TARGET_TOL = 2e-3
-LSE_TOL = 1e-4
+LSE_TOL = 2e-4   # the row logsumexp's bound (see test_parity_gpu)
 
 
 def dev(bits):
