@@ -26,6 +26,7 @@ cudaError_t launch_selftest_wait(int32_t* status, uint64_t limit_ns, cudaStream_
 cudaError_t launch_prefix_thresholds(const ThresholdParams& p, int n_kv_heads, int max_len, cudaStream_t stream);
 cudaError_t launch_compact_kv(const CompactParams& p, cudaStream_t stream);
 cudaError_t launch_decode_attention(const DecodeParams& p, int batch, cudaStream_t stream);
+int decode_parts(int rows, int n_chunks, int sm_count);
 cudaError_t launch_fused_targets(const FusedParams& fp, int head_dim, int grid, cudaStream_t stream);
 cudaError_t launch_merge_partials(const float* part, float* target, int group, int n_kv_heads, int total_tokens,
                                   int sm_count, int32_t* dbg, cudaStream_t stream);
@@ -678,7 +679,7 @@ kvpop_status kvpop_decode_attention(const void* q, const void* k_cache, const vo
   p.n_kv_heads = shape.n_kv_heads;
   p.head_dim = shape.head_dim;
   p.capacity = shape.capacity;
-  p.n_split = (shape.capacity + kDecSplit - 1) / kDecSplit;
+  p.n_split = decode_parts(shape.batch * shape.n_kv_heads, (shape.capacity + kDecSplit - 1) / kDecSplit, dev.sm_count);
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   cudaError_t e = launch_decode_attention(p, shape.batch, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "decode attention launch");
@@ -723,7 +724,7 @@ kvpop_status kvpop_decode_attention_noalloc(const void* q, const void* k_cache, 
   p.n_kv_heads = shape.n_kv_heads;
   p.head_dim = shape.head_dim;
   p.capacity = shape.capacity;
-  p.n_split = (shape.capacity + kDecSplit - 1) / kDecSplit;
+  p.n_split = decode_parts(shape.batch * shape.n_kv_heads, (shape.capacity + kDecSplit - 1) / kDecSplit, dev.sm_count);
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   e = launch_decode_attention(p, shape.batch, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? KVPOP_OK : cuda_fail(e, "decode attention launch");

@@ -10,6 +10,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "kvpop_cache.h"
@@ -245,51 +246,74 @@ __device__ __forceinline__ uint16_t* swz(uint16_t* base, int r, int c) {
   return base + r * HD + ((c ^ (r & 7)) << 3);
 }
 
-// One CTA: KV head h of sequence b, cache slots [split * kDecSplit, ...), all
-// G <= 16 query heads of the group.  Each warp stages its 32 rows of K and V
-// in shared memory with one burst of cp.async (rows past the filled slots
-// are zeroed so 0 x garbage cannot make a NaN), then:
+// One CTA: KV head h of sequence b, all G <= 16 query heads of its group, over
+// a contiguous range of the filled 128-slot chunks of its cache row (the
+// whole row when there are enough rows to fill the GPU; otherwise the row is
+// split over p.n_split CTAs whose partials a merge kernel combines).  Each of
+// the four warps owns 32 slots of every chunk and streams its slices through
+// a ring of kDecStages shared-memory buffers with cp.async, two chunks ahead
+// of the one it computes (rows past the filled slots are zeroed so that
+// 0 x garbage cannot make a NaN).  Per chunk:
 //   S = Q K^T   16 (heads, padded) x 32 keys, fp32, by MMA (q unscaled bf16,
 //               the scale applied to S in fp32)
-//   softmax     per head over its 32 keys (rows of S live on four lanes)
-//   O = P V     16 x d, P split into bf16 high and low parts (two MMAs) so the
+//   softmax     a running max and sum per head over the warp's keys so far
+//               (rows of S live on four lanes); O is rescaled when the max grows
+//   O += P V    16 x d, P split into bf16 high and low parts (two MMAs) so the
 //               product keeps ~16 bits of P
-// and the four warps' (max, sum, O) are merged in shared memory into this
-// split's partial.
-template <int HD>
+// and at the end the four warps' (max, sum, O) are merged in shared memory
+// into the output (one CTA per row) or this CTA's partial.  kDecStages
+// buffers (kDecStages - 1 chunks in flight while one is computed) when a CTA
+// streams several chunks; one buffer when it has a single chunk, which leaves
+// room for three CTAs per SM.
+template <int HD, int kDecStages>
 __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int kChunks = HD / 8;      // 16-byte chunks per row
   constexpr int KS = HD / 16;          // k-steps of S = Q K^T
   constexpr int NT = HD / 8;           // 8-column tiles of O
-  extern __shared__ __align__(16) uint16_t dec_smem[];     // K rows [kDecSplit][HD], then V rows (swizzled)
+  constexpr int kWarpStage = 2 * kDecRowsPerWarp * HD;     // bf16 elements: a warp's K then V rows of one chunk
+  extern __shared__ __align__(16) uint16_t dec_smem[];     // [warp][stage] K rows, V rows (swizzled)
   __shared__ float sm_m[kDecThreads / 32][16];
   __shared__ float sm_l[kDecThreads / 32][16];
 
-  const int bh = blockIdx.x, split = blockIdx.y;
+  const int bh = blockIdx.x, part = blockIdx.y;
   const int b = bh / p.n_kv_heads, h = bh - b * p.n_kv_heads;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gid = lane >> 2, tid4 = lane & 3;
   const int G = p.n_q_heads / p.n_kv_heads;
-  const int n = min(p.count[b * p.n_kv_heads + h], p.capacity);
-  const int w_lo = split * kDecSplit + warp * kDecRowsPerWarp;
-  const int rows = max(0, min(kDecRowsPerWarp, n - w_lo));
-  uint16_t* sk = dec_smem + warp * kDecRowsPerWarp * HD;
-  uint16_t* sv = dec_smem + kDecSplit * HD + warp * kDecRowsPerWarp * HD;
   [[maybe_unused]] const int batch = static_cast<int>(gridDim.x) / p.n_kv_heads;
-  {
-    const int64_t g0 = ((static_cast<int64_t>(b) * p.n_kv_heads + h) * p.capacity + w_lo) * HD;
+  const int n = min(p.count[b * p.n_kv_heads + h], p.capacity);
+  // This CTA's chunks: its share of the chunk range, cut at the filled slots.
+  const int n_chunks = (p.capacity + kDecSplit - 1) / kDecSplit;
+  const int per_part = (n_chunks + p.n_split - 1) / p.n_split;
+  const int c_lo = part * per_part;
+  const int c_hi = min(min(c_lo + per_part, n_chunks), (n + kDecSplit - 1) / kDecSplit);
+  const int nch = max(0, c_hi - c_lo);
+  uint16_t* wbase = dec_smem + warp * kDecStages * kWarpStage;
+  const int64_t row_base = (static_cast<int64_t>(b) * p.n_kv_heads + h) * p.capacity;
+
+  // Issues the cp.async copies of this warp's rows of chunk c_lo + k into stage k % kDecStages.
+  auto stage_in = [&](int k) {
+    const int w_lo = (c_lo + k) * kDecSplit + warp * kDecRowsPerWarp;
+    const int rows = max(0, min(kDecRowsPerWarp, n - w_lo));
+    uint16_t* sk = wbase + (k % kDecStages) * kWarpStage;
+    uint16_t* sv = sk + kDecRowsPerWarp * HD;
+    const int64_t g0 = (row_base + w_lo) * HD;
     for (int idx = lane; idx < rows * kChunks; idx += 32) {
       const int r = idx / kChunks, c = idx - r * kChunks;
       // Debug build: the staged row is one of this (sequence, KV head)'s filled slots.
-      if (!KVPOP_IN(w_lo + r < p.capacity && r < kDecRowsPerWarp && b < batch, p.dbg, DBG_DECODE, 1)) continue;
+      if (!KVPOP_IN(w_lo + r < p.capacity && w_lo + r < n && b < batch, p.dbg, DBG_DECODE, 1)) continue;
       cp_async16(swz<HD>(sk, r, c), p.k_cache + g0 + idx * 8);
       cp_async16(swz<HD>(sv, r, c), p.v_cache + g0 + idx * 8);
     }
+  };
+  // Chunks in flight ahead of the one being computed (a single buffer takes its
+  // one chunk here too, so its copies overlap the loads of q below).
+  constexpr int kLead = kDecStages > 1 ? kDecStages - 1 : 1;
+  constexpr int kWait = kDecStages > 1 ? kDecStages - 1 : 0;   // copy groups that may stay in flight
+#pragma unroll
+  for (int k = 0; k < kLead; ++k) {
+    if (k < nch) stage_in(k);
     cp_async_commit();
-    for (int idx = rows * kChunks + lane; idx < kDecRowsPerWarp * kChunks; idx += 32) {
-      const int r = idx / kChunks, c = idx - r * kChunks;
-      *reinterpret_cast<uint4*>(swz<HD>(sv, r, c)) = make_uint4(0, 0, 0, 0);
-    }
   }
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
@@ -307,96 +331,134 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
       qa[kk][3] = (gid + 8 < G) ? *reinterpret_cast<const uint32_t*>(qb + (gid + 8) * HD + d0 + 8) : 0u;
     }
   }
-  cp_async_wait<0>();
-  __syncwarp();
 
-  // S = Q K^T over the warp's 32 keys: four 8-key tiles.
-  float s[4][4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) s[j][e] = 0.f;
-  const int mi = lane >> 3, ri = lane & 7;    // this lane's ldmatrix row address: matrix mi, row ri
-#pragma unroll
-  for (int kk = 0; kk < KS; ++kk) {
-#pragma unroll
-    for (int np = 0; np < 2; ++np) {
-      uint32_t kb[4];
-      ldsm_x4(kb, swz<HD>(sk, 16 * np + (mi >> 1) * 8 + ri, 2 * kk + (mi & 1)));
-      mma_bf16(s[2 * np], qa[kk], kb[0], kb[1]);
-      mma_bf16(s[2 * np + 1], qa[kk], kb[2], kb[3]);
-    }
-  }
-  // Scale to log2 units, mask keys past the filled slots, softmax per head row
-  // (rows gid and gid + 8 of S; a row's 32 keys are spread over four lanes).
-  float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int key = 8 * j + 2 * tid4 + (e & 1);
-      s[j][e] = (key < rows) ? s[j][e] * p.scale_log2 : -INFINITY;
-      if (e < 2) mx0 = fmaxf(mx0, s[j][e]); else mx1 = fmaxf(mx1, s[j][e]);
-    }
-#pragma unroll
-  for (int off = 1; off <= 2; off <<= 1) {
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-  }
-  float l0 = 0.f, l1 = 0.f;
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float m = (e < 2) ? mx0 : mx1;
-      const float pe = (m == -INFINITY) ? 0.f : exp2f(s[j][e] - m);
-      s[j][e] = pe;
-      if (e < 2) l0 += pe; else l1 += pe;
-    }
-#pragma unroll
-  for (int off = 1; off <= 2; off <<= 1) {
-    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-  }
-
-  // O = P V: two k-steps of 16 keys, P as the A operand straight from S's
-  // registers (high and low bf16 parts), V through transposing matrix loads.
+  // Running state of head rows gid (0) and gid + 8 (1): max (log2 units), sum, O.
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   float o[NT][4];
 #pragma unroll
   for (int t = 0; t < NT; ++t)
 #pragma unroll
     for (int e = 0; e < 4; ++e) o[t][e] = 0.f;
-#pragma unroll
-  for (int kk = 0; kk < 2; ++kk) {
-    uint32_t ph[4], pl[4];
-    const float* t0 = s[2 * kk];
-    const float* t1 = s[2 * kk + 1];
-    const float src[4][2] = {{t0[0], t0[1]}, {t0[2], t0[3]}, {t1[0], t1[1]}, {t1[2], t1[3]}};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      ph[i] = pack_bf16x2(src[i][0], src[i][1]);
-      pl[i] = pack_bf16x2(src[i][0] - bf16_lo(ph[i]), src[i][1] - bf16_hi(ph[i]));
-    }
-#pragma unroll
-    for (int jp = 0; jp < NT / 2; ++jp) {
-      uint32_t vb[4];
-      ldsm_x4_trans(vb, swz<HD>(sv, 16 * kk + (mi & 1) * 8 + ri, 2 * jp + (mi >> 1)));
-      mma_bf16(o[2 * jp], ph, vb[0], vb[1]);
-      mma_bf16(o[2 * jp], pl, vb[0], vb[1]);
-      mma_bf16(o[2 * jp + 1], ph, vb[2], vb[3]);
-      mma_bf16(o[2 * jp + 1], pl, vb[2], vb[3]);
-    }
-  }
+  const int mi = lane >> 3, ri = lane & 7;    // this lane's ldmatrix row address: matrix mi, row ri
 
-  // Merge the four warps (the K/V staging area is reused for their outputs),
-  // then write this split's partial.
+  for (int k = 0; k < nch; ++k) {
+    if constexpr (kDecStages > 1) {
+      if (k + kDecStages - 1 < nch) stage_in(k + kDecStages - 1);
+    } else {
+      if (k >= 1) stage_in(k);                // one buffer: the previous chunk is done with it
+    }
+    cp_async_commit();
+    const int w_lo = (c_lo + k) * kDecSplit + warp * kDecRowsPerWarp;
+    const int rows = max(0, min(kDecRowsPerWarp, n - w_lo));
+    uint16_t* sk = wbase + (k % kDecStages) * kWarpStage;
+    uint16_t* sv = sk + kDecRowsPerWarp * HD;
+    // V rows past the filled slots (no copy lands there) are zeroed while the copies fly.
+    for (int idx = rows * kChunks + lane; idx < kDecRowsPerWarp * kChunks; idx += 32) {
+      const int r = idx / kChunks, c = idx - r * kChunks;
+      *reinterpret_cast<uint4*>(swz<HD>(sv, r, c)) = make_uint4(0, 0, 0, 0);
+    }
+    cp_async_wait<kWait>();                   // chunk k's copies have landed
+    __syncwarp();
+
+    // S = Q K^T over the warp's 32 keys: four 8-key tiles.
+    float s[4][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[j][e] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+#pragma unroll
+      for (int np = 0; np < 2; ++np) {
+        uint32_t kb[4];
+        ldsm_x4(kb, swz<HD>(sk, 16 * np + (mi >> 1) * 8 + ri, 2 * kk + (mi & 1)));
+        mma_bf16(s[2 * np], qa[kk], kb[0], kb[1]);
+        mma_bf16(s[2 * np + 1], qa[kk], kb[2], kb[3]);
+      }
+    }
+    // Scale to log2 units, mask keys past the filled slots, chunk max per head row.
+    float cm0 = -INFINITY, cm1 = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = 8 * j + 2 * tid4 + (e & 1);
+        s[j][e] = (key < rows) ? s[j][e] * p.scale_log2 : -INFINITY;
+        if (e < 2) cm0 = fmaxf(cm0, s[j][e]); else cm1 = fmaxf(cm1, s[j][e]);
+      }
+#pragma unroll
+    for (int off = 1; off <= 2; off <<= 1) {
+      cm0 = fmaxf(cm0, __shfl_xor_sync(0xffffffffu, cm0, off));
+      cm1 = fmaxf(cm1, __shfl_xor_sync(0xffffffffu, cm1, off));
+    }
+    // New running max; the old sum and O are rescaled by exp2(old - new) (exactly 1 when the max
+    // stays, 0 for a row that had nothing yet).
+    const float nm0 = fmaxf(m0, cm0), nm1 = fmaxf(m1, cm1);
+    const float sc0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - nm0);
+    const float sc1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - nm1);
+    m0 = nm0;
+    m1 = nm1;
+    float cl0 = 0.f, cl1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float m = (e < 2) ? nm0 : nm1;
+        const float pe = (m == -INFINITY) ? 0.f : exp2f(s[j][e] - m);
+        s[j][e] = pe;
+        if (e < 2) cl0 += pe; else cl1 += pe;
+      }
+#pragma unroll
+    for (int off = 1; off <= 2; off <<= 1) {
+      cl0 += __shfl_xor_sync(0xffffffffu, cl0, off);
+      cl1 += __shfl_xor_sync(0xffffffffu, cl1, off);
+    }
+    l0 = l0 * sc0 + cl0;
+    l1 = l1 * sc1 + cl1;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      o[t][0] *= sc0;
+      o[t][1] *= sc0;
+      o[t][2] *= sc1;
+      o[t][3] *= sc1;
+    }
+
+    // O += P V: two k-steps of 16 keys, P as the A operand straight from S's
+    // registers (high and low bf16 parts), V through transposing matrix loads.
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+      uint32_t ph[4], pl[4];
+      const float* t0 = s[2 * kk];
+      const float* t1 = s[2 * kk + 1];
+      const float src[4][2] = {{t0[0], t0[1]}, {t0[2], t0[3]}, {t1[0], t1[1]}, {t1[2], t1[3]}};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        ph[i] = pack_bf16x2(src[i][0], src[i][1]);
+        pl[i] = pack_bf16x2(src[i][0] - bf16_lo(ph[i]), src[i][1] - bf16_hi(ph[i]));
+      }
+#pragma unroll
+      for (int jp = 0; jp < NT / 2; ++jp) {
+        uint32_t vb[4];
+        ldsm_x4_trans(vb, swz<HD>(sv, 16 * kk + (mi & 1) * 8 + ri, 2 * jp + (mi >> 1)));
+        mma_bf16(o[2 * jp], ph, vb[0], vb[1]);
+        mma_bf16(o[2 * jp], pl, vb[0], vb[1]);
+        mma_bf16(o[2 * jp + 1], ph, vb[2], vb[3]);
+        mma_bf16(o[2 * jp + 1], pl, vb[2], vb[3]);
+      }
+    }
+    __syncwarp();    // every lane is done with this stage before a later chunk's copies overwrite it
+  }
+  cp_async_wait<0>();
+
+  // Merge the four warps (the staging area is reused for their outputs),
+  // then write the output or this CTA's partial.
   if (tid4 == 0) {
     if (gid < G) {
-      sm_m[warp][gid] = mx0;
+      sm_m[warp][gid] = m0;
       sm_l[warp][gid] = l0;
     }
     if (gid + 8 < G) {
-      sm_m[warp][gid + 8] = mx1;
+      sm_m[warp][gid + 8] = m1;
       sm_l[warp][gid + 8] = l1;
     }
   }
@@ -427,8 +489,16 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
         oo += so[(w * G + g) * HD + e] * c;
       }
     }
-    const int64_t at = ((static_cast<int64_t>(b) * p.n_q_heads + h * G + g) * p.n_split + split) * (HD + 2);
-    if (!KVPOP_IN(split < p.n_split && at + HD + 2 <= static_cast<int64_t>(batch) * p.n_q_heads * p.n_split * (HD + 2),
+    const int64_t bg = static_cast<int64_t>(b) * p.n_q_heads + h * G + g;
+    if (p.n_split == 1) {
+      // The whole row in this CTA: the final output.
+      if (!KVPOP_IN(bg < static_cast<int64_t>(batch) * p.n_q_heads, p.dbg, DBG_DECODE, 3)) continue;
+      p.out[bg * HD + e] = (ll > 0.f) ? oo / ll : 0.f;
+      if (e == 0 && p.lse != nullptr) p.lse[bg] = (ll > 0.f) ? (mm + log2f(ll)) * 0.6931471805599453f : -INFINITY;
+      continue;
+    }
+    const int64_t at = (bg * p.n_split + part) * (HD + 2);
+    if (!KVPOP_IN(part < p.n_split && at + HD + 2 <= static_cast<int64_t>(batch) * p.n_q_heads * p.n_split * (HD + 2),
                   p.dbg, DBG_DECODE, 3))
       continue;
     float* dst = p.partial + at;
@@ -550,19 +620,32 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
   if (tid == 0 && p.lse != nullptr) p.lse[bg] = (ll > 0.f) ? (mm + log2f(ll)) * 0.6931471805599453f : -INFINITY;
 }
 
-template <int HD>
+template <int HD, int kS>
 static cudaError_t launch_split(const DecodeParams& p, dim3 grid, cudaStream_t stream) {
-  const int smem = 2 * kDecSplit * HD * static_cast<int>(sizeof(uint16_t));
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const int smem = (kDecThreads / 32) * kS * 2 * kDecRowsPerWarp * HD * static_cast<int>(sizeof(uint16_t));
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<HD, kS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  decode_split_kernel<HD><<<grid, kDecThreads, smem, stream>>>(p);
+  decode_split_kernel<HD, kS><<<grid, kDecThreads, smem, stream>>>(p);
   return cudaGetLastError();
+}
+
+// Parts each cache row is split into.  One chunk per CTA (single-buffered,
+// three CTAs per SM) when that gives at most about one wave of CTAs; else one
+// CTA per row when the rows alone fill the GPU (no partials, no merge), or
+// enough parts for about one streaming CTA per SM.
+int decode_parts(int rows, int n_chunks, int sm_count) {
+  if (static_cast<int64_t>(rows) * n_chunks <= 3 * static_cast<int64_t>(sm_count)) return n_chunks;
+  return std::max(1, std::min(n_chunks, sm_count / std::max(1, rows)));
 }
 
 cudaError_t launch_decode_attention(const DecodeParams& p, int batch, cudaStream_t stream) {
   dim3 grid(batch * p.n_kv_heads, p.n_split);
-  cudaError_t e = (p.head_dim == 128) ? launch_split<128>(p, grid, stream) : launch_split<64>(p, grid, stream);
+  const int n_chunks = (p.capacity + kDecSplit - 1) / kDecSplit;
+  const bool single = (n_chunks + p.n_split - 1) / p.n_split == 1;   // one chunk per CTA
+  cudaError_t e = (p.head_dim == 128) ? (single ? launch_split<128, 1>(p, grid, stream) : launch_split<128, 3>(p, grid, stream))
+                                      : (single ? launch_split<64, 1>(p, grid, stream) : launch_split<64, 3>(p, grid, stream));
   if (e != cudaSuccess) return e;
+  if (p.n_split == 1) return cudaSuccess;   // the split kernel wrote the output
   // The merge overlaps its launch with the split kernel's tail.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(batch * p.n_q_heads);
