@@ -195,9 +195,12 @@ cudaError_t launch_compact_kv(const CompactParams& p, cudaStream_t stream) {
 
 // ------------------------------------------------------------------ decode attention
 
-constexpr int kDecThreads = 128;                          // 4 warps
-constexpr int kDecRowsPerWarp = kDecSplit / (kDecThreads / 32);
-static_assert(kDecRowsPerWarp == 32, "each warp stages 32 cache rows");
+// A decode CTA has kDecWarps(kS) warps, each owning kDecSplit / warps slots of
+// every chunk: 8 warps of 16 slots when it streams chunks through kS > 1
+// buffers (one CTA per SM: two warps per scheduler hide the MMA chains), 4
+// warps of 32 when it takes a single chunk (two CTAs per SM fit the registers).
+template <int kS>
+__host__ __device__ constexpr int kDecWarps() { return kS > 1 ? 8 : 4; }
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
   const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
@@ -249,24 +252,28 @@ __device__ __forceinline__ uint16_t* swz(uint16_t* base, int r, int c) {
 // One CTA: KV head h of sequence b, all G <= 16 query heads of its group, over
 // a contiguous range of the filled 128-slot chunks of its cache row (the
 // whole row when there are enough rows to fill the GPU; otherwise the row is
-// split over p.n_split CTAs whose partials a merge kernel combines).  Each of
-// the four warps owns 32 slots of every chunk and streams its slices through
+// split over p.n_split CTAs whose partials a merge kernel combines).  Each
+// warp owns its share of the slots of every chunk and streams its slices through
 // a ring of kDecStages shared-memory buffers with cp.async, two chunks ahead
 // of the one it computes (rows past the filled slots are zeroed so that
 // 0 x garbage cannot make a NaN).  Per chunk:
-//   S = Q K^T   16 (heads, padded) x 32 keys, fp32, by MMA (q unscaled bf16,
+//   S = Q K^T   16 (heads, padded) x the warp's keys, fp32, by MMA (q unscaled bf16,
 //               the scale applied to S in fp32)
 //   softmax     a running max and sum per head over the warp's keys so far
 //               (rows of S live on four lanes); O is rescaled when the max grows
 //   O += P V    16 x d, P split into bf16 high and low parts (two MMAs) so the
 //               product keeps ~16 bits of P
-// and at the end the four warps' (max, sum, O) are merged in shared memory
+// and at the end the warps' (max, sum, O) are merged in shared memory
 // into the output (one CTA per row) or this CTA's partial.  kDecStages
 // buffers (kDecStages - 1 chunks in flight while one is computed) when a CTA
 // streams several chunks; one buffer when it has a single chunk, which leaves
 // room for three CTAs per SM.
 template <int HD, int kDecStages>
-__global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(32 * kDecWarps<kDecStages>()) decode_split_kernel(const __grid_constant__ DecodeParams p) {
+  constexpr int kDecThreads = 32 * kDecWarps<kDecStages>();
+  constexpr int kDecRowsPerWarp = kDecSplit / kDecWarps<kDecStages>();
+  constexpr int kDecKeyTiles = kDecRowsPerWarp / 8;       // 8-key tiles of S per warp
+  static_assert(kDecRowsPerWarp % 16 == 0, "whole 16-key MMA steps per warp");
   constexpr int kChunks = HD / 8;      // 16-byte chunks per row
   constexpr int KS = HD / 16;          // k-steps of S = Q K^T
   constexpr int NT = HD / 8;           // 8-column tiles of O
@@ -360,16 +367,16 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     cp_async_wait<kWait>();                   // chunk k's copies have landed
     __syncwarp();
 
-    // S = Q K^T over the warp's 32 keys: four 8-key tiles.
-    float s[4][4];
+    // S = Q K^T over the warp's keys: 8-key tiles.
+    float s[kDecKeyTiles][4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < kDecKeyTiles; ++j)
 #pragma unroll
       for (int e = 0; e < 4; ++e) s[j][e] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < KS; ++kk) {
 #pragma unroll
-      for (int np = 0; np < 2; ++np) {
+      for (int np = 0; np < kDecKeyTiles / 2; ++np) {
         uint32_t kb[4];
         ldsm_x4(kb, swz<HD>(sk, 16 * np + (mi >> 1) * 8 + ri, 2 * kk + (mi & 1)));
         mma_bf16(s[2 * np], qa[kk], kb[0], kb[1]);
@@ -379,7 +386,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     // Scale to log2 units, mask keys past the filled slots, chunk max per head row.
     float cm0 = -INFINITY, cm1 = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < kDecKeyTiles; ++j)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int key = 8 * j + 2 * tid4 + (e & 1);
@@ -400,7 +407,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     m1 = nm1;
     float cl0 = 0.f, cl1 = 0.f;
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < kDecKeyTiles; ++j)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float m = (e < 2) ? nm0 : nm1;
@@ -423,10 +430,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
       o[t][3] *= sc1;
     }
 
-    // O += P V: two k-steps of 16 keys, P as the A operand straight from S's
+    // O += P V: one k-step per 16 keys, P as the A operand straight from S's
     // registers (high and low bf16 parts), V through transposing matrix loads.
 #pragma unroll
-    for (int kk = 0; kk < 2; ++kk) {
+    for (int kk = 0; kk < kDecKeyTiles / 2; ++kk) {
       uint32_t ph[4], pl[4];
       const float* t0 = s[2 * kk];
       const float* t1 = s[2 * kk + 1];
@@ -450,7 +457,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
   }
   cp_async_wait<0>();
 
-  // Merge the four warps (the staging area is reused for their outputs),
+  // Merge the warps (the staging area is reused for their outputs),
   // then write the output or this CTA's partial.
   if (tid4 == 0) {
     if (gid < G) {
@@ -463,7 +470,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const __grid_
     }
   }
   __syncthreads();
-  float* so = reinterpret_cast<float*>(dec_smem);          // [4][G][HD]
+  float* so = reinterpret_cast<float*>(dec_smem);          // [warps][G][HD]: fits in one stage's staging area
 #pragma unroll
   for (int t = 0; t < NT; ++t) {
     const int d0 = 8 * t + 2 * tid4;
@@ -622,10 +629,10 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
 
 template <int HD, int kS>
 static cudaError_t launch_split(const DecodeParams& p, dim3 grid, cudaStream_t stream) {
-  const int smem = (kDecThreads / 32) * kS * 2 * kDecRowsPerWarp * HD * static_cast<int>(sizeof(uint16_t));
+  const int smem = kS * 2 * kDecSplit * HD * static_cast<int>(sizeof(uint16_t));   // every warp's K and V rows
   cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<HD, kS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  decode_split_kernel<HD, kS><<<grid, kDecThreads, smem, stream>>>(p);
+  decode_split_kernel<HD, kS><<<grid, 32 * kDecWarps<kS>(), smem, stream>>>(p);
   return cudaGetLastError();
 }
 
