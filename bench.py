@@ -471,15 +471,18 @@ def run_ours(args):
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # twice the 126 MB L2
 
         def timed(fn, reps=20):
-            """Median device time of fn, with L2 flushed before every repetition.  A ~0.1 ms device-side
-            wait after the flush keeps the GPU busy while the host enqueues the start event and fn, so
-            the interval holds fn's device work and not the host's enqueue time."""
+            """Median device time of fn, with L2 flushed before every repetition: a 256 MiB buffer is
+            written and then read back, so the L2 holds none of fn's data and no dirty lines whose
+            write-back fn would pay for.  A ~0.1 ms device-side wait after the flush keeps the GPU busy
+            while the host enqueues the start event and fn, so the interval holds fn's device work and
+            not the host's enqueue time."""
             for _ in range(3):
                 fn()
             evs_x = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                      for _ in range(reps)]
             for a, z in evs_x:
                 flush.zero_()
+                torch.amax(flush.view(torch.int32))
                 torch.cuda._sleep(200_000)
                 a.record(stream)
                 fn()
@@ -598,8 +601,9 @@ def run_ours(args):
             "frac": moved_d16 / (ms_d16 * 1e-3) / 1e9 / hbm, "bytes": moved_d16, "cache_slots": C, "batch": nb,
             "timing": "mean of 20 back-to-back steps (K and V larger than L2)",
             "ms_l2_flushed_each": ms_d16_flushed}
-        extras["timing"] = ("median of 20 repetitions, L2 flushed (256 MiB write) before each, then a 0.1 ms "
-                            "device-side wait so that the host enqueue time stays outside the interval")
+        extras["timing"] = ("median of 20 repetitions, L2 flushed before each (a 256 MiB buffer written, then "
+                            "read back so that no dirty lines remain), then a 0.1 ms device-side wait so that the "
+                            "host enqueue time stays outside the interval")
         del kc16, vc16, flush
 
     # One problem (rank 0's layer) with its KV heads split over the ranks:
