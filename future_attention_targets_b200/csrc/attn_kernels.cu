@@ -199,6 +199,23 @@ __device__ __forceinline__ int cta_rank() {
   else return static_cast<int>(blockIdx.x & 1u);
 }
 
+// This CTA's rows of the 256-row B tile starting at row y0 (columns x0 ..
+// x0 + HD of the map): all of them for one CTA, rows 128 * rank .. + 127 of
+// the tile for a CTA of a pair.
+template <int HD, int kCta>
+__device__ __forceinline__ void load_b_rows(const CUtensorMap* map, int32_t x0, int32_t y0, uint8_t* dst,
+                                            uint64_t* bar) {
+  constexpr int kBRows = kStreamRows / kCta;
+#pragma unroll
+  for (int kh = 0; kh < HD / 64; ++kh) {
+    if constexpr (kCta == 1) {
+      tma_load_2d(dst + kh * kBRows * 128, map, bar, x0 + kh * 64, y0);
+    } else {
+      tma_load_2d_pair(dst + kh * kBRows * 128, map, bar, x0 + kh * 64, y0 + kBRows * cta_rank<kCta>());
+    }
+  }
+}
+
 // Pass 1: item = (sequence, query block = level, query head); a query block
 // is 128 rows for a single CTA and 256 rows (128 per CTA) for a pair.
 template <int kCta>
@@ -231,13 +248,7 @@ struct LsePassT {
   template <int HD>
   static __device__ __forceinline__ void load_b(const Phase& ph, const Item& it, int32_t t, uint8_t* dst,
                                                 uint64_t* bar) {
-    constexpr int kBRows = kStreamRows / kCta;
-    const int32_t y = it.s + t * kStreamRows + kBRows * cta_rank<kCta>();
-#pragma unroll
-    for (int kh = 0; kh < HD / 64; ++kh) {
-      if constexpr (kCta == 1) tma_load_2d(dst + kh * kBRows * 128, ph.tmap_k, bar, it.h * HD + kh * 64, y);
-      else tma_load_2d_pair(dst + kh * kBRows * 128, ph.tmap_k, bar, it.h * HD + kh * 64, y);
-    }
+    load_b_rows<HD, kCta>(ph.tmap_k, it.h * HD, it.s + t * kStreamRows, dst, bar);
   }
   // Single CTA: the last key tile holds the diagonal; when the query tile
   // starts on a 256-key boundary only its first 128 columns can be unmasked.
@@ -295,13 +306,7 @@ struct TargetPassT {
   template <int HD>
   static __device__ __forceinline__ void load_b(const Phase& ph, const Item& it, int32_t qh, int32_t qt,
                                                 uint8_t* dst, uint64_t* bar) {
-    constexpr int kBRows = kStreamRows / kCta;
-    const int32_t y = it.s + it.i0 + qt * kStreamRows + kBRows * cta_rank<kCta>();
-#pragma unroll
-    for (int kh = 0; kh < HD / 64; ++kh) {
-      if constexpr (kCta == 1) tma_load_2d(dst + kh * kBRows * 128, ph.tmap_q, bar, qh * HD + kh * 64, y);
-      else tma_load_2d_pair(dst + kh * kBRows * 128, ph.tmap_q, bar, qh * HD + kh * 64, y);
-    }
+    load_b_rows<HD, kCta>(ph.tmap_q, qh * HD, it.s + it.i0 + qt * kStreamRows, dst, bar);
   }
   static __device__ __forceinline__ bool half_tile(const Item&, int32_t) { return false; }
 };
@@ -700,6 +705,9 @@ __device__ __forceinline__ uint64_t exp2_mufu_pair(uint64_t y) {
 #ifndef KVPOP_POLY16_TARGET
 #define KVPOP_POLY16_TARGET 5
 #endif
+#ifndef KVPOP_CHUNK_BUFS
+#define KVPOP_CHUNK_BUFS 2
+#endif
 
 template <int kPoly>
 __device__ __forceinline__ constexpr bool poly_pair(int q) {
@@ -753,13 +761,37 @@ __device__ __forceinline__ float acc_total(uint64_t (&acc)[4]) {
 // Sum of exp2(x * c - off) over the kGroupCols = 64 columns of this thread's
 // TMEM lane starting at taddr: four chunks of 16, each load in flight while
 // the chunk before it is summed (small chunks shorten the load every warp of
-// the CTA waits for at the start of a tile).  kMasked: column m counts iff
-// lo <= m < hi.
-template <bool kMasked, int kPoly, bool kBiasFree = false, bool kDeg3 = kBiasFree>
-__device__ __forceinline__ float group_exp_sum(uint32_t taddr, uint64_t c2, uint64_t nb, int lo, int hi,
-                                               float xmin = 0.f) {
+// the CTA waits for at the start of a tile).  `release` runs (warp-converged)
+// once the last chunk's load has landed, before its exponentials: the
+// accumulator is free for the next MMA from then on.  kMasked: column m
+// counts iff lo <= m < hi.
+template <bool kMasked, int kPoly, bool kBiasFree = false, bool kDeg3 = kBiasFree, class Release>
+__device__ __forceinline__ float group_exp_sum(uint32_t taddr, uint64_t c2, uint64_t nb, int lo, int hi, float xmin,
+                                               Release&& release) {
   uint32_t ra[16], rb[16];
   uint64_t acc[4] = {0, 0, 0, 0};
+#if KVPOP_CHUNK_BUFS == 3
+  // Chunks 0-2 at once, chunk 3 into chunk 0's registers once those are
+  // summed: the accumulator is released after two chunks of work.
+  uint32_t rc[16];
+  tmem_load<16>(taddr, ra);
+  tmem_load<16>(taddr + 16, rb);
+  tmem_load<16>(taddr + 32, rc);
+  tmem_load_wait<16>(ra);
+  tmem_regs_landed(rb);
+  tmem_regs_landed(rc);
+  if constexpr (kMasked) chunk_exp_sum_masked(ra, c2, nb, lo, hi, acc);
+  else chunk_exp_sum<kPoly, kBiasFree, 0, kDeg3>(ra, c2, nb, xmin, acc);
+  tmem_load<16>(taddr + 48, ra);
+  if constexpr (kMasked) chunk_exp_sum_masked(rb, c2, nb, lo - 16, hi - 16, acc);
+  else chunk_exp_sum<kPoly, kBiasFree, 8, kDeg3>(rb, c2, nb, xmin, acc);
+  tmem_load_wait<16>(ra);
+  release();
+  if constexpr (kMasked) chunk_exp_sum_masked(rc, c2, nb, lo - 32, hi - 32, acc);
+  else chunk_exp_sum<kPoly, kBiasFree, 0, kDeg3>(rc, c2, nb, xmin, acc);
+  if constexpr (kMasked) chunk_exp_sum_masked(ra, c2, nb, lo - 48, hi - 48, acc);
+  else chunk_exp_sum<kPoly, kBiasFree, 8, kDeg3>(ra, c2, nb, xmin, acc);
+#else
   tmem_load<16>(taddr, ra);
   tmem_load_wait<16>(ra);
   tmem_load<16>(taddr + 16, rb);
@@ -774,8 +806,10 @@ __device__ __forceinline__ float group_exp_sum(uint32_t taddr, uint64_t c2, uint
   if constexpr (kMasked) chunk_exp_sum_masked(ra, c2, nb, lo - 32, hi - 32, acc);
   else chunk_exp_sum<kPoly, kBiasFree, 0, kDeg3>(ra, c2, nb, xmin, acc);
   tmem_load_wait<16>(rb);
+  release();
   if constexpr (kMasked) chunk_exp_sum_masked(rb, c2, nb, lo - 48, hi - 48, acc);
   else chunk_exp_sum<kPoly, kBiasFree, 8, kDeg3>(rb, c2, nb, xmin, acc);
+#endif
   return acc_total(acc);
 }
 
@@ -824,9 +858,8 @@ __device__ void lse_softmax_phase(const AttnParams& p, const Phase& ph, uint8_t*
   const float kBig = 18446744073709551616.0f;   // 2^64: larger tile sums force an exact rescale
   const float kRebase = 4294967296.0f;          // 2^32: keep the running sum moderate
   const float kTiny = 5.421010862427522e-20f;   // 2^-64: smaller first-tile sums take the exact max
-#if KVPOP_LSE_DEG3
   const float xmin = -126.f / p.scale_log2;     // below it exp2(c x) < 2^-126: clamp for the polynomial
-#endif
+  const auto no_release = []() {};
   const LevelSchedule& sched = *ph.sched;
   const int32_t total = sched.total_items;
   for (int32_t k = 0; st.ok; ++k) {
@@ -868,19 +901,20 @@ __device__ void lse_softmax_phase(const AttnParams& p, const Phase& ph, uint8_t*
           // Rows whose running offset is still 0 (the common case) take the
           // transposed pass's scale-folded polynomial; chosen per warp.
           if (masked)
-            ts = group_exp_sum<true, 0>(taddr, c2, nb, 0, hi);
+            ts = group_exp_sum<true, 0>(taddr, c2, nb, 0, hi, 0.f, no_release);
           else if (__all_sync(0xffffffffu, off == 0.f))
-            ts = group_exp_sum<false, KVPOP_POLY16_LSE, true>(taddr, c2, nb, 0, kGroupCols, xmin);
+            ts = group_exp_sum<false, KVPOP_POLY16_LSE, true>(taddr, c2, nb, 0, kGroupCols, xmin, no_release);
           else
-            ts = group_exp_sum<false, KVPOP_POLY16_LSE, false, true>(taddr, c2, nb, 0, kGroupCols);
+            ts = group_exp_sum<false, KVPOP_POLY16_LSE, false, true>(taddr, c2, nb, 0, kGroupCols, 0.f, no_release);
 #else
-          ts = masked ? group_exp_sum<true, 0>(taddr, c2, nb, 0, hi)
-                      : group_exp_sum<false, KVPOP_POLY16_LSE>(taddr, c2, nb, 0, kGroupCols);
+          ts = masked ? group_exp_sum<true, 0>(taddr, c2, nb, 0, hi, 0.f, no_release)
+                      : group_exp_sum<false, KVPOP_POLY16_LSE>(taddr, c2, nb, 0, kGroupCols, 0.f, no_release);
 #endif
         }
         const bool rescale = !(ts < kBig) || (first && !(ts >= kTiny));
         if (rescale && first) off = -INFINITY;
-        // Warp-uniform: the rescale path issues warp-collective TMEM loads.
+        // Warp-uniform: the rescale path issues warp-collective TMEM loads
+        // (so the accumulator is released only after the tile's sum).
         if (__any_sync(0xffffffffu, rescale)) {
           const float tm = group_max(taddr, c, 0, hi);
           const float noff = fmaxf(off, tm);
@@ -889,9 +923,9 @@ __device__ void lse_softmax_phase(const AttnParams& p, const Phase& ph, uint8_t*
             off = noff;
           }
           const uint64_t nb = f2_pack(-off, -off);
-          ts = masked ? group_exp_sum<true, 0>(taddr, c2, nb, 0, hi)
+          ts = masked ? group_exp_sum<true, 0>(taddr, c2, nb, 0, hi, 0.f, no_release)
                       : group_exp_sum<false, KVPOP_POLY16_LSE, false, KVPOP_LSE_DEG3 != 0>(taddr, c2, nb, 0,
-                                                                                        kGroupCols);
+                                                                                        kGroupCols, 0.f, no_release);
           if (!(off > -INFINITY)) ts = 0.f;
         }
         sum += ts;
@@ -1016,14 +1050,18 @@ __device__ void target_softmax_phase(const AttnParams& p, const Phase& ph, uint8
         const bool ragged = (qt == it.nq - 1) && ragged_end;
         const int lo = diag ? max(0, rk + row - c0) : 0;
         const int hi = ragged ? min(kGroupCols, it.L - it.i0 - qt * kStreamRows - c0) : kGroupCols;
-        const float ts = skip ? 0.f
-                         : (diag || ragged)
-                             ? group_exp_sum<true, 0>(taddr, c2, zero2, lo, hi)
-                             : group_exp_sum<false, KVPOP_POLY16_TARGET, true>(taddr, c2, zero2, 0, kGroupCols,
-                                                                                  xmin);
-        tc_fence_before_sync();
-        __syncwarp();
-        if (lane == 0) release_acc<kCta>(&bars.acc_empty[acc]);
+        auto release = [&]() {
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) release_acc<kCta>(&bars.acc_empty[acc]);
+        };
+        float ts = 0.f;
+        if (skip)
+          release();
+        else if (diag || ragged)
+          ts = group_exp_sum<true, 0>(taddr, c2, zero2, lo, hi, 0.f, release);
+        else
+          ts = group_exp_sum<false, KVPOP_POLY16_TARGET, true>(taddr, c2, zero2, 0, kGroupCols, xmin, release);
         ++st.acc_cnt;
         const float yk = ts - comp;
         const float tk = run + yk;

@@ -120,6 +120,10 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_kv_kernel(const __
   const uint8_t* mask = p.keep + static_cast<int64_t>(h) * p.total_tokens + s0;
   const int64_t row0 = (static_cast<int64_t>(b) * p.n_kv_heads + h) * p.capacity;   // first slot of (b, h)
   const int S0 = c * kCompactSlots, S1 = min(S0 + kCompactSlots, p.capacity);
+  // Launched as a programmatic dependent: everything above overlapped the
+  // previous kernel's tail; its writes (the keep mask) are visible after this.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const int chunk = (L + kCompactThreads - 1) / kCompactThreads;
   const int c0 = min(L, tid * chunk), c1 = min(L, c0 + chunk);
@@ -184,13 +188,29 @@ __global__ void __launch_bounds__(kCompactThreads, 2) compact_kv_kernel(const __
   if (c == 0 && tid == 0 && KVPOP_IN(b < p.n_seqs, p.dbg, DBG_COMPACT, 6)) p.count[b * p.n_kv_heads + h] = total;
 }
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel in the stream finishes, and waits for it
+// (griddepcontrol.wait) before its first read of global memory.
+template <class Kern, class Params>
+static cudaError_t launch_dependent(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                                    const Params& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
 cudaError_t launch_compact_kv(const CompactParams& p, cudaStream_t stream) {
   dim3 grid(p.n_seqs * p.n_kv_heads, (p.capacity + kCompactSlots - 1) / kCompactSlots);
-  if (p.head_dim == 128)
-    compact_kv_kernel<128><<<grid, kCompactThreads, 0, stream>>>(p);
-  else
-    compact_kv_kernel<64><<<grid, kCompactThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+  return p.head_dim == 128 ? launch_dependent(compact_kv_kernel<128>, grid, dim3(kCompactThreads), 0, stream, p)
+                           : launch_dependent(compact_kv_kernel<64>, grid, dim3(kCompactThreads), 0, stream, p);
 }
 
 // ------------------------------------------------------------------ decode attention
@@ -288,6 +308,9 @@ __global__ void __launch_bounds__(32 * kDecWarps<kDecStages>()) decode_split_ker
   const int gid = lane >> 2, tid4 = lane & 3;
   const int G = p.n_q_heads / p.n_kv_heads;
   [[maybe_unused]] const int batch = static_cast<int>(gridDim.x) / p.n_kv_heads;
+  // A programmatic dependent of the previous kernel (the compaction, or the
+  // last step): its writes to the cache are visible after this.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int n = min(p.count[b * p.n_kv_heads + h], p.capacity);
   // This CTA's chunks: its share of the chunk range, cut at the filled slots.
   const int n_chunks = (p.capacity + kDecSplit - 1) / kDecSplit;
@@ -632,8 +655,7 @@ static cudaError_t launch_split(const DecodeParams& p, dim3 grid, cudaStream_t s
   const int smem = kS * 2 * kDecSplit * HD * static_cast<int>(sizeof(uint16_t));   // every warp's K and V rows
   cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<HD, kS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  decode_split_kernel<HD, kS><<<grid, 32 * kDecWarps<kS>(), smem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_dependent(decode_split_kernel<HD, kS>, grid, dim3(32 * kDecWarps<kS>()), smem, stream, p);
 }
 
 // Parts each cache row is split into.  One chunk per CTA (single-buffered,
@@ -654,17 +676,7 @@ cudaError_t launch_decode_attention(const DecodeParams& p, int batch, cudaStream
   if (e != cudaSuccess) return e;
   if (p.n_split == 1) return cudaSuccess;   // the split kernel wrote the output
   // The merge overlaps its launch with the split kernel's tail.
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(batch * p.n_q_heads);
-  cfg.blockDim = dim3(128);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_combine_kernel, p);
+  return launch_dependent(decode_combine_kernel, dim3(batch * p.n_q_heads), dim3(128), 0, stream, p);
 }
 
 // ------------------------------------------------------------------ fixed scratch for the allocation-free decode
