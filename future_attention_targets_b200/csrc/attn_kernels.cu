@@ -705,9 +705,6 @@ __device__ __forceinline__ uint64_t exp2_mufu_pair(uint64_t y) {
 #ifndef KVPOP_POLY16_TARGET
 #define KVPOP_POLY16_TARGET 5
 #endif
-#ifndef KVPOP_CHUNK_BUFS
-#define KVPOP_CHUNK_BUFS 2
-#endif
 
 template <int kPoly>
 __device__ __forceinline__ constexpr bool poly_pair(int q) {
@@ -770,28 +767,6 @@ __device__ __forceinline__ float group_exp_sum(uint32_t taddr, uint64_t c2, uint
                                                Release&& release) {
   uint32_t ra[16], rb[16];
   uint64_t acc[4] = {0, 0, 0, 0};
-#if KVPOP_CHUNK_BUFS == 3
-  // Chunks 0-2 at once, chunk 3 into chunk 0's registers once those are
-  // summed: the accumulator is released after two chunks of work.
-  uint32_t rc[16];
-  tmem_load<16>(taddr, ra);
-  tmem_load<16>(taddr + 16, rb);
-  tmem_load<16>(taddr + 32, rc);
-  tmem_load_wait<16>(ra);
-  tmem_regs_landed(rb);
-  tmem_regs_landed(rc);
-  if constexpr (kMasked) chunk_exp_sum_masked(ra, c2, nb, lo, hi, acc);
-  else chunk_exp_sum<kPoly, kBiasFree, 0, kDeg3>(ra, c2, nb, xmin, acc);
-  tmem_load<16>(taddr + 48, ra);
-  if constexpr (kMasked) chunk_exp_sum_masked(rb, c2, nb, lo - 16, hi - 16, acc);
-  else chunk_exp_sum<kPoly, kBiasFree, 8, kDeg3>(rb, c2, nb, xmin, acc);
-  tmem_load_wait<16>(ra);
-  release();
-  if constexpr (kMasked) chunk_exp_sum_masked(rc, c2, nb, lo - 32, hi - 32, acc);
-  else chunk_exp_sum<kPoly, kBiasFree, 0, kDeg3>(rc, c2, nb, xmin, acc);
-  if constexpr (kMasked) chunk_exp_sum_masked(ra, c2, nb, lo - 48, hi - 48, acc);
-  else chunk_exp_sum<kPoly, kBiasFree, 8, kDeg3>(ra, c2, nb, xmin, acc);
-#else
   tmem_load<16>(taddr, ra);
   tmem_load_wait<16>(ra);
   tmem_load<16>(taddr + 16, rb);
@@ -809,7 +784,6 @@ __device__ __forceinline__ float group_exp_sum(uint32_t taddr, uint64_t c2, uint
   release();
   if constexpr (kMasked) chunk_exp_sum_masked(rb, c2, nb, lo - 48, hi - 48, acc);
   else chunk_exp_sum<kPoly, kBiasFree, 8, kDeg3>(rb, c2, nb, xmin, acc);
-#endif
   return acc_total(acc);
 }
 

@@ -364,17 +364,6 @@ __device__ __forceinline__ void tmem_load_wait<16>(uint32_t (&r)[16]) {
                : "memory");
 }
 
-// After a tcgen05.wait::ld that also covered loads into r: keeps every use of
-// r after that point (the wait helper ties only its own array).
-__device__ __forceinline__ void tmem_regs_landed(uint32_t (&r)[16]) {
-  asm volatile(""
-               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
-                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
-                 "+r"(r[14]), "+r"(r[15])
-               :
-               : "memory");
-}
-
 // ------------------------------------------------------------------ schedule
 
 struct WorkItem {
