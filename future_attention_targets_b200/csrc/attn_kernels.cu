@@ -787,21 +787,45 @@ __device__ __forceinline__ float group_exp_sum(uint32_t taddr, uint64_t c2, uint
   return acc_total(acc);
 }
 
-// Max of x * c over columns lo <= m < hi of the group's 64 (pass-1 rescale path).
-__device__ __forceinline__ float group_max(uint32_t taddr, float c, int lo, int hi) {
-  float m = -INFINITY;
-#pragma unroll 1
-  for (int ch = 0; ch < kGroupCols / 32; ++ch) {
-    uint32_t r[32];
-    tmem_load<32>(taddr + 32 * ch, r);
-    tmem_load_wait<32>(r);
+// q . k of one bf16 row pair of HD elements, in fp32, on CUDA cores.
+template <int HD>
+__device__ __forceinline__ float dot_bf16_row(const uint16_t* a, const uint16_t* b) {
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll 4
+  for (int d = 0; d < HD; d += 8) {
+    const uint4 x = __ldg(reinterpret_cast<const uint4*>(a + d));
+    const uint4 y = __ldg(reinterpret_cast<const uint4*>(b + d));
+    const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const int col = 32 * ch + e;
-      if (col >= lo && col < hi) m = fmaxf(m, __uint_as_float(r[e]) * c);
+    for (int w = 0; w < 4; ++w) {
+      s0 = fmaf(__uint_as_float(xs[w] << 16), __uint_as_float(ys[w] << 16), s0);
+      s1 = fmaf(__uint_as_float(xs[w] & 0xffff0000u), __uint_as_float(ys[w] & 0xffff0000u), s1);
     }
   }
-  return m;
+  return s0 + s1;
+}
+
+// Pass 1's exact path for one lane whose tile sum left the safe range (a
+// row's first tile outside [2^-64, 2^64), any later tile past 2^64): the
+// scores of its row over the group's columns 0 .. hi-1 are computed again on
+// CUDA cores from Q and K in global memory (qrow: the query row; k0: the key
+// of column 0, the next column kstride elements further on), because the
+// accumulator has already gone back to the MMA.  Their exact max, if above
+// the running offset, becomes the new offset (the running sum rescaled), and
+// the tile's sum is returned at that offset.  Rare: ordinary inputs never
+// reach it; logits spanning more than ~60 (in log2 units) within a tile do.
+template <int HD>
+__device__ __noinline__ float lse_tile_exact(const uint16_t* qrow, const uint16_t* k0, int64_t kstride, int hi,
+                                             float c, float& off, float& sum) {
+  float m = -INFINITY;
+  for (int e = 0; e < hi; ++e) m = fmaxf(m, dot_bf16_row<HD>(qrow, k0 + e * kstride) * c);
+  const float noff = fmaxf(off, m);
+  if (!(noff > -INFINITY)) return 0.f;   // no column counts
+  sum = (off > -INFINITY) ? sum * ex2_approx(off - noff) : 0.f;
+  off = noff;
+  float ts = 0.f;
+  for (int e = 0; e < hi; ++e) ts += ex2_approx(dot_bf16_row<HD>(qrow, k0 + e * kstride) * c - off);
+  return ts;
 }
 
 // ------------------------------------------------------------------ softmax: pass 1
@@ -833,7 +857,6 @@ __device__ void lse_softmax_phase(const AttnParams& p, const Phase& ph, uint8_t*
   const float kRebase = 4294967296.0f;          // 2^32: keep the running sum moderate
   const float kTiny = 5.421010862427522e-20f;   // 2^-64: smaller first-tile sums take the exact max
   const float xmin = -126.f / p.scale_log2;     // below it exp2(c x) < 2^-126: clamp for the polynomial
-  const auto no_release = []() {};
   const LevelSchedule& sched = *ph.sched;
   const int32_t total = sched.total_items;
   for (int32_t k = 0; st.ok; ++k) {
@@ -860,7 +883,17 @@ __device__ void lse_softmax_phase(const AttnParams& p, const Phase& ph, uint8_t*
                                            : c0 > dcol + kTileRows - 1);
       const bool masked = last && !skip && c0 + kGroupCols - 1 > dcol;
       const int hi = masked ? min(kGroupCols, max(0, row - (c0 - dcol) + 1)) : kGroupCols;
-      if (!skip) {
+      // The accumulator goes back to the MMA once the group's last chunk is
+      // in registers (at once for a skipped group): the rare exact path
+      // below recomputes scores on CUDA cores instead of re-reading it.
+      auto release = [&]() {
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) release_acc<kCta>(&bars.acc_empty[acc]);
+      };
+      if (skip) {
+        release();
+      } else {
         const uint32_t taddr = lane_addr + acc * kStreamRows;
         float ts = 0.f;
         // A row's first tile is summed with offset 0 instead of its exact max
@@ -875,32 +908,33 @@ __device__ void lse_softmax_phase(const AttnParams& p, const Phase& ph, uint8_t*
           // Rows whose running offset is still 0 (the common case) take the
           // transposed pass's scale-folded polynomial; chosen per warp.
           if (masked)
-            ts = group_exp_sum<true, 0>(taddr, c2, nb, 0, hi, 0.f, no_release);
+            ts = group_exp_sum<true, 0>(taddr, c2, nb, 0, hi, 0.f, release);
           else if (__all_sync(0xffffffffu, off == 0.f))
-            ts = group_exp_sum<false, KVPOP_POLY16_LSE, true>(taddr, c2, nb, 0, kGroupCols, xmin, no_release);
+            ts = group_exp_sum<false, KVPOP_POLY16_LSE, true>(taddr, c2, nb, 0, kGroupCols, xmin, release);
           else
-            ts = group_exp_sum<false, KVPOP_POLY16_LSE, false, true>(taddr, c2, nb, 0, kGroupCols, 0.f, no_release);
+            ts = group_exp_sum<false, KVPOP_POLY16_LSE, false, true>(taddr, c2, nb, 0, kGroupCols, 0.f, release);
 #else
-          ts = masked ? group_exp_sum<true, 0>(taddr, c2, nb, 0, hi, 0.f, no_release)
-                      : group_exp_sum<false, KVPOP_POLY16_LSE>(taddr, c2, nb, 0, kGroupCols, 0.f, no_release);
+          ts = masked ? group_exp_sum<true, 0>(taddr, c2, nb, 0, hi, 0.f, release)
+                      : group_exp_sum<false, KVPOP_POLY16_LSE>(taddr, c2, nb, 0, kGroupCols, 0.f, release);
 #endif
         }
         const bool rescale = !(ts < kBig) || (first && !(ts >= kTiny));
-        if (rescale && first) off = -INFINITY;
-        // Warp-uniform: the rescale path issues warp-collective TMEM loads
-        // (so the accumulator is released only after the tile's sum).
-        if (__any_sync(0xffffffffu, rescale)) {
-          const float tm = group_max(taddr, c, 0, hi);
-          const float noff = fmaxf(off, tm);
-          if (noff > -INFINITY) {
-            sum = (off > -INFINITY) ? sum * ex2_approx(off - noff) : 0.f;
-            off = noff;
+        if (rescale) {
+          if (first) off = -INFINITY;
+          // Per lane (no TMEM access): rows past the sequence end are not
+          // written, and their keys may lie past T, so they only reset.
+          const int32_t i = it.i0 + kTileRows * cta_rank<kCta>() + row;   // query row within the sequence
+          const int32_t j = t * kStreamRows + c0;                          // key of the group's column 0
+          if (i < it.L &&
+              KVPOP_IN(it.s + i < p.total_tokens && (hi <= 0 || it.s + j + hi <= p.total_tokens) &&
+                           it.g < p.n_q_heads,
+                       p.dbg, DBG_ROW_LSE, 7)) {
+            const uint16_t* qrow = p.q + (static_cast<int64_t>(it.s + i) * p.n_q_heads + it.g) * HD;
+            const uint16_t* k0 = p.k + (static_cast<int64_t>(it.s + j) * p.n_kv_heads + it.h) * HD;
+            ts = lse_tile_exact<HD>(qrow, k0, static_cast<int64_t>(p.n_kv_heads) * HD, hi, c, off, sum);
+          } else {
+            ts = 0.f;
           }
-          const uint64_t nb = f2_pack(-off, -off);
-          ts = masked ? group_exp_sum<true, 0>(taddr, c2, nb, 0, hi, 0.f, no_release)
-                      : group_exp_sum<false, KVPOP_POLY16_LSE, false, KVPOP_LSE_DEG3 != 0>(taddr, c2, nb, 0,
-                                                                                        kGroupCols, 0.f, no_release);
-          if (!(off > -INFINITY)) ts = 0.f;
         }
         sum += ts;
         if (sum > kRebase) {
@@ -909,9 +943,6 @@ __device__ void lse_softmax_phase(const AttnParams& p, const Phase& ph, uint8_t*
           off = off + static_cast<float>(e);
         }
       }
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) release_acc<kCta>(&bars.acc_empty[acc]);
       ++st.acc_cnt;
     }
     if (!st.ok) break;

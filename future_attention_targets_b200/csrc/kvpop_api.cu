@@ -276,6 +276,8 @@ kvpop_status fill_attn_common(AttnParams* p, const void* q, const void* k, const
                      target_pass ? a_rows : b_rows)) != KVPOP_OK)
     return st;
   p->cta = cta;
+  p->q = static_cast<const uint16_t*>(q);
+  p->k = static_cast<const uint16_t*>(k);
   p->wait_ns = wait_limit_ns();
   p->total_tokens = sh.total_tokens;
   p->n_q_heads = sh.n_q_heads;

@@ -33,6 +33,8 @@ struct AttnParams {
   CUtensorMap tmap_q;     // bf16 [T, H_q * d], box {64, rows}
   CUtensorMap tmap_k;     // bf16 [T, H_kv * d], box {64, rows}
   CUtensorMap tmap_rows;  // CTA pairs, pass 2: normaliser rows [H_q][T][8 x bf16], box {8, 128, 1}
+  const uint16_t* q;      // bf16 [T, H_q, d] (pass 1's exact-max fallback reads scores from it)
+  const uint16_t* k;      // bf16 [T, H_kv, d]
   void* nrm_rows;         // normaliser rows [H_q, T] x 16 bytes: pass 2 reads them, pass 1
                           // writes them when non-null (next to lse)
   float* out;             // pass 1: lse [H_q, T]; pass 2: target [H_kv, T]
