@@ -664,17 +664,16 @@ __device__ __forceinline__ uint64_t exp2_poly_pair(uint64_t y) {
 
 // 2^(c x) for a pair with the scale folded into the range reduction:
 // x is clamped so that c x >= -126, then t = rm(c x + 1.5 * 2^23) in one
-// fused multiply-add, n = t - 1.5 * 2^23 = floor(c x), f = c x - n (exact).
+// fused multiply-add, n = t - 1.5 * 2^23 = floor(c x) (taken negated, in one
+// packed FMA), f = c x - n (exact).
 __device__ __forceinline__ uint64_t exp2_poly_pair_scaled(uint64_t x, uint64_t c2, float xmin) {
   float x0, x1;
   f2_unpack(x, x0, x1);
   const uint64_t xc = f2_pack(fmaxf(x0, xmin), fmaxf(x1, xmin));
   uint64_t t;
   asm("fma.rm.ftz.f32x2 %0, %1, %2, %3;" : "=l"(t) : "l"(xc), "l"(c2), "l"(f2_pack(kRoundMagic, kRoundMagic)));
-  const uint64_t n = f2_add(t, f2_pack(-kRoundMagic, -kRoundMagic));
-  float n0, n1;
-  f2_unpack(n, n0, n1);
-  const uint64_t f = f2_fma(xc, c2, f2_pack(-n0, -n1));
+  const uint64_t neg_n = f2_fma(t, f2_pack(-1.f, -1.f), f2_pack(kRoundMagic, kRoundMagic));   // -n, exact
+  const uint64_t f = f2_fma(xc, c2, neg_n);
   uint64_t q = f2_fma(f, f2_pack(kT3, kT3), f2_pack(kT2, kT2));
   q = f2_fma(q, f, f2_pack(kT1, kT1));
   q = f2_fma(q, f, f2_pack(1.f, 1.f));
