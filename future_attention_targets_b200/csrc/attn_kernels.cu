@@ -812,7 +812,8 @@ __device__ __forceinline__ float dot_bf16_row(const uint16_t* a, const uint16_t*
 // accumulator has already gone back to the MMA.  Their exact max, if above
 // the running offset, becomes the new offset (the running sum rescaled), and
 // the tile's sum is returned at that offset.  Rare: ordinary inputs never
-// reach it; logits spanning more than ~60 (in log2 units) within a tile do.
+// reach it; scores (in log2 units) beyond about +-64 in a row's first tile,
+// or more than about 58 above the running offset later, do.
 template <int HD>
 __device__ __noinline__ float lse_tile_exact(const uint16_t* qrow, const uint16_t* k0, int64_t kstride, int hi,
                                              float c, float& off, float& sum) {
