@@ -108,3 +108,61 @@ def test_decode_step_in_a_graph():
         cnt.copy_(torch.randint(1, C + 1, (B, Hkv), dtype=torch.int32, device="cuda"))
 
     _replays_match(graph, lambda: decode_attention(q, kc, vc, cnt), (out, lse), refill)
+
+
+def test_targets_compaction_decode_chain_in_a_graph():
+    """Keep mask -> compaction -> decode in one graph.  The compaction and decode kernels are launched as
+    programmatic dependents of the kernel before them; a replay after new Q/K/V and decode queries were
+    copied in must still see the new keep mask and cache (their waits order them after their producers)."""
+    from future_attention_targets_b200 import compact_kv
+    from future_attention_targets_b200.workloads import random_qk
+    d = make_inputs("qwen3_4b_4k")
+    w = d["workload"]
+    q, k = dev(d["q_bits"]), dev(d["k_bits"])
+    T = q.shape[0]
+    cu, W, S, budgets, scale = d["cu_seqlens"], d["window"], d["sinks"], d["budgets"], d["scale"]
+    C = int(max(budgets))
+    nb = len(cu) - 1
+    v_bits, _ = random_qk(T, w.n_kv_heads, w.n_kv_heads, w.head_dim, seed=3)
+    v = dev(v_bits)
+    qd_bits, _ = random_qk(nb, w.n_q_heads, w.n_kv_heads, w.head_dim, seed=4)
+    qd = dev(qd_bits.reshape(nb, w.n_q_heads, w.head_dim))
+    lse = torch.empty((w.n_q_heads, T), dtype=torch.float32, device="cuda")
+    tgt = torch.empty((w.n_kv_heads, T), dtype=torch.float32, device="cuda")
+    keep = torch.empty((w.n_kv_heads, T), dtype=torch.uint8, device="cuda")
+    cache = (torch.empty((nb, w.n_kv_heads, C, w.head_dim), dtype=torch.bfloat16, device="cuda"),
+             torch.empty((nb, w.n_kv_heads, C, w.head_dim), dtype=torch.bfloat16, device="cuda"),
+             torch.empty((nb, w.n_kv_heads, C), dtype=torch.int32, device="cuda"),
+             torch.empty((nb, w.n_kv_heads), dtype=torch.int32, device="cuda"))
+    out = torch.empty((nb, w.n_q_heads, w.head_dim), device="cuda")
+    dl = torch.empty((nb, w.n_q_heads), device="cuda")
+    ws = torch.empty(target_workspace_bytes(T, w.n_q_heads, w.n_kv_heads, w.head_dim), dtype=torch.uint8,
+                     device="cuda")
+    wsd = torch.empty(decode_workspace_bytes(nb, w.n_q_heads, w.n_kv_heads, w.head_dim, C), dtype=torch.uint8,
+                      device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def run():
+        future_targets(q, k, cu, W, S, budgets, scale=scale, lse=lse, target=tgt, keep=keep, workspace=ws,
+                       status=status)
+        compact_kv(k, v, keep, cu, C, out=cache)
+        decode_attention(qd, cache[0], cache[1], cache[3], scale, out=out, lse=dl, workspace=wsd)
+
+    graph = _capture(run)
+    other = make_inputs("qwen3_4b_4k", seed=9)
+    v2_bits, _ = random_qk(T, w.n_kv_heads, w.n_kv_heads, w.head_dim, seed=10)
+    qd2_bits, _ = random_qk(nb, w.n_q_heads, w.n_kv_heads, w.head_dim, seed=11)
+
+    def refill():
+        q.copy_(dev(other["q_bits"]))
+        k.copy_(dev(other["k_bits"]))
+        v.copy_(dev(v2_bits))
+        qd.copy_(dev(qd2_bits.reshape(nb, w.n_q_heads, w.head_dim)))
+
+    def eager():
+        _, _, kp = future_targets(q, k, cu, W, S, budgets, scale=scale)
+        kc, vc, pos, cnt = compact_kv(k, v, kp, cu, C)
+        o, l = decode_attention(qd, kc, vc, cnt, scale)
+        return kp, kc, vc, pos, cnt, o, l
+
+    _replays_match(graph, eager, (keep,) + cache + (out, dl), refill, status)
