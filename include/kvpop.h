@@ -211,7 +211,10 @@ typedef struct {
  *   pos        device int32 [batch, n_kv_heads, capacity]: the source position
  *              (relative to the sequence start) of each slot, -1 when unused
  *   count      device int32 [batch, n_kv_heads]: kept positions per row
- * shape.n_q_heads is ignored; no status word (no on-chip waits). */
+ * shape.n_q_heads is ignored; no status word (no on-chip waits).  The kernel
+ * is launched as a programmatic dependent of the stream's previous kernel: it
+ * may start while that kernel finishes and waits for it (griddepcontrol.wait)
+ * before reading any global memory, so stream order holds as usual. */
 KVPOP_API kvpop_status kvpop_compact_kv(const void* k, const void* v, const uint8_t* keep,
                                         const int32_t* cu_seqlens, kvpop_shape shape, int32_t capacity,
                                         void* k_cache, void* v_cache, int32_t* pos, int32_t* count,
@@ -230,9 +233,10 @@ KVPOP_API size_t kvpop_decode_workspace_bytes(kvpop_cache_shape shape);
  *   lse        device fp32 [batch, n_q_heads] natural log, or NULL
  *   workspace  device, >= kvpop_decode_workspace_bytes(shape) bytes, 16-byte aligned;
  *              holds the per-split partial results (its contents on entry are ignored)
- * Split-K over the cache slots (128 per CTA, staged in shared memory), then
- * one merge kernel launched as a programmatic dependent of the first; no
- * on-chip spin waits. */
+ * Split-K over the cache slots (128 per CTA, staged in shared memory), and
+ * one merge kernel when a row is split over several CTAs; both launched as
+ * programmatic dependents of the kernel before them in the stream (each waits
+ * for it before reading global memory); no on-chip spin waits. */
 KVPOP_API kvpop_status kvpop_decode_attention(const void* q, const void* k_cache, const void* v_cache,
                                               const int32_t* count, kvpop_cache_shape shape, float scale,
                                               float* out, float* lse, void* workspace, size_t workspace_bytes,
