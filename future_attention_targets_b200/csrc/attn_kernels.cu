@@ -1215,6 +1215,13 @@ __device__ __forceinline__ void attn_kernel_body(const AttnParams& p, uint8_t* s
     ctl.peer_abort = cluster_map(const_cast<int*>(reinterpret_cast<volatile int*>(abort_flag)),
                                  static_cast<uint32_t>(cta_rank<kCta>() ^ 1));
   const Phase ph{&p.sched, &p.tmap_q, &p.tmap_k, p.out, nullptr, nullptr, 0, nullptr};
+#if KVPOP_PDL_PASSES
+  // Launched as a programmatic dependent: the setup above (barriers, TMEM,
+  // tensor-map prefetch) overlapped the previous kernel's tail; every global
+  // read and write of the roles comes after this wait.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#endif
 
   if (warp == 0) {
     ProducerState st;
@@ -1366,13 +1373,15 @@ static cudaError_t launch_attn(const AttnParams& p, int sm_count, cudaStream_t s
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = L::ALLOC;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = KVPOP_PDL_PASSES ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, kern, p);
   }
 }

@@ -63,6 +63,12 @@ __global__ void __launch_bounds__(kKeepThreads, 2) keep_mask_kernel(const __grid
     return KVPOP_IN(i >= 0 && i < L && s >= 0 && s + i < p.total_tokens, p.dbg, DBG_KEEP, site);
   };
 
+#if KVPOP_PDL_PASSES
+  // A programmatic dependent of the kernel that wrote the scores: everything
+  // above overlapped its tail.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#endif
   // Every branch below depends only on (b, h): all CTAs of a cluster take it.
   if (L <= B) {
     for (int32_t i = r * kKeepThreads + tid; i < L; i += kKeepCluster * kKeepThreads)
@@ -202,13 +208,15 @@ static cudaError_t launch_keep_cluster(const KeepParams& p, int n_kv_heads, int 
   cfg.blockDim = dim3(kKeepThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = kC;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = KVPOP_PDL_PASSES ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, keep_mask_kernel<kC>, p);
 }
 

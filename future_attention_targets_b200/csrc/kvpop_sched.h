@@ -13,6 +13,12 @@ constexpr int kStreamRows = 256;     // rows of a streamed (B) tile = MMA N
 constexpr int kThreads = 576;        // producer warp + MMA warp + 16 softmax warps
 constexpr uint64_t kDefaultWaitNs = 1000000000ull;  // 1 s per on-chip wait
 
+// The standalone attention passes (CTA pairs) and the keep mask launch as
+// programmatic dependents of the kernel before them in the stream.
+#ifndef KVPOP_PDL_PASSES
+#define KVPOP_PDL_PASSES 1
+#endif
+
 // Work items ordered longest first.  An item is (level, sequence, head); all
 // items of one level cost (nearly) the same, so walking the levels from the
 // top gives a sorted list without sorting on the device.
