@@ -1454,6 +1454,10 @@ int target_split_groups() { return kColGroups; }
 // standalone pass; the pipelines have pass 1 write them next to lse).
 __global__ void __launch_bounds__(256) norm_rows_kernel(const float* __restrict__ lse, uint4* __restrict__ rows,
                                                         int64_t n, float inv_scale, int32_t* dbg) {
+#if KVPOP_PDL_PASSES
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // lse comes from the kernel before
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#endif
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
     if (KVPOP_IN(i >= 0 && i < n, dbg, DBG_NORM_ROWS, 1)) rows[i] = norm_row(__ldg(lse + i), inv_scale);
@@ -1462,8 +1466,16 @@ __global__ void __launch_bounds__(256) norm_rows_kernel(const float* __restrict_
 cudaError_t launch_norm_rows(const float* lse, void* rows, int64_t n, float inv_scale, int sm_count, int32_t* dbg,
                              cudaStream_t stream) {
   const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, static_cast<int64_t>(sm_count) * 8));
-  norm_rows_kernel<<<std::max(blocks, 1), 256, 0, stream>>>(lse, static_cast<uint4*>(rows), n, inv_scale, dbg);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(std::max(blocks, 1));
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = KVPOP_PDL_PASSES ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, norm_rows_kernel, lse, static_cast<uint4*>(rows), n, inv_scale, dbg);
 }
 
 // ------------------------------------------------------------------ bounded-wait self-test
