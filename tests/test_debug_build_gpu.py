@@ -160,3 +160,12 @@ def test_max_batch(word):
     q_bits, k_bits = random_qk(int(cu[-1]), 4, 2, 64, seed=22, gain=2.0)
     budgets = [max(2 + 16, int(L) // 2) for L in seqlens]
     all_entry_points(q_bits, k_bits, cu, 16, 2, budgets, 1.0 / 8.0, word, 23)
+
+
+def test_large_scores_exact_path(word):
+    """Scores large enough that pass 1 takes its exact path (scores recomputed from Q and K on CUDA
+    cores) for most rows: every index that path reads is checked too."""
+    seqlens = (700, 300)
+    q_bits, k_bits = random_qk(sum(seqlens), 4, 2, 128, seed=219, gain=6.0)
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    all_entry_points(q_bits, k_bits, cu, 16, 4, [16 + 4 + 37] * len(seqlens), 1.0 / math.sqrt(128), word, 220)
