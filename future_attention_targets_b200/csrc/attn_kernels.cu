@@ -630,8 +630,13 @@ __device__ __forceinline__ uint64_t f2_add_rm(uint64_t a, uint64_t b) {
 // same relative amount, against 2e-3; degree 4, 3.0e-6, is kept for the
 // KVPOP_LSE_DEG3 = 0 build of the row logsumexp),
 // and 2^n applied by adding n to the exponent field.  Inputs are clamped to
-// >= -126 so the exponent arithmetic cannot wrap; results below 2^-126 are
-// therefore at most 2^-125 instead of 0, far below any tolerance.
+// >= -126 so the exponent arithmetic cannot wrap below; results below 2^-126
+// are therefore at most 2^-125 instead of 0, far below any tolerance.  Where
+// an argument can be large (the row logsumexp, whose scores may lie far above
+// the running offset), it is also clamped to <= 127: the result is then at
+// least 2^127, so the tile's sum reaches the overflow check (>= 2^64) that
+// sends the row to its exact path, as MUFU's +inf does, instead of the
+// exponent field wrapping to a tiny value that would drop the term.
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
 constexpr float kP1 = 0x1.62d6c6p-1f, kP2 = 0x1.ee2450p-3f, kP3 = 0x1.abf868p-5f, kP4 = 0x1.b7f730p-7f;
 constexpr float kT1 = 0x1.63e658p-1f, kT2 = 0x1.d2378ap-3f, kT3 = 0x1.3baaa6p-4f;
@@ -640,7 +645,8 @@ template <bool kDeg3 = false>
 __device__ __forceinline__ uint64_t exp2_poly_pair(uint64_t y) {
   float y0, y1;
   f2_unpack(y, y0, y1);
-  const uint64_t yc = f2_pack(fmaxf(y0, -126.f), fmaxf(y1, -126.f));
+  // The row logsumexp's path (the only user): both clamps.
+  const uint64_t yc = f2_pack(fminf(fmaxf(y0, -126.f), 127.f), fminf(fmaxf(y1, -126.f), 127.f));
   const uint64_t t = f2_add_rm(yc, f2_pack(kRoundMagic, kRoundMagic));
   const uint64_t n = f2_add(t, f2_pack(-kRoundMagic, -kRoundMagic));
   const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), yc);
@@ -665,11 +671,20 @@ __device__ __forceinline__ uint64_t exp2_poly_pair(uint64_t y) {
 // 2^(c x) for a pair with the scale folded into the range reduction:
 // x is clamped so that c x >= -126, then t = rm(c x + 1.5 * 2^23) in one
 // fused multiply-add, n = t - 1.5 * 2^23 = floor(c x) (taken negated, in one
-// packed FMA), f = c x - n (exact).
-__device__ __forceinline__ uint64_t exp2_poly_pair_scaled(uint64_t x, uint64_t c2, float xmin) {
+// packed FMA), f = c x - n (exact).  kClampHigh: x is also clamped to
+// <= xmax (c xmax = 127; the row logsumexp at offset 0); the transposed pass
+// needs no upper clamp, its arguments are <= 0 up to rounding.
+template <bool kClampHigh>
+__device__ __forceinline__ uint64_t exp2_poly_pair_scaled(uint64_t x, uint64_t c2, float xmin, float xmax) {
   float x0, x1;
   f2_unpack(x, x0, x1);
-  const uint64_t xc = f2_pack(fmaxf(x0, xmin), fmaxf(x1, xmin));
+  x0 = fmaxf(x0, xmin);
+  x1 = fmaxf(x1, xmin);
+  if constexpr (kClampHigh) {
+    x0 = fminf(x0, xmax);
+    x1 = fminf(x1, xmax);
+  }
+  const uint64_t xc = f2_pack(x0, x1);
   uint64_t t;
   asm("fma.rm.ftz.f32x2 %0, %1, %2, %3;" : "=l"(t) : "l"(xc), "l"(c2), "l"(f2_pack(kRoundMagic, kRoundMagic)));
   const uint64_t neg_n = f2_fma(t, f2_pack(-1.f, -1.f), f2_pack(kRoundMagic, kRoundMagic));   // -n, exact
@@ -713,17 +728,19 @@ __device__ __forceinline__ constexpr bool poly_pair(int q) {
 // acc += exp2(x * c + nb) over one 16-column chunk (nb: one negated offset
 // for the whole chunk); of every 16 pairs kPoly go through the polynomial
 // (pairs kQ0 .. kQ0+7 of that pattern are this chunk's), the rest through
-// MUFU.  kBiasFree: nb is zero (pass 2), the scale is folded into the
-// polynomial's range reduction and x >= xmin keeps c x >= -126.
-template <int kPoly, bool kBiasFree, int kQ0, bool kDeg3 = kBiasFree>
+// MUFU.  kBiasFree: nb is zero, the scale is folded into the polynomial's
+// range reduction and xmin <= x (<= xmax with kClampHigh) keeps c x in
+// [-126, 127].
+template <int kPoly, bool kBiasFree, int kQ0, bool kDeg3 = kBiasFree, bool kClampHigh = false>
 __device__ __forceinline__ void chunk_exp_sum(const uint32_t (&r)[16], uint64_t c2, uint64_t nb, float xmin,
-                                              uint64_t (&acc)[4]) {
+                                              float xmax, uint64_t (&acc)[4]) {
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
     const uint64_t x = f2_pack(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
     uint64_t e;
     if (poly_pair<kPoly>(kQ0 + q)) {
-      e = kBiasFree ? exp2_poly_pair_scaled(x, c2, xmin) : exp2_poly_pair<kDeg3>(f2_fma(x, c2, nb));
+      e = kBiasFree ? exp2_poly_pair_scaled<kClampHigh>(x, c2, xmin, xmax)
+                    : exp2_poly_pair<kDeg3>(f2_fma(x, c2, nb));
     } else {
       e = exp2_mufu_pair(f2_fma(x, c2, nb));
     }
@@ -761,28 +778,29 @@ __device__ __forceinline__ float acc_total(uint64_t (&acc)[4]) {
 // once the last chunk's load has landed, before its exponentials: the
 // accumulator is free for the next MMA from then on.  kMasked: column m
 // counts iff lo <= m < hi.
-template <bool kMasked, int kPoly, bool kBiasFree = false, bool kDeg3 = kBiasFree, class Release>
+template <bool kMasked, int kPoly, bool kBiasFree = false, bool kDeg3 = kBiasFree, bool kClampHigh = false,
+          class Release>
 __device__ __forceinline__ float group_exp_sum(uint32_t taddr, uint64_t c2, uint64_t nb, int lo, int hi, float xmin,
-                                               Release&& release) {
+                                               float xmax, Release&& release) {
   uint32_t ra[16], rb[16];
   uint64_t acc[4] = {0, 0, 0, 0};
   tmem_load<16>(taddr, ra);
   tmem_load_wait<16>(ra);
   tmem_load<16>(taddr + 16, rb);
   if constexpr (kMasked) chunk_exp_sum_masked(ra, c2, nb, lo, hi, acc);
-  else chunk_exp_sum<kPoly, kBiasFree, 0, kDeg3>(ra, c2, nb, xmin, acc);
+  else chunk_exp_sum<kPoly, kBiasFree, 0, kDeg3, kClampHigh>(ra, c2, nb, xmin, xmax, acc);
   tmem_load_wait<16>(rb);
   tmem_load<16>(taddr + 32, ra);
   if constexpr (kMasked) chunk_exp_sum_masked(rb, c2, nb, lo - 16, hi - 16, acc);
-  else chunk_exp_sum<kPoly, kBiasFree, 8, kDeg3>(rb, c2, nb, xmin, acc);
+  else chunk_exp_sum<kPoly, kBiasFree, 8, kDeg3, kClampHigh>(rb, c2, nb, xmin, xmax, acc);
   tmem_load_wait<16>(ra);
   tmem_load<16>(taddr + 48, rb);
   if constexpr (kMasked) chunk_exp_sum_masked(ra, c2, nb, lo - 32, hi - 32, acc);
-  else chunk_exp_sum<kPoly, kBiasFree, 0, kDeg3>(ra, c2, nb, xmin, acc);
+  else chunk_exp_sum<kPoly, kBiasFree, 0, kDeg3, kClampHigh>(ra, c2, nb, xmin, xmax, acc);
   tmem_load_wait<16>(rb);
   release();
   if constexpr (kMasked) chunk_exp_sum_masked(rb, c2, nb, lo - 48, hi - 48, acc);
-  else chunk_exp_sum<kPoly, kBiasFree, 8, kDeg3>(rb, c2, nb, xmin, acc);
+  else chunk_exp_sum<kPoly, kBiasFree, 8, kDeg3, kClampHigh>(rb, c2, nb, xmin, xmax, acc);
   return acc_total(acc);
 }
 
@@ -857,6 +875,7 @@ __device__ void lse_softmax_phase(const AttnParams& p, const Phase& ph, uint8_t*
   const float kRebase = 4294967296.0f;          // 2^32: keep the running sum moderate
   const float kTiny = 5.421010862427522e-20f;   // 2^-64: smaller first-tile sums take the exact max
   const float xmin = -126.f / p.scale_log2;     // below it exp2(c x) < 2^-126: clamp for the polynomial
+  const float xmax = 127.f / p.scale_log2;      // above it the exponent field would wrap: clamp
   const LevelSchedule& sched = *ph.sched;
   const int32_t total = sched.total_items;
   for (int32_t k = 0; st.ok; ++k) {
@@ -908,14 +927,16 @@ __device__ void lse_softmax_phase(const AttnParams& p, const Phase& ph, uint8_t*
           // Rows whose running offset is still 0 (the common case) take the
           // transposed pass's scale-folded polynomial; chosen per warp.
           if (masked)
-            ts = group_exp_sum<true, 0>(taddr, c2, nb, 0, hi, 0.f, release);
+            ts = group_exp_sum<true, 0>(taddr, c2, nb, 0, hi, 0.f, 0.f, release);
           else if (__all_sync(0xffffffffu, off == 0.f))
-            ts = group_exp_sum<false, KVPOP_POLY16_LSE, true>(taddr, c2, nb, 0, kGroupCols, xmin, release);
+            ts = group_exp_sum<false, KVPOP_POLY16_LSE, true, true, true>(taddr, c2, nb, 0, kGroupCols, xmin, xmax,
+                                                                         release);
           else
-            ts = group_exp_sum<false, KVPOP_POLY16_LSE, false, true>(taddr, c2, nb, 0, kGroupCols, 0.f, release);
+            ts = group_exp_sum<false, KVPOP_POLY16_LSE, false, true>(taddr, c2, nb, 0, kGroupCols, 0.f, 0.f,
+                                                                    release);
 #else
-          ts = masked ? group_exp_sum<true, 0>(taddr, c2, nb, 0, hi, 0.f, release)
-                      : group_exp_sum<false, KVPOP_POLY16_LSE>(taddr, c2, nb, 0, kGroupCols, 0.f, release);
+          ts = masked ? group_exp_sum<true, 0>(taddr, c2, nb, 0, hi, 0.f, 0.f, release)
+                      : group_exp_sum<false, KVPOP_POLY16_LSE>(taddr, c2, nb, 0, kGroupCols, 0.f, 0.f, release);
 #endif
         }
         const bool rescale = !(ts < kBig) || (first && !(ts >= kTiny));
@@ -1064,9 +1085,9 @@ __device__ void target_softmax_phase(const AttnParams& p, const Phase& ph, uint8
         if (skip)
           release();
         else if (diag || ragged)
-          ts = group_exp_sum<true, 0>(taddr, c2, zero2, lo, hi, 0.f, release);
+          ts = group_exp_sum<true, 0>(taddr, c2, zero2, lo, hi, 0.f, 0.f, release);
         else
-          ts = group_exp_sum<false, KVPOP_POLY16_TARGET, true>(taddr, c2, zero2, 0, kGroupCols, xmin, release);
+          ts = group_exp_sum<false, KVPOP_POLY16_TARGET, true>(taddr, c2, zero2, 0, kGroupCols, xmin, 0.f, release);
         ++st.acc_cnt;
         const float yk = ts - comp;
         const float tk = run + yk;

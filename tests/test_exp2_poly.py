@@ -45,11 +45,14 @@ def test_kernel_coefficients_are_the_fit(degree):
     assert fit.fp32_horner_error(_kernel_coefficients(degree)) < SETS[degree][2]
 
 
-def _emulated_exp2(y, coeffs):
-    """The kernel's steps in float32: clamp, n = floor(y) (what adding 1.5 * 2^23
-    rounded toward minus infinity leaves), f = y - n, Horner from the highest
-    coefficient down to the pinned 1, then n added to the exponent bits."""
+def _emulated_exp2(y, coeffs, hi=None):
+    """The kernel's steps in float32: clamp (below at -126; above at `hi` where the
+    kernel clamps there too), n = floor(y) (what adding 1.5 * 2^23 rounded toward
+    minus infinity leaves), f = y - n, Horner from the highest coefficient down to
+    the pinned 1, then n added to the exponent bits."""
     y = np.maximum(y.astype(np.float32), np.float32(-126.0))
+    if hi is not None:
+        y = np.minimum(y, np.float32(hi))
     n = np.floor(y).astype(np.float32)
     f = (y - n).astype(np.float32)
     q = np.full_like(f, coeffs[-1])
@@ -57,7 +60,7 @@ def _emulated_exp2(y, coeffs):
         q = (q * f + ck).astype(np.float32)
     q = (q * f + np.float32(1.0)).astype(np.float32)
     bits = q.view(np.uint32).astype(np.int64) + (n.astype(np.int64) << 23)
-    return bits.astype(np.uint32).view(np.float32)
+    return (bits & 0xFFFFFFFF).astype(np.uint32).view(np.float32)   # the 32-bit add wraps
 
 
 @pytest.mark.parametrize("degree", [4, 3])
@@ -70,3 +73,21 @@ def test_emulated_exp2_error_bound(degree):
     # integers are exact: p(0) = 1
     k = -np.arange(0, 127, dtype=np.float32)
     np.testing.assert_array_equal(_emulated_exp2(k, coeffs), np.exp2(k.astype(np.float64)).astype(np.float32))
+
+
+@pytest.mark.parametrize("degree", [4, 3])
+def test_large_arguments_need_the_upper_clamp(degree):
+    """Above 127 the exponent add wraps: without the upper clamp 2^y of a large argument comes out tiny
+    (so a tile's sum would silently lose its largest terms); with it the result is at least 2^127, so the
+    sum reaches the row logsumexp's overflow check."""
+    coeffs = _kernel_coefficients(degree)
+    y = np.linspace(128.0, 300.0, 2000, dtype=np.float32)
+    wrapped = _emulated_exp2(y, coeffs)
+    with np.errstate(invalid="ignore"):   # some wrapped bit patterns are NaNs
+        reaches_check = np.isfinite(wrapped) & (np.abs(wrapped) >= np.float32(2.0 ** 64))
+    assert np.mean(reaches_check) < 0.5
+    clamped = _emulated_exp2(y, coeffs, hi=127.0).astype(np.float64)
+    assert np.all(np.isfinite(clamped)) and np.all(clamped >= 2.0 ** 127)
+    # below the clamp nothing changes
+    z = np.linspace(-126.0, 127.0, 5000, dtype=np.float32)
+    np.testing.assert_array_equal(_emulated_exp2(z, coeffs, hi=127.0), _emulated_exp2(z, coeffs))
