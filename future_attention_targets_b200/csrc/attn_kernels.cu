@@ -625,7 +625,7 @@ __device__ __forceinline__ uint64_t f2_add_rm(uint64_t a, uint64_t b) {
 // n = floor(y) (adding 1.5 * 2^23 rounded toward -inf leaves n in the low
 // mantissa bits), 2^f from a minimax polynomial with p(0) = 1 (coefficients
 // from fit_exp2_poly.py: degree 3, max relative error 8.6e-5 in fp32, on
-// 5 of every 16 pairs in both passes: a row's lse moves by at most that
+// 3 (row logsumexp) or 5 (transposed pass) of every 16 pairs: a row's lse moves by at most that
 // relative error of its polynomial terms' share, and a target by about the
 // same relative amount, against 2e-3; degree 4, 3.0e-6, is kept for the
 // KVPOP_LSE_DEG3 = 0 build of the row logsumexp),
@@ -709,12 +709,14 @@ __device__ __forceinline__ uint64_t exp2_mufu_pair(uint64_t y) {
 // Split between the exponent paths: pairs (of the 16 in a 32-column chunk)
 // evaluated by the polynomial, spread evenly over the chunk, and the row
 // logsumexp's polynomial degree (measured on B200 for each pass at the
-// Qwen3-8B 16k shape: degree 3 on 5 of 16 pairs beat degree 4 on 3 to 6).
+// Qwen3-8B 16k shape: degree 3 beat degree 4; pass 1, whose polynomial also
+// clamps from above, is fastest at 3 of 16 pairs (2 to 6 measured), pass 2
+// at 5).
 #ifndef KVPOP_LSE_DEG3
 #define KVPOP_LSE_DEG3 1
 #endif
 #ifndef KVPOP_POLY16_LSE
-#define KVPOP_POLY16_LSE 5
+#define KVPOP_POLY16_LSE 3
 #endif
 #ifndef KVPOP_POLY16_TARGET
 #define KVPOP_POLY16_TARGET 5

@@ -99,7 +99,7 @@ typedef struct {
  *   scale       softmax scale s (finite, > 0; 1/sqrt(head_dim) for the workloads)
  *   lse         device fp32 [n_q_heads, T], written for every (g, i)
  *   dev_status  device int32 or NULL; receives a nonzero code if a wait times out
- * Accuracy: the exponentials are fp32, 5 of every 16 from a degree-3
+ * Accuracy: the exponentials are fp32, 3 of every 16 from a degree-3
  * polynomial (relative error at most 8.6e-5), the rest from the hardware
  * exp2; sums in fp32.  |lse - exact| stays within 2e-4 (tested on every row
  * of the workloads and edge shapes); a target moves by about that relative

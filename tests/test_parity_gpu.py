@@ -22,7 +22,7 @@ from future_attention_targets_b200.workloads import WORKLOADS, make_inputs, rand
 pytestmark = pytest.mark.gpu
 
 TARGET_TOL = 2e-3       # elementwise relative error bound on the targets (floor 1e-3)
-LSE_TOL = 2e-4          # absolute error on the natural-log row logsumexp: a 5/16 share of
+LSE_TOL = 2e-4          # absolute error on the natural-log row logsumexp: a 3/16 share of
 #                        degree-3 polynomial exponentials (max relative error 8.6e-5) and fp32 sums
 
 

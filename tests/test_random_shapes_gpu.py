@@ -22,7 +22,7 @@ from future_attention_targets_b200.workloads import random_qk
 pytestmark = pytest.mark.gpu
 
 TARGET_TOL, LSE_TOL = 2e-3, 2e-4
-N_CASES = 16
+N_CASES = 40
 
 
 def dev(bits):
