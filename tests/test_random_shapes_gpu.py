@@ -2,7 +2,8 @@
 
 Each case draws (from a fixed seed) a batch of ragged sequences, a GQA shape, a head dimension, a
 window, sinks, budgets and an input gain (gains up to 6 send many of pass 1's tiles down its exact
-path), then checks:
+path); a few long cases (1-2 sequences of 2,000-6,000 tokens, gains 4 and 6) give rows many key tiles
+whose scores can jump far above the running offset.  Each case checks:
 - lse within 2e-4 and every target within 2e-3 (floor 1e-3) of the fp64 oracle;
 - the keep mask bit-exact against the oracle's mask from the same fp32 targets;
 - the prefix top-k thresholds bit-exact;
@@ -29,10 +30,14 @@ def dev(bits):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
 
 
+N_LONG = 4   # cases with fewer, longer sequences (many key tiles per row), large gains among them
+
+
 def draw(seed):
     rng = np.random.default_rng(1000 + seed)
-    nb = int(rng.integers(1, 6))
-    seqlens = [int(x) for x in rng.integers(0, 1300, nb)]
+    long_case = seed >= N_CASES
+    nb = int(rng.integers(1, 3 if long_case else 6))
+    seqlens = [int(x) for x in rng.integers(2000 if long_case else 0, 6000 if long_case else 1300, nb)]
     if sum(seqlens) == 0:
         seqlens[0] = 1
     hkv = int(rng.choice([1, 2, 4]))
@@ -41,11 +46,13 @@ def draw(seed):
     W = int(rng.choice([0, 1, 16, 100, 256, 700]))
     S = int(rng.integers(0, 5))
     budgets = [W + S + int(rng.integers(0, 400)) for _ in seqlens]
-    gain = float(rng.choice([0.5, 1.0, 2.0, 4.0, 6.0]))
+    gain = float(rng.choice([4.0, 6.0] if long_case else [0.5, 1.0, 2.0, 4.0, 6.0]))
+    if long_case:
+        hkv, G = 1, int(rng.choice([1, 2, 4]))
     return seqlens, hkv * G, hkv, d, W, S, budgets, gain
 
 
-@pytest.mark.parametrize("seed", range(N_CASES))
+@pytest.mark.parametrize("seed", range(N_CASES + N_LONG))
 def test_random_problem(seed):
     seqlens, hq, hkv, d, W, S, budgets, gain = draw(seed)
     T = sum(seqlens)
