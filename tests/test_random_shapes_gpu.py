@@ -8,7 +8,8 @@ whose scores can jump far above the running offset.  Each case checks:
 - the keep mask bit-exact against the oracle's mask from the same fp32 targets;
 - the prefix top-k thresholds bit-exact;
 - the compacted cache bit-exact and one decode step within 2e-3 (global reading) of the oracle;
-- the same results from the separate calls (row_lse, future_target, keep_mask) as from the pipeline.
+- the same results from the separate calls (row_lse, future_target, keep_mask) as from the pipeline,
+  and from the single launch the same lse bits, its targets against the oracle and its keep mask exact.
 """
 import math
 
@@ -70,6 +71,18 @@ def test_random_problem(seed):
     err = np.abs(tgt_h.astype(np.float64) - ref_t) / np.maximum(np.abs(ref_t), 1e-3)
     assert float(np.max(err, initial=0.0)) <= TARGET_TOL
     np.testing.assert_array_equal(keep_h, oracle.keep_mask(tgt_h, cu, W, S, budgets))
+
+    # The single launch (one CTA per SM, both passes): the same lse bits; its targets against the oracle
+    # like the pipeline's (its 128-key blocks align query tiles differently, so an element may take the
+    # polynomial in one path and MUFU in the other: they differ by up to the polynomial's 8.6e-5), and
+    # its own keep mask exact.
+    lf, tf, kf = B.future_targets_fused(q, k, cu, W, S, budgets, scale=scale, status=st)
+    B.check_status(st)
+    assert torch.equal(lf, lse)
+    tf_h = tf.cpu().numpy()
+    errf = np.abs(tf_h.astype(np.float64) - ref_t) / np.maximum(np.abs(ref_t), 1e-3)
+    assert float(np.max(errf, initial=0.0)) <= TARGET_TOL
+    np.testing.assert_array_equal(kf.cpu().numpy(), oracle.keep_mask(tf_h, cu, W, S, budgets))
 
     # The separate calls give the same bits as the pipeline.
     l2 = B.row_lse(q, k, cu, scale, status=st)
