@@ -103,7 +103,11 @@ typedef struct {
  * polynomial (relative error at most 8.6e-5), the rest from the hardware
  * exp2; sums in fp32.  |lse - exact| stays within 2e-4 (tested on every row
  * of the workloads and edge shapes); a target moves by about that relative
- * amount, well inside its 2e-3 bound.
+ * amount, well inside its 2e-3 bound.  A row whose scores lie far outside
+ * the fp32 range of the fast path (a first key tile summing outside
+ * [2^-64, 2^64) at offset 0, or a later tile past 2^64 above the running
+ * offset: score spreads beyond ~40-90 nats) takes an exact path for that
+ * tile, its scores recomputed on CUDA cores: slower, equally accurate.
  * Runs as CTA pairs: each M = 256 MMA is shared by two SMs.
  */
 KVPOP_API kvpop_status kvpop_row_lse(const void* q, const void* k, const int32_t* cu_seqlens,
